@@ -1,0 +1,218 @@
+"""Python face of the CommVQ CPU oracle -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the bench's CPU-baseline leg use
+this module. It loads ``libcommvq_oracle.so`` (plain C, built with
+``-ffp-contract=off``; see ``commvq_oracle.c`` for the definitions and their
+sources) and marshals numpy arrays. The codebook-fit driver below strings the C
+primitives together in the order the pages give (CommVQ machine review, "What
+carries the argument": codebooks fit by EM, R residual rounds).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import time
+from typing import Optional
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "commvq_oracle.c")
+LIB = os.path.join(HERE, "libcommvq_oracle.so")
+CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-std=c99"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (a test checker, not part of the product)."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, SRC, "-lm"])
+        os.replace(tmp, LIB)
+    return LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        _lib.oracle_encode.argtypes = [P, I64, I, I, I, I, P, P, P, P]
+        _lib.oracle_decode.argtypes = [P, I64, I, I, I, I, P, P]
+        _lib.oracle_scores_plain.argtypes = [P, P, I64, I64, I, ctypes.c_double, P]
+        _lib.oracle_scores_table.argtypes = [P, P, I64, I64, I, I, I, I, P, ctypes.c_double, P]
+        _lib.oracle_attend.argtypes = [P, P, P, P, I, I, I, I, ctypes.c_double, P, P]
+        _lib.oracle_em_step.argtypes = [P, I64, I, I, I, P, P, P]
+        _lib.oracle_values_hist.argtypes = [P, P, I64, I64, I, I, I, I, P, P, P]
+        for f in ("oracle_encode", "oracle_decode", "oracle_scores_plain", "oracle_scores_table",
+                  "oracle_attend", "oracle_em_step", "oracle_values_hist"):
+            getattr(_lib, f).restype = ctypes.c_int
+    return _lib
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with status {rc}")
+
+
+def encode(x: np.ndarray, cb: np.ndarray, want_residual: bool = False):
+    """Residual nearest-codeword codes of rows x[..., d] against cb [R, d/g, Nc', g].
+
+    Returns (codes [..., R, d/g] int32, near_tie_count[, residual [..., d] fp32])."""
+    R, G, Nc, g = cb.shape
+    d = G * g
+    lead = x.shape[:-1]
+    xf = _c(x.reshape(-1, d).astype(np.float32), np.float32)   # f16 widens exactly
+    n = xf.shape[0]
+    cbf = _c(cb, np.float32)
+    codes = np.empty((n, R, G), dtype=np.int32)
+    res = np.empty((n, d), dtype=np.float32) if want_residual else None
+    ties = ctypes.c_int64(0)
+    _check(lib().oracle_encode(_p(xf), n, d, g, R, Nc, _p(cbf), _p(codes), _p(res),
+                               ctypes.byref(ties)), "encode")
+    codes = codes.reshape(*lead, R, G)
+    if want_residual:
+        return codes, int(ties.value), res.reshape(*lead, d)
+    return codes, int(ties.value)
+
+
+def decode(codes: np.ndarray, cb: np.ndarray) -> np.ndarray:
+    """Sum of the selected codewords in fp64: codes [..., R, d/g] -> [..., d]."""
+    R, G, Nc, g = cb.shape
+    d = G * g
+    lead = codes.shape[:-2]
+    cc = _c(codes.reshape(-1, R, G), np.int32)
+    out = np.empty((cc.shape[0], d), dtype=np.float64)
+    _check(lib().oracle_decode(_p(cc), cc.shape[0], d, g, R, Nc, _p(_c(cb, np.float32)), _p(out)),
+           "decode")
+    return out.reshape(*lead, d)
+
+
+def scores_plain(q: np.ndarray, keys: np.ndarray, base: float) -> np.ndarray:
+    """Plain RoPE scores of one query [d] against decoded keys [T, d] at positions 0..T-1."""
+    qd = _c(q, np.float64)
+    kd = _c(keys, np.float64)
+    T, d = kd.shape
+    out = np.empty(T, dtype=np.float64)
+    _check(lib().oracle_scores_plain(_p(qd), _p(kd), d, T, d, float(base), _p(out)), "scores_plain")
+    return out
+
+
+def scores_table(q: np.ndarray, codes: np.ndarray, cb: np.ndarray, base: float) -> np.ndarray:
+    """Scores of one query [d] through the query x codebook table; codes [T, R, d/g]."""
+    R, G, Nc, g = cb.shape
+    d = G * g
+    cc = _c(codes, np.int32)
+    T = cc.shape[0]
+    out = np.empty(T, dtype=np.float64)
+    _check(lib().oracle_scores_table(_p(_c(q, np.float64)), _p(cc), R * G, T, d, g, R, Nc,
+                                     _p(_c(cb, np.float32)), float(base), _p(out)), "scores_table")
+    return out
+
+
+def values_hist(p: np.ndarray, codes: np.ndarray, cb: np.ndarray):
+    """Value output through histograms: weights p [T], codes [T, R, d/g].
+    Returns (o [d] fp64, H [R, d/g, Nc'] fp64)."""
+    R, G, Nc, g = cb.shape
+    d = G * g
+    cc = _c(codes, np.int32)
+    T = cc.shape[0]
+    o = np.empty(d, dtype=np.float64)
+    H = np.empty((R, G, Nc), dtype=np.float64)
+    _check(lib().oracle_values_hist(_p(_c(p, np.float64)), _p(cc), R * G, T, d, g, R, Nc,
+                                    _p(_c(cb, np.float32)), _p(H), _p(o)), "values_hist")
+    return o, H
+
+
+def bits_per_scalar(R: int, n_codes: int, g: int) -> float:
+    """Average stored bits per scalar, R * log2(Nc') / g (Eq. 21 as the review quotes it)."""
+    return R * float(np.log2(n_codes)) / g
+
+
+def reduction_vs_fp16(bits: float) -> float:
+    """Fraction of an FP16 cache saved at `bits` per scalar."""
+    return 1.0 - bits / 16.0
+
+
+def kv_cache_bytes(tokens: int, layers: int, kv_dim: int, batch: int, bits: float) -> float:
+    """Bytes of a K+V cache: 2 tensors x batch x tokens x layers x kv_dim x bits / 8."""
+    return 2.0 * batch * tokens * layers * kv_dim * bits / 8.0
+
+
+def attend(q: np.ndarray, khat: np.ndarray, vhat: np.ndarray, offsets: np.ndarray,
+           base: float):
+    """Plain decode attention on decoded caches. q [B, Hq, d]; khat/vhat [sum T, Hkv, d].
+    Returns (out [B, Hq, d] fp64, lse [B, Hq] fp64)."""
+    B, Hq, d = q.shape
+    Hkv = khat.shape[1]
+    out = np.empty((B, Hq, d), dtype=np.float64)
+    lse = np.empty((B, Hq), dtype=np.float64)
+    _check(lib().oracle_attend(_p(_c(q, np.float64)), _p(_c(khat, np.float64)),
+                               _p(_c(vhat, np.float64)), _p(_c(offsets, np.int64)), B, Hq, Hkv, d,
+                               float(base), _p(out), _p(lse)), "attend")
+    return out, lse
+
+
+def attend_codes(q: np.ndarray, k_codes: np.ndarray, v_codes: np.ndarray, offsets: np.ndarray,
+                 kcb: np.ndarray, vcb: np.ndarray, base: float):
+    """Decode attention straight from codes [sum T, Hkv, R, d/g]: decode, then attend."""
+    return attend(q, decode(k_codes, kcb), decode(v_codes, vcb), offsets, base)
+
+
+def em_step(rows: np.ndarray, cb_round: np.ndarray):
+    """One EM step on residual rows [N, d] for one round's codebook [d/g, Nc', g].
+    Returns (new codebook, codes [N, d/g], sse)."""
+    G, Nc, g = cb_round.shape
+    d = G * g
+    rf = _c(rows, np.float32)
+    N = rf.shape[0]
+    cb = _c(cb_round, np.float32).copy()
+    codes = np.empty((N, G), dtype=np.int32)
+    sse = ctypes.c_double(0.0)
+    _check(lib().oracle_em_step(_p(rf), N, d, g, Nc, _p(cb), _p(codes), ctypes.byref(sse)),
+           "em_step")
+    return cb, codes, float(sse.value)
+
+
+def forgy_init(rows: np.ndarray, idx: np.ndarray, g: int) -> np.ndarray:
+    """Round codebook [d/g, Nc', g] whose entry c of group j is sub-vector j of row idx[c]."""
+    N, d = rows.shape
+    G = d // g
+    return np.ascontiguousarray(rows[idx].reshape(len(idx), G, g).transpose(1, 0, 2),
+                                dtype=np.float32)
+
+
+def fit_codebook(rows: np.ndarray, R: int, g: int, n_codes: int, iters: int, init_indices):
+    """Sequential residual fit: for each round, Forgy init from that round's residual rows,
+    `iters` EM steps, then advance the residuals by one encoder round against the final
+    codebook. init_indices(r, N) -> row indices. Returns (cb [R, d/g, Nc', g], sse history)."""
+    res = _c(rows, np.float32).copy()
+    N, d = res.shape
+    rounds, hist = [], []
+    for r in range(R):
+        cb_r = forgy_init(res, init_indices(r, N), g)
+        h = []
+        for _ in range(iters):
+            cb_r, _, sse = em_step(res, cb_r)
+            h.append(sse)
+        hist.append(h)
+        rounds.append(cb_r)
+        _, _, res = encode(res, cb_r[None], want_residual=True)
+    return np.stack(rounds).astype(np.float32), hist
+
+
+def time_call(fn, *a, **kw):
+    t0 = time.perf_counter()
+    out = fn(*a, **kw)
+    return out, time.perf_counter() - t0

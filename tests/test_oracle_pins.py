@@ -1,0 +1,450 @@
+"""Pins for the CPU oracle: each test ties an oracle function to something other than
+itself -- numbers printed on the CommVQ pages, closed forms, invariants, exact brute
+force on tiny inputs, or a library routine (torch's scaled_dot_product_attention).
+
+Runs on CPU only.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from decode_attention_commvq_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "bits_per_scalar.txt")
+
+
+# ----------------------------------------------------------------------------------------
+# exact fp32 arithmetic for brute force (independent of the C oracle)
+
+def round_f32(x: Fraction) -> np.float32:
+    """Correctly rounded (nearest, ties to even) float32 of an exact rational."""
+    if x == 0:
+        return np.float32(0.0)
+    sign = -1 if x < 0 else 1
+    a = abs(x)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    e = max(e, -126)                      # subnormals share the 2^-149 quantum
+    quantum = Fraction(2) ** (e - 23)
+    scaled = a / quantum
+    n = scaled.numerator // scaled.denominator
+    rem = scaled - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    val = n * quantum
+    if val >= Fraction(2) ** 128:
+        return np.float32(sign * np.inf)
+    return np.float32(sign * float(val))
+
+
+def fmaf_exact(a, b, c) -> np.float32:
+    return round_f32(Fraction(float(a)) * Fraction(float(b)) + Fraction(float(c)))
+
+
+def brute_nearest(res: np.ndarray, sub_cb: np.ndarray):
+    """Distances by the definition (fp32 subtract, exactly rounded fused multiply-add in
+    index order); first strict minimum."""
+    dists = []
+    for c in range(sub_cb.shape[0]):
+        dist = np.float32(0.0)
+        for k in range(res.shape[0]):
+            e = np.float32(res[k] - sub_cb[c, k])
+            dist = fmaf_exact(e, e, dist)
+        dists.append(dist)
+    best = 0
+    for c in range(1, len(dists)):
+        if dists[c] < dists[best]:
+            best = c
+    return best, dists
+
+
+def brute_encode(x: np.ndarray, cb: np.ndarray):
+    R, G, Nc, g = cb.shape
+    N = x.shape[0]
+    codes = np.zeros((N, R, G), dtype=np.int32)
+    for n in range(N):
+        for j in range(G):
+            res = x[n, j * g:(j + 1) * g].astype(np.float32).copy()
+            for r in range(R):
+                c, _ = brute_nearest(res, cb[r, j])
+                codes[n, r, j] = c
+                res = (res - cb[r, j, c]).astype(np.float32)
+    return codes
+
+
+# ----------------------------------------------------------------------------------------
+# bit-rate arithmetic against the pages' printed figures
+
+def _golden_rows():
+    rows = []
+    with open(GOLDEN) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            rows.append(line.split())
+    return rows
+
+
+def test_bits_and_sizes_match_printed_figures():
+    rows = _golden_rows()
+    assert len(rows) >= 12
+    for r in rows:
+        kind = r[0]
+        if kind == "bits":
+            R, Nc, g, want = int(r[1]), int(r[2]), int(r[3]), float(r[4])
+            assert O.bits_per_scalar(R, Nc, g) == pytest.approx(want, abs=1e-12), r
+        elif kind == "reduction":
+            bits, want = float(r[1]), float(r[2])
+            assert O.reduction_vs_fp16(bits) == pytest.approx(want, abs=1e-12), r
+        elif kind == "cache_bytes":
+            tokens, layers, kv_dim, batch, bits = map(float, r[1:6])
+            want, tol = float(r[6]), float(r[7])
+            got = O.kv_cache_bytes(int(tokens), int(layers), int(kv_dim), int(batch), bits)
+            assert abs(got - want) <= tol * want, (r, got)
+        else:
+            raise AssertionError(r)
+
+
+def test_workload_bit_rates():
+    w = synth.WORKLOADS
+    assert O.bits_per_scalar(w[0].R, w[0].n_codes, w[0].g) == 0.5
+    assert O.bits_per_scalar(w[1].R, w[1].n_codes, w[1].g) == 2.0
+    assert O.bits_per_scalar(w[2].R, w[2].n_codes, w[2].g) == 1.0
+    assert O.reduction_vs_fp16(O.bits_per_scalar(2, 256, 8)) == 0.875
+    assert O.reduction_vs_fp16(O.bits_per_scalar(1, 256, 8)) == 0.9375
+
+
+# ----------------------------------------------------------------------------------------
+# commutation (review, "What carries the argument": R_m C = C R_m, Property 1)
+
+def _rot(phi):
+    return np.array([[math.cos(phi), -math.sin(phi)], [math.sin(phi), math.cos(phi)]])
+
+
+def test_commutation_identity():
+    rng = np.random.default_rng(11)
+    d, base = 128, 500000.0
+    for _ in range(200):
+        x, y = rng.standard_normal(2)
+        C = np.array([[x, y], [-y, x]])
+        m = int(rng.integers(0, 2 ** 17))
+        p = int(rng.integers(0, d // 2))
+        Rm = _rot(m * base ** (-2.0 * p / d))
+        assert np.abs(Rm @ C - C @ Rm).max() <= 1e-12
+
+
+def test_stored_pair_block_reorders_score():
+    """q . R_m (C e1) == (q^T C) . (R_m e1) for C = [[a, -b], [b, a]]: the reorder the table uses."""
+    rng = np.random.default_rng(12)
+    for _ in range(100):
+        a, b, q0, q1 = rng.standard_normal(4)
+        phi = rng.uniform(-1e3, 1e3)
+        C = np.array([[a, -b], [b, a]])
+        q = np.array([q0, q1])
+        lhs = q @ (_rot(phi) @ C @ np.array([1.0, 0.0]))
+        rhs = (q @ C) @ (_rot(phi) @ np.array([1.0, 0.0]))
+        assert abs(lhs - rhs) <= 1e-12 * (1 + abs(lhs))
+        # C e1 is the stored pair itself
+        assert np.allclose(C @ np.array([1.0, 0.0]), [a, b])
+
+
+# ----------------------------------------------------------------------------------------
+# RoPE closed forms: theta_0 = 1; for d = 128, base 1e4: theta_16 = 0.1, theta_32 = 0.01,
+# theta_48 = 0.001; direction: key (1, 0) rotates to (cos, sin).
+
+@pytest.mark.parametrize("p,theta", [(0, 1.0), (16, 0.1), (32, 0.01), (48, 0.001)])
+def test_rope_closed_forms(p, theta):
+    d, base, T = 128, 10000.0, 300
+    keys = np.zeros((T, d))
+    keys[:, 2 * p] = 1.0
+    qa = np.zeros(d); qa[2 * p] = 1.0
+    qb = np.zeros(d); qb[2 * p + 1] = 1.0
+    t = np.arange(T)
+    sa = O.scores_plain(qa, keys, base)
+    sb = O.scores_plain(qb, keys, base)
+    assert np.allclose(sa, np.cos(t * theta) / math.sqrt(d), atol=1e-12, rtol=0)
+    assert np.allclose(sb, np.sin(t * theta) / math.sqrt(d), atol=1e-12, rtol=0)
+
+
+def test_rope_position_zero_is_plain_dot():
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal(128)
+    k = rng.standard_normal((1, 128))
+    s = O.scores_plain(q, k, 500000.0)
+    assert s[0] == pytest.approx(float(q @ k[0]) / math.sqrt(128), rel=1e-14)
+
+
+# ----------------------------------------------------------------------------------------
+# table path (query x codebook table, rotation after) == decompress-then-RoPE
+
+@pytest.mark.parametrize("wi", [0, 1])
+def test_table_scores_equal_plain_scores(wi):
+    w = synth.WORKLOADS[wi]
+    T = 256 if wi == 0 else 1500
+    kcb = synth.normal_codebook(w, key=True)
+    codes = synth.uniform_codes(w.with_(kv_heads=1), key=True, total_T=T)[:, 0]
+    q = synth.as_f32(synth.queries(w), w.q_dtype)[0, 0].astype(np.float64)
+    khat = O.decode(codes, kcb)
+    s_plain = O.scores_plain(q, khat, w.rope_base)
+    s_tab = O.scores_table(q, codes, kcb, w.rope_base)
+    assert np.abs(s_plain - s_tab).max() <= 1e-10 * np.abs(s_plain).max()
+
+
+def test_table_scores_at_long_positions():
+    w = synth.WORKLOADS[2]
+    kcb = synth.normal_codebook(w, key=True)
+    rng = np.random.default_rng(5)
+    T = 131072
+    codes = rng.integers(0, w.n_codes, size=(T, w.R, w.groups)).astype(np.int32)
+    q = rng.standard_normal(w.d)
+    sel = slice(T - 300, T)
+    khat = O.decode(codes, kcb)
+    s_plain = O.scores_plain(q, khat, w.rope_base)[sel]
+    s_tab = O.scores_table(q, codes, kcb, w.rope_base)[sel]
+    assert np.abs(s_plain - s_tab).max() <= 1e-10 * np.abs(s_plain).max()
+
+
+# ----------------------------------------------------------------------------------------
+# value histograms (softmax weights times codes before the codebook multiply)
+
+def test_value_histogram_path():
+    w = synth.WORKLOADS[1]
+    vcb = synth.normal_codebook(w, key=False)
+    rng = np.random.default_rng(8)
+    T = 700
+    codes = rng.integers(0, w.n_codes, size=(T, w.R, w.groups)).astype(np.int32)
+    s = rng.standard_normal(T) * 3
+    p = np.exp(s - s.max()); p /= p.sum()
+    o, H = O.values_hist(p, codes, vcb)
+    vhat = O.decode(codes, vcb)
+    ref = (p[:, None] * vhat).sum(0)
+    assert np.abs(o - ref).max() <= 1e-12 * np.abs(ref).max()
+    assert np.allclose(H.sum(-1), 1.0, atol=1e-12)
+    # zero-weight codes contribute nothing: a histogram bin is empty iff no token uses it
+    used = np.zeros((w.R, w.groups, w.n_codes), dtype=bool)
+    for r in range(w.R):
+        for j in range(w.groups):
+            used[r, j, np.unique(codes[:, r, j])] = True
+    assert np.all((H > 0) == used)
+
+
+# ----------------------------------------------------------------------------------------
+# attention: library reduction, special cases, GQA mapping, ragged batches
+
+def _rope_complex(k: np.ndarray, base: float) -> np.ndarray:
+    """Rotate rows k [T, d] at positions 0..T-1 as complex numbers z_p = k_2p + i k_2p+1."""
+    T, d = k.shape
+    z = k[:, 0::2] + 1j * k[:, 1::2]
+    freq = base ** (-np.arange(0, d, 2) / d)
+    z = z * np.exp(1j * np.outer(np.arange(T), freq))
+    out = np.empty_like(k)
+    out[:, 0::2] = z.real
+    out[:, 1::2] = z.imag
+    return out
+
+
+def test_attend_equals_torch_sdpa_on_rotated_cache():
+    rng = np.random.default_rng(21)
+    B, Hq, Hkv, d, T, base = 1, 4, 2, 128, 333, 500000.0
+    q = rng.standard_normal((B, Hq, d))
+    kh = rng.standard_normal((T, Hkv, d)) * 2
+    vh = rng.standard_normal((T, Hkv, d))
+    out, lse = O.attend(q, kh, vh, np.array([0, T]), base)
+    kr = np.stack([_rope_complex(kh[:, h], base) for h in range(Hkv)])          # [Hkv, T, d]
+    K = torch.from_numpy(np.repeat(kr, Hq // Hkv, axis=0))[None]                # [1, Hq, T, d]
+    V = torch.from_numpy(np.repeat(vh.transpose(1, 0, 2), Hq // Hkv, axis=0))[None]
+    Q = torch.from_numpy(q)[:, :, None, :]                                       # [1, Hq, 1, d]
+    ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V)[:, :, 0].numpy()
+    assert np.abs(out - ref).max() <= 1e-12 * np.abs(ref).max()
+    s = (Q @ K.transpose(-1, -2))[:, :, 0] / math.sqrt(d)
+    assert np.allclose(lse, torch.logsumexp(s, -1).numpy(), rtol=0, atol=1e-12)
+
+
+def test_attend_single_token_returns_its_value():
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((1, 2, 128))
+    kh = rng.standard_normal((1, 1, 128))
+    vh = rng.standard_normal((1, 1, 128))
+    out, lse = O.attend(q, kh, vh, np.array([0, 1]), 10000.0)
+    assert np.array_equal(out[0, 0], vh[0, 0]) and np.array_equal(out[0, 1], vh[0, 0])
+    assert lse[0, 0] == pytest.approx(float(q[0, 0] @ kh[0, 0]) / math.sqrt(128), rel=1e-14)
+
+
+def test_attend_zero_query_is_mean_of_values():
+    rng = np.random.default_rng(6)
+    T = 517
+    kh = rng.standard_normal((T, 1, 128))
+    vh = rng.standard_normal((T, 1, 128))
+    out, lse = O.attend(np.zeros((1, 1, 128)), kh, vh, np.array([0, T]), 500000.0)
+    assert np.abs(out[0, 0] - vh[:, 0].mean(0)).max() <= 1e-13
+    assert lse[0, 0] == pytest.approx(math.log(T), rel=1e-14)
+
+
+def test_attend_empty_sequence():
+    out, lse = O.attend(np.ones((2, 1, 128)), np.ones((3, 1, 128)), np.ones((3, 1, 128)),
+                        np.array([0, 0, 3]), 10000.0)
+    assert np.all(out[0] == 0) and lse[0, 0] == -np.inf
+    assert np.allclose(out[1, 0], 1.0)
+
+
+def test_attend_gqa_and_ragged_batch_mapping():
+    rng = np.random.default_rng(9)
+    Hq, Hkv, d, base = 4, 2, 128, 500000.0
+    L = [50, 80]
+    offs = np.array([0, 50, 130])
+    q = rng.standard_normal((2, Hq, d))
+    kh = rng.standard_normal((130, Hkv, d))
+    vh = rng.standard_normal((130, Hkv, d))
+    out, lse = O.attend(q, kh, vh, offs, base)
+    for b in range(2):
+        sl = slice(offs[b], offs[b + 1])
+        for h in range(Hq):
+            kvh = h // (Hq // Hkv)
+            o1, l1 = O.attend(q[b:b + 1, h:h + 1], kh[sl, kvh:kvh + 1], vh[sl, kvh:kvh + 1],
+                              np.array([0, L[b]]), base)
+            assert np.array_equal(o1[0, 0], out[b, h])
+            assert l1[0, 0] == lse[b, h]
+
+
+# ----------------------------------------------------------------------------------------
+# encoder: exact brute force, planted codes, ties
+
+def test_encoder_matches_exact_brute_force():
+    rng = np.random.default_rng(31)
+    R, G, Nc, g = 2, 2, 7, 8
+    cb = rng.standard_normal((R, G, Nc, g)).astype(np.float32)
+    x = rng.standard_normal((9, G * g)).astype(np.float32)
+    codes, _ = O.encode(x, cb)
+    assert np.array_equal(codes, brute_encode(x, cb))
+
+
+def test_encoder_fp16_rows_brute_force():
+    w = synth.WORKLOADS[1]
+    rows = synth.kv_rows(w, key=True, T=2)[:, :2].reshape(-1, w.d)        # f16, outliers
+    cb = synth.normal_codebook(w.with_(n_codes=9), key=True)[:, :, :9] * 3
+    cb = cb.astype(np.float32)
+    x = rows.astype(np.float32)
+    sub = x[:, :16]
+    codes, _ = O.encode(sub, cb[:, :2])
+    assert np.array_equal(codes, brute_encode(sub, cb[:, :2]))
+
+
+def test_encoder_recovers_planted_codes():
+    rng = np.random.default_rng(32)
+    R, G, Nc, g = 2, 16, 256, 8
+    cb = np.empty((R, G, Nc, g), dtype=np.float32)
+    cb[0] = rng.standard_normal((G, Nc, g)) * 100.0
+    cb[1] = rng.standard_normal((G, Nc, g)) * 1.0
+    truth = rng.integers(0, Nc, size=(64, R, G))
+    x = np.zeros((64, G * g), dtype=np.float32)
+    for n in range(64):
+        for j in range(G):
+            x[n, j * g:(j + 1) * g] = cb[0, j, truth[n, 0, j]] + cb[1, j, truth[n, 1, j]]
+    codes, _ = O.encode(x, cb)
+    assert np.array_equal(codes, truth)
+    dec = O.decode(codes, cb)
+    assert np.abs(dec - x).max() <= 1e-4 * np.abs(x).max()
+
+
+def test_encoder_ties_go_to_lowest_index_and_are_counted():
+    g = 8
+    cb = np.zeros((1, 1, 4, g), dtype=np.float32)
+    cb[0, 0, 1] = 1.0
+    cb[0, 0, 3] = 1.0          # duplicate of entry 1
+    cb[0, 0, 0] = -5.0
+    cb[0, 0, 2] = 7.0
+    x = np.full((1, g), 1.0, dtype=np.float32)
+    codes, ties = O.encode(x, cb)
+    assert codes[0, 0, 0] == 1 and ties == 1
+    x2 = np.full((1, g), -5.0, dtype=np.float32)
+    codes, ties = O.encode(x2, cb)
+    assert codes[0, 0, 0] == 0 and ties == 0
+
+
+def test_encoder_residual_output():
+    rng = np.random.default_rng(33)
+    cb = rng.standard_normal((2, 2, 5, 8)).astype(np.float32)
+    x = rng.standard_normal((6, 16)).astype(np.float32)
+    codes, _, res = O.encode(x, cb, want_residual=True)
+    for n in range(6):
+        for j in range(2):
+            r_ = x[n, j * 8:(j + 1) * 8].copy()
+            for r in range(2):
+                r_ = (r_ - cb[r, j, codes[n, r, j]]).astype(np.float32)
+            assert np.array_equal(res[n, j * 8:(j + 1) * 8], r_)
+
+
+# ----------------------------------------------------------------------------------------
+# EM step: brute-force assignment and means, SSE bit-exact, Lloyd monotonicity, fixed points
+
+def test_em_step_brute_force():
+    rng = np.random.default_rng(41)
+    N, G, Nc, g = 40, 2, 6, 8
+    rows = rng.standard_normal((N, G * g)).astype(np.float32)
+    cb0 = rng.standard_normal((G, Nc, g)).astype(np.float32)
+    cb1, codes, sse = O.em_step(rows, cb0)
+    want_sse = 0.0
+    sums = np.zeros((G, Nc, g)); cnt = np.zeros((G, Nc), dtype=np.int64)
+    for n in range(N):
+        for j in range(G):
+            c, dists = brute_nearest(rows[n, j * g:(j + 1) * g], cb0[j])
+            assert codes[n, j] == c
+            want_sse += float(dists[c])
+            cnt[j, c] += 1
+            for k in range(g):
+                sums[j, c, k] += float(rows[n, j * g + k])
+    assert sse == want_sse
+    for j in range(G):
+        for c in range(Nc):
+            if cnt[j, c] == 0:
+                assert np.array_equal(cb1[j, c], cb0[j, c])
+            else:
+                assert np.array_equal(cb1[j, c], (sums[j, c] / cnt[j, c]).astype(np.float32))
+
+
+def test_em_sse_non_increasing_and_fit_driver():
+    w = synth.WORKLOADS[1].with_(em_rows=512)
+    rows = synth.fit_rows(w, key=True)
+    cb, hist = O.fit_codebook(rows, R=2, g=w.g, n_codes=32, iters=6,
+                              init_indices=lambda r, N: synth.forgy_indices(w.with_(n_codes=32),
+                                                                            True, r, N))
+    for h in hist:
+        for a, b in zip(h, h[1:]):
+            assert b <= a * (1 + 1e-9)
+    assert hist[1][0] < hist[0][-1]       # the second round fits what the first left over
+    assert cb.shape == (2, 16, 32, 8)
+
+
+def test_em_exact_fixed_point_when_entries_cover_rows():
+    rng = np.random.default_rng(42)
+    Nc, g = 12, 8
+    distinct = rng.standard_normal((Nc, g)).astype(np.float32)
+    labels = rng.integers(0, Nc, size=200)
+    rows = distinct[labels]                                   # d = g, one group
+    cb = distinct[rng.permutation(Nc)][None]
+    cb1, codes, sse = O.em_step(rows, cb)
+    assert sse == 0.0
+    assert np.array_equal(cb1, cb)
+
+
+def test_em_separated_clusters_converge_to_means():
+    rng = np.random.default_rng(43)
+    Nc, g, N = 8, 8, 400
+    centers = rng.standard_normal((Nc, g)) * 50
+    labels = rng.integers(0, Nc, size=N)
+    rows = (centers[labels] + rng.standard_normal((N, g))).astype(np.float32)
+    init = np.stack([rows[np.nonzero(labels == c)[0][0]] for c in range(Nc)])[None]
+    cb = init.astype(np.float32)
+    for _ in range(3):
+        cb, codes, _ = O.em_step(rows, cb)
+    assert np.array_equal(codes[:, 0], labels)
+    for c in range(Nc):
+        mean = rows[labels == c].astype(np.float64).mean(0)
+        assert np.allclose(cb[0, c], mean, rtol=0, atol=1e-5)
