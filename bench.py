@@ -1,0 +1,451 @@
+"""Decode-attention benchmark over a CommVQ-compressed KV cache on B200.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME]
+
+One step is one commvq_attend_decode over the whole workload (all heads of one layer,
+every cached position). The default workload is the LLaMA-3.1-8B-shaped 2-bit layer:
+batch 1, 32 query / 8 KV heads, d = 128, T = 32768, R = 2, g = 8, Nc' = 256. Inputs are
+seeded synthetic rows, codebooks fit on the GPU by the library's EM step, codes made by
+the library's encoder. Under torchrun each rank runs its own replica (weak scaling; the
+path has no exchange step); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attention context-tokens/s and compressed-KV HBM GB/s vs B200 peak (1 GPU)"
+UNIT = "context-tokens/s"
+DEFAULT_WORKLOAD = "llama8b_2bit_T32768"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--algo", type=int, default=0)
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-heads", type=int, default=8, help="query heads in the oracle sample")
+    return ap.parse_args()
+
+
+def workload(name):
+    from decode_attention_commvq_b200 import synth
+    for w in synth.WORKLOADS:
+        if w.name == name:
+            return w
+    raise SystemExit(f"unknown workload {name}; known: {[w.name for w in synth.WORKLOADS]}")
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha():
+    src = os.path.join(ROOT, "decode_attention_commvq_b200", "csrc", "attend_table.cu")
+    with open(src, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload_name: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on this exact source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload_name)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return float(e["dram_bytes_per_launch"])
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index: int, bus_id: str | None):
+        self.sel = bus_id if bus_id else str(device_index)
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.sel, f"--query-gpu=timestamp,{self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.flush()
+        with open(self.f.name) as f:
+            lines = [l.strip() for l in f if l.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        for l in lines:
+            parts = [x.strip() for x in l.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                s, m = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            sm.append(s)
+            mx = m
+            for name, val in zip(self.NAMES, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------
+# our arm
+
+def setup_inputs(w, dev, torch, api, fit):
+    """Codebooks (GPU EM fit), encoded K/V cache, queries, offsets, all on the device."""
+    from decode_attention_commvq_b200 import synth
+    cfg = api.Config(d=w.d, g=w.g, R=w.R, n_codes=w.n_codes, q_heads=w.q_heads,
+                     kv_heads=w.kv_heads, rope_base=w.rope_base)
+    cbs = []
+    for key in (True, False):
+        if w.codebook == "normal":
+            cbs.append(torch.from_numpy(synth.normal_codebook(w, key)).to(dev))
+        else:
+            rows = torch.from_numpy(synth.fit_rows(w, key)).to(dev)
+            cbs.append(fit.fit_codebook(rows, w.R, w.n_codes, w.em_iters,
+                                        lambda r, N, key=key: synth.forgy_indices(w, key, r, N)))
+    kcb, vcb = cbs
+    codes = []
+    for key, cb in ((True, kcb), (False, vcb)):
+        parts = []
+        L = w.lengths()
+        for b in range(w.batch):
+            x = torch.from_numpy(synth.kv_rows(w, key, int(L[b]), sub=b)).to(dev)
+            parts.append(api.encode(cfg, x, cb))
+            del x
+        codes.append(torch.cat(parts, 0).contiguous())
+    q_np = synth.queries(w)
+    if w.q_dtype == "bf16":
+        q = torch.from_numpy(q_np.view(np.int16)).to(dev).view(torch.bfloat16)
+    else:
+        q = torch.from_numpy(q_np.astype(np.float32)).to(dev)
+    offs = torch.from_numpy(w.offsets()).to(dev)
+    return cfg, kcb, vcb, codes[0], codes[1], q, offs
+
+
+def run_ours(args, w, rank, world, dev):
+    import torch
+    import torch.distributed as dist
+    from decode_attention_commvq_b200 import api, fit, synth
+
+    torch.manual_seed(0)
+    cfg, kcb, vcb, kc, vc, q, offs = setup_inputs(w, dev, torch, api, fit)
+    L = w.lengths()
+    total_T = int(L.sum())
+    max_T = int(L.max())
+    code_bytes = kc.numel() + vc.numel()
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    n_copies = max(1, math.ceil(3 * l2 / code_bytes))
+    kcs = [kc] + [kc.clone() for _ in range(n_copies - 1)]
+    vcs = [vc] + [vc.clone() for _ in range(n_copies - 1)]
+    ws = api.attend_workspace(cfg, w.batch, max_T, dev, args.algo, args.splits)
+    out = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.batch, w.q_heads), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    K, W = args.steps, args.warmup
+
+    def step(i, events=None):
+        api.attend_decode(cfg, q, kcs[i % n_copies], vcs[i % n_copies], offs, max_T, kcb, vcb,
+                          out=out, lse=lse, workspace=ws, algo=args.algo, splits=args.splits,
+                          stream=stream, main_events=events)
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    with torch.cuda.stream(stream):
+        for a, b in evs:            # materialise the CUDA events before capture
+            a.record(stream)
+            b.record(stream)
+        for i in range(W):
+            step(i)
+    torch.cuda.synchronize(dev)
+    assert api.workspace_error(ws, stream) == 0
+
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(K):
+            step(W + i, evs[i])
+    graph.replay()                   # one untimed replay (the graph's own upload)
+    torch.cuda.synchronize(dev)
+
+    bus = None
+    try:
+        bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    except AttributeError:
+        pass
+    clocks = ClockSampler(dev.index or 0, bus)
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    graph.replay()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    kern_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    del graph
+
+    # ---- e2e: one decode step through the API with host buffers -----------------------
+    e2e = run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, ws, stream, dev, torch,
+                  api, synth, world, dist)
+
+    value = world * K * total_T / (ms_max / 1e3)
+    peak, peak_kind = measured_peaks()
+    achieved = code_bytes / (kern_ms / 1e3) / 1e9
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
+                   "d": w.d, "T": total_T, "R": w.R, "g": w.g, "n_codes": w.n_codes,
+                   "q_dtype": w.q_dtype, "parallelism": f"replicas{world}",
+                   "algo": args.algo, "splits": args.splits,
+                   "l2_defence": f"rotating {n_copies} cache copies ({n_copies * code_bytes / 2**20:.0f} MiB "
+                                 f">= 3x L2 {l2 / 2**20:.0f} MiB)",
+                   "timing": "K steps in one CUDA graph, CUDA events on the launch stream"},
+        "compressed_cache_gbs": code_bytes * K / (ms_max / 1e3) / 1e9 * 1.0 / world * world,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
+                     "kernel": "attend_table_kernel", "algorithmic_bytes_per_launch": code_bytes,
+                     "kernel_ms_mean": kern_ms,
+                     "traffic": recorded_traffic("attend_table_kernel", w.name)},
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+    }
+    return result
+
+
+def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, ws, stream, dev, torch, api,
+            synth, world, dist):
+    """Per step: pinned host -> device copy of the step's query and the new position's K/V
+    rows, encode of the new position into the cache (position T-1 of sequence 0), decode
+    attention, device -> host copy of the output."""
+    K, W = args.steps, args.warmup
+    n_copies = len(kcs)
+    q_h = torch.from_numpy(synth.queries(w).view(np.int16) if w.q_dtype == "bf16"
+                           else synth.queries(w).astype(np.float32)).pin_memory()
+    kv_new = np.stack([synth.kv_rows(w, True, 1, sub=1000, dtype="f16"),
+                       synth.kv_rows(w, False, 1, sub=1000, dtype="f16")])   # [2, 1, Hkv, d]
+    kv_h = torch.from_numpy(kv_new).pin_memory()
+    out_h = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32).pin_memory()
+    q_d = torch.empty(q_h.shape, dtype=q_h.dtype, device=dev)
+    kv_d = torch.empty(kv_h.shape, dtype=kv_h.dtype, device=dev)
+    out_d = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32, device=dev)
+    last = int(w.offsets()[1]) - 1
+    qv = q_d.view(torch.bfloat16) if w.q_dtype == "bf16" else q_d
+
+    def step(i):
+        kc, vc = kcs[i % n_copies], vcs[i % n_copies]
+        q_d.copy_(q_h, non_blocking=True)
+        kv_d.copy_(kv_h, non_blocking=True)
+        api.encode(cfg, kv_d[0], kcb, codes=kc[last:last + 1], stream=stream)
+        api.encode(cfg, kv_d[1], vcb, codes=vc[last:last + 1], stream=stream)
+        api.attend_decode(cfg, qv, kc, vc, offs, max_T, kcb, vcb, out=out_d, workspace=ws,
+                          want_lse=False, stream=stream, algo=args.algo, splits=args.splits)
+        out_h.copy_(out_d, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            step(i)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(K):
+                step(W + i)
+        graph.replay()
+        torch.cuda.synchronize(dev)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        t0.record(stream)
+        graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    del graph
+    return {"value": world * K * total_T / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(q_h.numel() * q_h.element_size() + kv_h.numel() * kv_h.element_size()),
+            "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()),
+            "ms_per_step": ms / K,
+            "note": "q + new position's K/V rows in, encode + attend, output out; one CUDA graph of K steps"}
+
+
+# ---------------------------------------------------------------------------------------
+# the oracle (CPU baseline and the reference arm)
+
+def oracle_sample(w, n_heads):
+    """Inputs for timing the oracle on n_heads query heads (whole GQA groups) of the
+    workload's first sequence: uniform codes and N(0,1) codebooks (the oracle's time does
+    not depend on the values)."""
+    from decode_attention_commvq_b200 import synth
+    group = w.q_heads // w.kv_heads
+    n_heads = max(group, min(w.q_heads, n_heads // group * group))
+    n_kv = n_heads // group
+    T = int(w.lengths()[0])
+    ws = w.with_(kv_heads=n_kv, q_heads=n_heads, batch=1, ragged=None, seq_len=T)
+    kc = synth.uniform_codes(ws, True, T)
+    vc = synth.uniform_codes(ws, False, T)
+    kcb = synth.normal_codebook(w, True)
+    vcb = synth.normal_codebook(w, False)
+    q = synth.as_f32(synth.queries(w), w.q_dtype)[:1, :n_heads].astype(np.float64)
+    return q, kc, vc, np.array([0, T]), kcb, vcb, n_heads, T
+
+
+def time_oracle_step(w, sample):
+    from oracle import oracle as O
+    q, kc, vc, offs, kcb, vcb, n_heads, T = sample
+    t0 = time.perf_counter()
+    O.attend_codes(q, kc, vc, offs, kcb, vcb, w.rope_base)
+    dt = time.perf_counter() - t0
+    tokens = T * n_heads / w.q_heads        # context tokens of the full step this sample covers
+    return dt, tokens
+
+
+def cpu_baseline(w, n_heads):
+    sample = oracle_sample(w, n_heads)
+    dt, tokens = time_oracle_step(w, sample)
+    return {"value": tokens / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{sample[6]} of {w.q_heads} query heads of sequence 0 (T={sample[7]}), "
+                      f"single-threaded C oracle in fp64, {dt:.1f} s",
+            "seconds": dt, "cpu": cpu_model()}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for l in f:
+                if l.startswith("model name"):
+                    return l.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return None
+    sample = oracle_sample(w, w.q_heads // w.kv_heads)
+    for _ in range(args.warmup):
+        time_oracle_step(w, sample)
+    tot_t, tot_tok = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, tok = time_oracle_step(w, sample)
+        tot_t += dt
+        tot_tok += tok
+    value = tot_tok / tot_t
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads,
+                       "kv_heads": w.kv_heads, "d": w.d, "T": int(w.lengths().sum()), "R": w.R,
+                       "g": w.g, "n_codes": w.n_codes},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"each step: {sample[6]} of {w.q_heads} query heads (one GQA "
+                                       f"group) of sequence 0, T={sample[7]}; single-threaded C oracle"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    w = workload(args.workload)
+    if args.impl == "reference":
+        res = run_reference(args, w)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    try:
+        res = run_ours(args, w, rank, world, dev)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(w, args.cpu_heads)
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,217 @@
+"""ctypes binding of libcommvq_b200.so (the C ABI declared in include/commvq.h).
+
+Argument marshalling only: every step of the computation runs in the library's CUDA
+kernels. PyTorch supplies device memory and the current stream. There is no CPU
+fallback: if the shared library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcommvq_b200.so")
+
+F32, F16, BF16 = 0, 1, 2
+ATTN_AUTO, ATTN_TABLE, ATTN_DECODE_MMA = 0, 1, 2
+
+STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "WORKSPACE", 5: "DEVICE_CHECK"}
+
+EXPORTS = ("commvq_encode", "commvq_attend_workspace_bytes", "commvq_attend_decode",
+           "commvq_em_workspace_bytes", "commvq_em_step", "commvq_workspace_error",
+           "commvq_status_string", "commvq_abi_version")
+
+
+class CConfig(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("g", ctypes.c_int32), ("R", ctypes.c_int32),
+                ("n_codes", ctypes.c_int32), ("q_heads", ctypes.c_int32),
+                ("kv_heads", ctypes.c_int32), ("rope_base", ctypes.c_double),
+                ("code_bytes", ctypes.c_int32)]
+
+
+class CAttendOptions(ctypes.Structure):
+    _fields_ = [("algo", ctypes.c_int32), ("splits", ctypes.c_int32),
+                ("main_start", ctypes.c_void_p), ("main_stop", ctypes.c_void_p)]
+
+
+class CommVQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m decode_attention_commvq_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    CP = ctypes.POINTER(CConfig)
+    OP = ctypes.POINTER(CAttendOptions)
+    lib.commvq_encode.argtypes = [CP, P, I32, I64, P, P, P, P, P]
+    lib.commvq_encode.restype = I32
+    lib.commvq_attend_workspace_bytes.argtypes = [CP, I32, I64, OP]
+    lib.commvq_attend_workspace_bytes.restype = SZ
+    lib.commvq_attend_decode.argtypes = [CP, P, I32, P, P, P, I32, I64, P, P, P, P, P, SZ, OP, P]
+    lib.commvq_attend_decode.restype = I32
+    lib.commvq_em_workspace_bytes.argtypes = [CP, I64]
+    lib.commvq_em_workspace_bytes.restype = SZ
+    lib.commvq_em_step.argtypes = [CP, P, I64, P, P, P, P, SZ, P]
+    lib.commvq_em_step.restype = I32
+    lib.commvq_workspace_error.argtypes = [P, ctypes.POINTER(I32), P]
+    lib.commvq_workspace_error.restype = I32
+    lib.commvq_status_string.argtypes = [I32]
+    lib.commvq_status_string.restype = ctypes.c_char_p
+    lib.commvq_abi_version.argtypes = []
+    lib.commvq_abi_version.restype = I32
+    return lib
+
+
+LIB = _load()
+
+
+def status_string(status: int) -> str:
+    return LIB.commvq_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise CommVQError(status, what)
+
+
+@dataclass(frozen=True)
+class Config:
+    d: int = 128
+    g: int = 8
+    R: int = 2
+    n_codes: int = 256
+    q_heads: int = 32
+    kv_heads: int = 8
+    rope_base: float = 500000.0
+
+    @property
+    def code_bytes(self) -> int:
+        return 1 if self.n_codes <= 256 else 2
+
+    @property
+    def groups(self) -> int:
+        return self.d // self.g
+
+    def c(self) -> CConfig:
+        return CConfig(self.d, self.g, self.R, self.n_codes, self.q_heads, self.kv_heads,
+                       float(self.rope_base), self.code_bytes)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+_DT = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
+
+
+def code_dtype(cfg: Config):
+    return torch.uint8 if cfg.code_bytes == 1 else torch.int16
+
+
+def encode(cfg: Config, x: torch.Tensor, codebook: torch.Tensor, codes: Optional[torch.Tensor] = None,
+           near_ties: Optional[torch.Tensor] = None, residual_out: Optional[torch.Tensor] = None,
+           stream=None) -> torch.Tensor:
+    """commvq_encode: x [T, kv_heads, d] f16/f32 -> codes [T, kv_heads, R, d/g]."""
+    T = x.shape[0]
+    if codes is None:
+        codes = torch.empty((T, cfg.kv_heads, cfg.R, cfg.groups), dtype=code_dtype(cfg),
+                            device=x.device)
+    cc = cfg.c()
+    _check(LIB.commvq_encode(ctypes.byref(cc), _ptr(x), _DT[x.dtype], T, _ptr(codebook),
+                             _ptr(codes), _ptr(near_ties), _ptr(residual_out), _stream(stream)),
+           "commvq_encode")
+    return codes
+
+
+def _opts(algo: int, splits: int, events=None) -> CAttendOptions:
+    o = CAttendOptions(int(algo), int(splits), None, None)
+    if events is not None:
+        o.main_start = ctypes.c_void_p(events[0].cuda_event)
+        o.main_stop = ctypes.c_void_p(events[1].cuda_event)
+    return o
+
+
+def attend_workspace_bytes(cfg: Config, B: int, max_T: int, algo: int = ATTN_AUTO, splits: int = 0) -> int:
+    cc = cfg.c()
+    o = _opts(algo, splits)
+    return int(LIB.commvq_attend_workspace_bytes(ctypes.byref(cc), int(B), int(max_T), ctypes.byref(o)))
+
+
+def attend_workspace(cfg: Config, B: int, max_T: int, device, algo: int = ATTN_AUTO, splits: int = 0):
+    n = attend_workspace_bytes(cfg, B, max_T, algo, splits)
+    if n == 0:
+        raise CommVQError(1, "commvq_attend_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def attend_decode(cfg: Config, q: torch.Tensor, k_codes: torch.Tensor, v_codes: torch.Tensor,
+                  seq_offsets: torch.Tensor, max_T: int, k_codebook: torch.Tensor,
+                  v_codebook: torch.Tensor, out: Optional[torch.Tensor] = None,
+                  lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  algo: int = ATTN_AUTO, splits: int = 0, want_lse: bool = True, stream=None,
+                  main_events=None):
+    """commvq_attend_decode: returns (out [B, q_heads, d] f32, lse [B, q_heads] f32 or None).
+    main_events: optional (start, stop) torch.cuda.Event pair recorded around the main kernel."""
+    B = q.shape[0]
+    if out is None:
+        out = torch.empty((B, cfg.q_heads, cfg.d), dtype=torch.float32, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, cfg.q_heads), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = attend_workspace(cfg, B, max_T, q.device, algo, splits)
+    cc = cfg.c()
+    o = _opts(algo, splits, main_events)
+    _check(LIB.commvq_attend_decode(ctypes.byref(cc), _ptr(q), _DT[q.dtype], _ptr(k_codes),
+                                    _ptr(v_codes), _ptr(seq_offsets), int(B), int(max_T),
+                                    _ptr(k_codebook), _ptr(v_codebook), _ptr(out), _ptr(lse),
+                                    _ptr(workspace), workspace.numel(), ctypes.byref(o),
+                                    _stream(stream)), "commvq_attend_decode")
+    return out, lse
+
+
+def em_workspace_bytes(cfg: Config, N: int) -> int:
+    cc = cfg.c()
+    return int(LIB.commvq_em_workspace_bytes(ctypes.byref(cc), int(N)))
+
+
+def em_step(cfg: Config, rows: torch.Tensor, codebook_round: torch.Tensor,
+            codes_out: Optional[torch.Tensor] = None, sse_out: Optional[torch.Tensor] = None,
+            workspace: Optional[torch.Tensor] = None, stream=None):
+    """commvq_em_step: updates codebook_round [d/g, Nc', g] in place."""
+    N = rows.shape[0]
+    if workspace is None:
+        n = em_workspace_bytes(cfg, N)
+        if n == 0:
+            raise CommVQError(1, "commvq_em_workspace_bytes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=rows.device)
+    cc = cfg.c()
+    _check(LIB.commvq_em_step(ctypes.byref(cc), _ptr(rows), int(N), _ptr(codebook_round),
+                              _ptr(codes_out), _ptr(sse_out), _ptr(workspace), workspace.numel(),
+                              _stream(stream)), "commvq_em_step")
+    return codebook_round
+
+
+def workspace_error(workspace: torch.Tensor, stream=None) -> int:
+    v = ctypes.c_int32(0)
+    st = LIB.commvq_workspace_error(_ptr(workspace), ctypes.byref(v), _stream(stream))
+    if st not in (0, 5):
+        raise CommVQError(st, "commvq_workspace_error")
+    return int(v.value)
+
+
+def abi_version() -> int:
+    return int(LIB.commvq_abi_version())

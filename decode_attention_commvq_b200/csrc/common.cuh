@@ -1,0 +1,111 @@
+// Shared host/device helpers of the CommVQ B200 library (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "commvq.h"
+
+namespace commvq {
+
+constexpr int kThreads = 256;
+constexpr int kG = 8;          // scalars per shared index
+constexpr int kD = 128;        // head dimension of the attention kernels
+constexpr int kGroups = kD / kG;
+constexpr int kPairs = kG / 2; // RoPE pairs per group
+
+// Device error word bits (first 4 bytes of an attention workspace).
+constexpr int kErrCodeRange = 1;
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline commvq_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? COMMVQ_OK : COMMVQ_ERR_CUDA;
+}
+
+// Cached per-device attributes (the only state the library keeps).
+struct DeviceInfo {
+  int device = -1;
+  int sms = 0;
+  size_t smem_optin = 0;
+};
+DeviceInfo current_device_info();
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------------------------------
+// Nearest entry of a sub-codebook, the encoder's distance rule. Exactly the fp32 operations
+// the definition names, so codes are reproducible bit for bit:
+//   e_k = res_k - c_k (round to nearest), dist = fma(e_k, e_k, dist), k = 0..7 in order,
+//   strictly smaller distance replaces the winner (ties -> lowest index).
+struct Nearest {
+  float best;
+  float second;
+  int idx;
+};
+
+__device__ __forceinline__ void nearest_init(Nearest& n) {
+  n.best = __int_as_float(0x7f800000);
+  n.second = __int_as_float(0x7f800000);
+  n.idx = 0;
+}
+
+template <bool kTrack>
+__device__ __forceinline__ void nearest_step(Nearest& n, const float (&res)[kG], const float4 lo,
+                                             const float4 hi, int c) {
+  float dist = 0.0f;
+  float e;
+  e = __fsub_rn(res[0], lo.x); dist = __fmaf_rn(e, e, dist);
+  e = __fsub_rn(res[1], lo.y); dist = __fmaf_rn(e, e, dist);
+  e = __fsub_rn(res[2], lo.z); dist = __fmaf_rn(e, e, dist);
+  e = __fsub_rn(res[3], lo.w); dist = __fmaf_rn(e, e, dist);
+  e = __fsub_rn(res[4], hi.x); dist = __fmaf_rn(e, e, dist);
+  e = __fsub_rn(res[5], hi.y); dist = __fmaf_rn(e, e, dist);
+  e = __fsub_rn(res[6], hi.z); dist = __fmaf_rn(e, e, dist);
+  e = __fsub_rn(res[7], hi.w); dist = __fmaf_rn(e, e, dist);
+  if (dist < n.best) {
+    if (kTrack) n.second = n.best;
+    n.best = dist;
+    n.idx = c;
+  } else if (kTrack && dist < n.second) {
+    n.second = dist;
+  }
+}
+
+// Near tie: at least two entries and (d2 - d1) <= 1e-5 * d2, in fp32.
+__device__ __forceinline__ bool near_tie(const Nearest& n, int n_codes) {
+  if (n_codes < 2) return false;
+  const float gap = __fsub_rn(n.second, n.best);
+  const float lim = __fmul_rn(1e-5f, n.second);
+  return gap <= lim;
+}
+
+__device__ __forceinline__ void load_row8(const float* p, float (&v)[kG]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ void load_row8(const __half* p, float (&v)[kG]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+__device__ __forceinline__ void store_code(void* codes, int64_t at, int code, int code_bytes) {
+  if (code_bytes == 1)
+    static_cast<uint8_t*>(codes)[at] = static_cast<uint8_t>(code);
+  else
+    static_cast<uint16_t*>(codes)[at] = static_cast<uint16_t>(code);
+}
+
+}  // namespace commvq

@@ -1,0 +1,191 @@
+/*
+ * commvq.h -- C ABI of the CommVQ decode-attention library for B200 (sm_100a).
+ *
+ * CommVQ (CommVQ: Commutative Vector Quantization for KV Cache Compression) stores the
+ * key/value cache as additive vector-quantization codes: g consecutive scalars share one
+ * index, R residual rounds each pick one entry of an Nc'-entry sub-codebook, and a row is
+ * decoded as the sum of its selected entries (abstract: decoding is a matrix multiply;
+ * machine review, "What carries the argument": index sharing, R rounds,
+ * R*log2(Nc')/g bits per scalar). The key codebook's 2x2 blocks [[x, y], [-y, x]] commute
+ * with the RoPE rotation, so attention scores can be formed from a per-query
+ * query x codebook table and rotated afterwards ("What carries the argument",
+ * Property 1 / Eq. 7-8). Values are decoded after the softmax weights have been folded
+ * into the codes ("If this is right": weights multiply value codes before the codebook
+ * multiply).
+ *
+ * Conventions shared by every call
+ *  - d = 128, g = 8 (4 RoPE pairs per index), d/g = 16 groups for attention; the
+ *    encoder and the EM step accept any d that is a multiple of 8 with g = 8.
+ *  - RoPE pair p is channels (2p, 2p+1), theta_p = rope_base^(-2p/d); the key of row t of
+ *    a sequence sits at position t; queries arrive already rotated; scores are scaled
+ *    by 1/sqrt(d); there is no mask.
+ *  - A stored key pair (a, b) is the reconstructed 2-vector (its commuting block is
+ *    [[a, -b], [b, a]]).
+ *  - Codes: [T, kv_heads, R, d/g], one code per element, uint8 when Nc' <= 256
+ *    (code_bytes = 1) else uint16 (code_bytes = 2), little-endian.
+ *  - Codebooks: [R, d/g, Nc', g] float32, shared by all KV heads and sequences.
+ *  - Query head h reads KV head h / (q_heads / kv_heads).
+ *
+ * Ownership and memory: the caller owns every buffer. All tensor pointers are device
+ * pointers (CUDA global memory) unless stated; the config struct is host memory. The
+ * library allocates nothing, keeps no state besides cached device attributes, and never
+ * synchronises a stream except where a call says so. Calls are asynchronous on `stream`
+ * (a cudaStream_t; NULL = legacy default stream).
+ *
+ * Errors: arguments are validated on the host before any launch; a failed check returns
+ * a status and launches nothing. A launch failure returns COMMVQ_ERR_CUDA. Data errors
+ * found on the device (a code >= Nc') never trap: the kernel clamps the code, records
+ * the error in the workspace's error word and carries on; read it with
+ * commvq_workspace_error().
+ */
+#ifndef COMMVQ_H_
+#define COMMVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  COMMVQ_OK = 0,
+  COMMVQ_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size or shape */
+  COMMVQ_ERR_UNSUPPORTED = 2,   /* valid CommVQ shape this build does not implement */
+  COMMVQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+  COMMVQ_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
+  COMMVQ_ERR_DEVICE_CHECK = 5   /* the device recorded a data error (code out of range) */
+} commvq_status;
+
+typedef enum { COMMVQ_F32 = 0, COMMVQ_F16 = 1, COMMVQ_BF16 = 2 } commvq_dtype;
+
+/* Attention algorithms (both compute the same attention; see commvq_attend_decode). */
+typedef enum {
+  COMMVQ_ATTN_AUTO = 0,       /* the library's fastest for the shape */
+  COMMVQ_ATTN_TABLE = 1,      /* per-query table + value histograms, one CTA per (b, q head, split) */
+  COMMVQ_ATTN_DECODE_MMA = 2  /* decode each (token, KV head) once, rotate, tensor-core QK and PV */
+} commvq_attn_algo;
+
+typedef struct {
+  int32_t d;          /* head dimension */
+  int32_t g;          /* scalars per shared index */
+  int32_t R;          /* residual rounds */
+  int32_t n_codes;    /* Nc', entries per sub-codebook */
+  int32_t q_heads;    /* query heads (attention only) */
+  int32_t kv_heads;   /* KV heads */
+  double rope_base;   /* RoPE base (attention only) */
+  int32_t code_bytes; /* 1 if n_codes <= 256 else 2 */
+} commvq_config;
+
+typedef struct {
+  int32_t algo;        /* commvq_attn_algo */
+  int32_t splits;      /* split-T partitions per sequence; 0 = chosen by the library */
+  void* main_start;    /* nullable cudaEvent_t, recorded on `stream` right before the main
+                          attention kernel (instrumentation; no effect on the result) */
+  void* main_stop;     /* nullable cudaEvent_t, recorded right after it, before the merge */
+} commvq_attend_options;
+
+/* Residual nearest-codeword encoder (abstract: additive quantization; "What carries the
+ * argument": g scalars per index, R residual rounds; Figure 1: every K/V vector is
+ * encoded on its own).
+ * For each row n of x and group j, with res = x[n, j*g:(j+1)*g] in fp32 and r = 0..R-1:
+ *   dist(c) = fused sum over k = 0..g-1 in order of e_k^2, e_k = res_k - cb[r,j,c,k]
+ *             (fp32 subtract, then fmaf(e, e, dist) starting from 0),
+ *   code = first c with the strictly smallest dist (ties -> lowest index),
+ *   res  = res - cb[r, j, code, :] (fp32).
+ * x        [n_tokens, kv_heads, d] in x_dtype (COMMVQ_F32 or COMMVQ_F16), pre-RoPE keys or
+ *          values, 16-byte aligned, contiguous.
+ * codebook [R, d/g, Nc', g] float32, 16-byte aligned.
+ * codes    [n_tokens, kv_heads, R, d/g] out, code_bytes per element.
+ * near_ties nullable device counter; if given, the number of (row, round, group)
+ *          decisions whose two smallest distances d1 <= d2 satisfy d2 - d1 <= 1e-5 * d2
+ *          (fp32, Nc' >= 2) is ADDED to it.
+ * residual_out nullable [n_tokens, kv_heads, d] float32, 16-byte aligned: the residual
+ *          after the last round (what a further round, or the next round of a codebook
+ *          fit, would encode).
+ * Supports g = 8, d % 8 == 0, 1 <= Nc' <= 65536, 1 <= R <= 16. n_tokens = 0 is a no-op. */
+commvq_status commvq_encode(const commvq_config* cfg, const void* x, commvq_dtype x_dtype,
+                            int64_t n_tokens, const float* codebook, void* codes,
+                            unsigned long long* near_ties, float* residual_out, void* stream);
+
+/* Bytes of device workspace commvq_attend_decode needs for B sequences whose longest
+ * has max_T cached rows (options may be NULL = defaults). Returns 0 for invalid input. */
+size_t commvq_attend_workspace_bytes(const commvq_config* cfg, int32_t B, int64_t max_T,
+                                     const commvq_attend_options* options);
+
+/* Decode-step attention computed on the codes (no decompressed cache is formed in HBM).
+ * For sequence b (rows seq_offsets[b] .. seq_offsets[b+1]-1, positions 0..T_b-1) and
+ * query head h reading KV head kvh = h / (q_heads / kv_heads):
+ *   k^_t = sum_r kcb[r, j, kcode[t,kvh,r,j], :] per group j, k~_t = RoPE_t(k^_t),
+ *   s_t = q[b,h] . k~_t / sqrt(d), p = softmax(s),
+ *   out[b,h] = sum_t p_t v^_t, v^_t = sum_r vcb[r, j, vcode[t,kvh,r,j], :],
+ *   lse[b,h] = log(sum_t exp(s_t)) (natural log); an empty sequence gives out = 0 and
+ *   lse = -inf.
+ * The rotation is applied per position to query x codebook products (key side) and the
+ * softmax weights are accumulated per code before the value codebook multiply, as the
+ * review describes. Precision: fp32 accumulation; the per-query table / decoded rows are
+ * held in fp16 (relative error ~5e-4 per product).
+ * q           [B, q_heads, d] in q_dtype (F32, F16 or BF16), 16-byte aligned.
+ * k_codes, v_codes  [total_T, kv_heads, R, d/g] uint8 (attention supports Nc' <= 256),
+ *             16-byte aligned; total_T = seq_offsets[B].
+ * seq_offsets [B+1] int64 device array, non-decreasing, seq_offsets[0] = 0, every
+ *             T_b <= max_T (a longer sequence is truncated to max_T rows: the caller
+ *             must pass the true maximum).
+ * k_codebook, v_codebook [R, d/g, Nc', g] float32, 16-byte aligned.
+ * out         [B, q_heads, d] float32 out, 16-byte aligned.
+ * lse         [B, q_heads] float32 out, nullable.
+ * workspace   device buffer of at least commvq_attend_workspace_bytes(...) bytes,
+ *             256-byte aligned; its first 64 bytes hold the device error word, which this
+ *             call clears. Calls that share a workspace must be ordered on one stream.
+ * options     nullable (defaults: AUTO algorithm, library-chosen splits).
+ * Supports d = 128, g = 8, Nc' <= 256 (code_bytes = 1), 1 <= R <= 4, q_heads % kv_heads == 0,
+ * B >= 0 (B = 0 is a no-op). */
+commvq_status commvq_attend_decode(const commvq_config* cfg, const void* q, commvq_dtype q_dtype,
+                                   const void* k_codes, const void* v_codes,
+                                   const int64_t* seq_offsets, int32_t B, int64_t max_T,
+                                   const float* k_codebook, const float* v_codebook,
+                                   float* out, float* lse, void* workspace,
+                                   size_t workspace_bytes, const commvq_attend_options* options,
+                                   void* stream);
+
+/* Bytes of device workspace commvq_em_step needs for N rows. 0 for invalid input. */
+size_t commvq_em_workspace_bytes(const commvq_config* cfg, int64_t N);
+
+/* One EM step for one residual round's codebook (review: codebook fit by EM, Algorithm 1
+ * and Eq. 20 -- hard assignment, closed-form centroid update; "no convergence guarantee
+ * beyond local").
+ *   assignment: the encoder's rule (one round) of every row's groups against the input
+ *               codebook_round;
+ *   update:     entry (j, c) = (float)(S / m), S the fp64 sum of the m fp32 sub-vectors
+ *               assigned to it; an entry with m = 0 keeps its value.
+ * Every stored pair already has the commuting-block form, so the key codebook needs no
+ * projection after the mean.
+ * rows           [N, d] float32 residual rows of this round, 16-byte aligned.
+ * codebook_round [d/g, Nc', g] float32, read and overwritten in place.
+ * codes_out      [N, d/g] nullable, code_bytes per element: assignments against the input
+ *                codebook.
+ * sse_out        nullable device double: sum over (row, group) of the assignment distance,
+ *                accumulated in fp64.
+ * workspace      >= commvq_em_workspace_bytes(cfg, N) bytes, 256-byte aligned.
+ * The result does not depend on launch order (fixed-order fp64 reductions). Supports
+ * g = 8, d % 8 == 0, 1 <= Nc' <= 4096, N >= 1. cfg->R is ignored. */
+commvq_status commvq_em_step(const commvq_config* cfg, const float* rows, int64_t N,
+                             float* codebook_round, void* codes_out, double* sse_out,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* The device error word in an attention workspace: synchronises `stream`, copies the word
+ * to the host and writes it to *device_error (0 = none; bit 0 = a code >= Nc' was seen
+ * and clamped). Returns COMMVQ_ERR_DEVICE_CHECK when the word is non-zero. */
+commvq_status commvq_workspace_error(const void* workspace, int32_t* device_error, void* stream);
+
+/* Static description of a status code. */
+const char* commvq_status_string(commvq_status status);
+
+/* ABI version of this library (incremented on any signature change). */
+int32_t commvq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* COMMVQ_H_ */

@@ -1,0 +1,118 @@
+"""CPU checks of the C ABI: the library builds and loads, exports every function the
+header declares, and rejects bad arguments on the host before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "commvq.h")
+
+
+@pytest.fixture(scope="module")
+def api():
+    from decode_attention_commvq_b200 import build
+    build.build()
+    from decode_attention_commvq_b200 import api as A
+    return A
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(commvq_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for n in ("commvq_encode", "commvq_attend_decode", "commvq_em_step",
+              "commvq_attend_workspace_bytes", "commvq_em_workspace_bytes",
+              "commvq_workspace_error", "commvq_status_string", "commvq_abi_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(api):
+    lib = ctypes.CDLL(api.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    assert set(api.EXPORTS) == set(declared_functions())
+
+
+def test_status_strings_and_version(api):
+    assert api.abi_version() == 1
+    for s in range(6):
+        assert api.status_string(s)
+    assert "unknown" in api.status_string(99)
+
+
+def _cfg(api, **kw):
+    base = dict(d=128, g=8, R=2, n_codes=256, q_heads=32, kv_heads=8, rope_base=5e5)
+    base.update(kw)
+    return api.Config(**base)
+
+
+FAKE = 0x10000  # a 256-byte-aligned non-null address; never dereferenced by these calls
+
+
+def _attend(api, cfg, B=1, max_T=100, ws_bytes=1 << 20, q=FAKE, kc=FAKE, vc=FAKE, offs=FAKE,
+            kcb=FAKE, vcb=FAKE, out=FAKE, lse=None, ws=FAKE, qdt=2, opts=None):
+    cc = cfg.c()
+    P = ctypes.c_void_p
+    return api.LIB.commvq_attend_decode(ctypes.byref(cc), P(q), qdt, P(kc), P(vc), P(offs), B, max_T,
+                                        P(kcb), P(vcb), P(out), P(lse) if lse else None, P(ws),
+                                        ws_bytes, ctypes.byref(opts) if opts else None, None)
+
+
+def test_attend_rejects_bad_arguments(api):
+    INVALID, UNSUP, WS = 1, 2, 4
+    cfg = _cfg(api)
+    assert _attend(api, _cfg(api, q_heads=30)) == INVALID          # Hq % Hkv
+    assert _attend(api, _cfg(api, g=7)) == INVALID                  # d % g
+    assert _attend(api, _cfg(api, n_codes=0)) == INVALID
+    assert _attend(api, _cfg(api, rope_base=-1.0)) == INVALID
+    assert _attend(api, _cfg(api, d=64)) == UNSUP
+    assert _attend(api, _cfg(api, n_codes=512)) == UNSUP            # uint16 codes
+    assert _attend(api, _cfg(api, R=5)) == UNSUP
+    assert _attend(api, cfg, q=0) == INVALID
+    assert _attend(api, cfg, q=FAKE + 8) == INVALID                 # misaligned
+    assert _attend(api, cfg, ws=FAKE + 16) == INVALID               # workspace alignment
+    assert _attend(api, cfg, qdt=7) == INVALID
+    assert _attend(api, cfg, B=-1) == INVALID
+    assert _attend(api, cfg, ws_bytes=16) == WS
+    assert _attend(api, cfg, B=0) == 0                               # no-op
+    bad = api.CAttendOptions(9, 0)
+    assert _attend(api, cfg, opts=bad) == INVALID
+    bad = api.CAttendOptions(0, -2)
+    assert _attend(api, cfg, opts=bad) == INVALID
+
+
+def test_workspace_sizes(api):
+    cfg = _cfg(api)
+    one = api.attend_workspace_bytes(cfg, 1, 32768, splits=4)
+    assert one == 256 + 32 * 4 * 528
+    assert api.attend_workspace_bytes(cfg, 16, 8192, splits=1) == 256 + 16 * 32 * 528
+    assert api.attend_workspace_bytes(_cfg(api, q_heads=30), 1, 10) == 0
+    em = api.em_workspace_bytes(cfg, 65536)
+    assert em >= 32 * 16 * 256 * (8 * 8 + 4)
+    assert api.em_workspace_bytes(cfg, 0) == 0
+    assert api.em_workspace_bytes(_cfg(api, n_codes=5000), 10) == 0
+
+
+def test_encode_and_em_reject_bad_arguments(api):
+    INVALID, UNSUP = 1, 2
+    P = ctypes.c_void_p
+    cc = _cfg(api).c()
+    enc = api.LIB.commvq_encode
+    assert enc(ctypes.byref(cc), P(FAKE), 1, 0, P(FAKE), P(FAKE), None, None, None) == 0   # T = 0
+    assert enc(ctypes.byref(cc), None, 1, 5, P(FAKE), P(FAKE), None, None, None) == INVALID
+    assert enc(ctypes.byref(cc), P(FAKE + 4), 1, 5, P(FAKE), P(FAKE), None, None, None) == INVALID
+    assert enc(ctypes.byref(cc), P(FAKE), 2, 5, P(FAKE), P(FAKE), None, None, None) == UNSUP  # bf16 rows
+    c2 = _cfg(api, n_codes=300).c()                  # code_bytes must be 2
+    c2.code_bytes = 1
+    assert enc(ctypes.byref(c2), P(FAKE), 1, 5, P(FAKE), P(FAKE), None, None, None) == INVALID
+    em = api.LIB.commvq_em_step
+    assert em(ctypes.byref(cc), P(FAKE), 0, P(FAKE), None, None, P(FAKE), 1 << 30, None) == INVALID
+    assert em(ctypes.byref(cc), P(FAKE), 100, P(FAKE), None, None, P(FAKE), 16, None) == 4
+    c3 = _cfg(api, n_codes=5000).c()
+    assert em(ctypes.byref(c3), P(FAKE), 100, P(FAKE), None, None, P(FAKE), 1 << 30, None) == UNSUP

@@ -1,0 +1,207 @@
+"""Decode-attention parity: CUDA output vs the fp64 oracle (decompress, RoPE, softmax)
+within 2e-3 (fp32 query) / 5e-3 (bf16 query) max relative error per (b, h), on every
+workload, every algorithm and several split counts; plus the degenerate cases."""
+import numpy as np
+import pytest
+import torch
+
+from decode_attention_commvq_b200 import synth
+from oracle import oracle as O
+from tests.helpers import oracle_codebooks, q_as_f64, rel_err, to_torch_q, tol_for
+
+pytestmark = pytest.mark.gpu
+
+ALGOS = [1]   # table path
+
+
+@pytest.fixture(scope="module")
+def api():
+    from decode_attention_commvq_b200 import api as A
+    return A
+
+
+def _cfg(api, w):
+    return api.Config(d=w.d, g=w.g, R=w.R, n_codes=w.n_codes, q_heads=w.q_heads,
+                      kv_heads=w.kv_heads, rope_base=w.rope_base)
+
+
+def _codes_np_to_gpu(c, gpu):
+    return torch.from_numpy(np.ascontiguousarray(c.astype(np.uint8))).to(gpu)
+
+
+def _run(api, w, q_np, kc, vc, offs, kcb, vcb, gpu, algo=0, splits=0):
+    cfg = _cfg(api, w)
+    q = to_torch_q(q_np, w.q_dtype, gpu)
+    offsets = torch.from_numpy(offs.astype(np.int64)).to(gpu)
+    max_T = int(np.diff(offs).max()) if len(offs) > 1 else 0
+    out, lse = api.attend_decode(cfg, q, _codes_np_to_gpu(kc, gpu), _codes_np_to_gpu(vc, gpu),
+                                 offsets, max_T, torch.from_numpy(kcb).to(gpu),
+                                 torch.from_numpy(vcb).to(gpu), algo=algo, splits=splits)
+    torch.cuda.synchronize()
+    return out.cpu().numpy(), lse.cpu().numpy()
+
+
+def _encoded_inputs(w, T=None):
+    """Seeded K/V rows encoded by the oracle (small sizes)."""
+    kcb, vcb = oracle_codebooks(w)
+    if T is not None:
+        w = w.with_(seq_len=T)
+    kx = synth.kv_cache_rows(w, True)
+    vx = synth.kv_cache_rows(w, False)
+    kc, _ = O.encode(kx, kcb)
+    vc, _ = O.encode(vx, vcb)
+    return w, kc, vc, kcb, vcb
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("splits", [0, 1, 3])
+def test_tiny_workload(api, gpu, algo, splits):
+    w, kc, vc, kcb, vcb = _encoded_inputs(synth.WORKLOADS[0])
+    q = synth.queries(w)
+    offs = w.offsets()
+    out, lse = _run(api, w, q, kc, vc, offs, kcb, vcb, gpu, algo, splits)
+    ref, ref_lse = O.attend_codes(q_as_f64(w, q), kc, vc, offs, kcb, vcb, w.rope_base)
+    assert rel_err(out, ref) <= tol_for(w)
+    assert np.allclose(lse, ref_lse, rtol=1e-3, atol=5e-3)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("splits", [0, 2, 7])
+def test_2bit_layer_short_context_all_heads(api, gpu, algo, splits):
+    """All 32 heads on 3000 encoded positions: several 256-position chunks and a ragged tail."""
+    w, kc, vc, kcb, vcb = _encoded_inputs(synth.WORKLOADS[1], T=3000)
+    q = synth.queries(w)
+    offs = w.offsets()
+    out, lse = _run(api, w, q, kc, vc, offs, kcb, vcb, gpu, algo, splits)
+    ref, ref_lse = O.attend_codes(q_as_f64(w, q), kc, vc, offs, kcb, vcb, w.rope_base)
+    assert rel_err(out, ref) <= tol_for(w)
+    assert np.allclose(lse, ref_lse, rtol=1e-3, atol=5e-3)
+
+
+def _full_size_sampled(api, gpu, w, heads, algo=0, splits=0):
+    """Full-size workload with uniform random codes; the oracle computes selected heads."""
+    kcb, vcb = oracle_codebooks(w)
+    offs = w.offsets()
+    total = int(offs[-1])
+    kc = synth.uniform_codes(w, True, total)
+    vc = synth.uniform_codes(w, False, total)
+    q = synth.queries(w)
+    out, lse = _run(api, w, q, kc, vc, offs, kcb, vcb, gpu, algo, splits)
+    qf = q_as_f64(w, q)
+    group = w.q_heads // w.kv_heads
+    errs = []
+    for b, h in heads:
+        kvh = h // group
+        sl = slice(offs[b], offs[b + 1])
+        ref, ref_lse = O.attend_codes(qf[b:b + 1, h:h + 1], kc[sl, kvh:kvh + 1], vc[sl, kvh:kvh + 1],
+                                      np.array([0, offs[b + 1] - offs[b]]), kcb, vcb, w.rope_base)
+        errs.append(rel_err(out[b, h], ref[0, 0]))
+        assert abs(lse[b, h] - ref_lse[0, 0]) <= 1e-3 * max(1.0, abs(ref_lse[0, 0]))
+    assert max(errs) <= tol_for(w), errs
+    return out
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_2bit_layer_full_size(api, gpu, algo):
+    w = synth.WORKLOADS[1]
+    _full_size_sampled(api, gpu, w, [(0, 0), (0, 5), (0, 18), (0, 31)], algo)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_1bit_layer_full_size(api, gpu, algo):
+    w = synth.WORKLOADS[2]
+    _full_size_sampled(api, gpu, w, [(0, 0), (0, 13), (0, 27)], algo)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_ragged_batch_full_size(api, gpu, algo):
+    w = synth.WORKLOADS[3]
+    _full_size_sampled(api, gpu, w, [(0, 0), (3, 9), (7, 31), (15, 16)], algo)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_split_count_invariance(api, gpu, algo):
+    w, kc, vc, kcb, vcb = _encoded_inputs(synth.WORKLOADS[1], T=2000)
+    q = synth.queries(w)
+    offs = w.offsets()
+    outs = [_run(api, w, q, kc, vc, offs, kcb, vcb, gpu, algo, s)[0] for s in (1, 2, 5, 16)]
+    for o in outs[1:]:
+        assert rel_err(o, outs[0]) <= 1e-5
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_degenerate_lengths(api, gpu, algo):
+    """Empty sequences (out 0, lse -inf), a single position (out = its value), and
+    lengths shorter than the split count, mixed in one ragged batch."""
+    w = synth.WORKLOADS[1].with_(batch=5, ragged=(0, 0))
+    kcb, vcb = oracle_codebooks(synth.WORKLOADS[1])
+    lens = np.array([0, 1, 3, 0, 300])
+    offs = np.concatenate([[0], np.cumsum(lens)])
+    total = int(offs[-1])
+    kc = synth.uniform_codes(w, True, total)
+    vc = synth.uniform_codes(w, False, total)
+    q = synth.queries(w)
+    out, lse = _run(api, w, q, kc, vc, offs, kcb, vcb, gpu, algo, splits=4)
+    ref, ref_lse = O.attend_codes(q_as_f64(w, q), kc, vc, offs, kcb, vcb, w.rope_base)
+    for b in (0, 3):
+        assert np.all(out[b] == 0) and np.all(np.isneginf(lse[b]))
+    for b in (1, 2, 4):
+        assert rel_err(out[b], ref[b]) <= tol_for(w)
+    row = int(offs[1])                               # sequence 1's only position
+    vhat = O.decode(vc[row:row + 1], vcb)[0]         # [Hkv, d]
+    for h in range(w.q_heads):
+        assert np.allclose(out[1, h], vhat[h // 4], rtol=1e-3, atol=1e-3)
+
+
+def test_zero_query_gives_mean_value(api, gpu):
+    w = synth.WORKLOADS[1].with_(seq_len=777)
+    kcb, vcb = oracle_codebooks(synth.WORKLOADS[1])
+    offs = w.offsets()
+    kc = synth.uniform_codes(w, True, 777)
+    vc = synth.uniform_codes(w, False, 777)
+    q = np.zeros((1, w.q_heads, w.d), dtype=np.uint16)    # bf16 zeros
+    out, lse = _run(api, w, q, kc, vc, offs, kcb, vcb, gpu)
+    vhat = O.decode(vc, vcb)                               # [T, Hkv, d]
+    mean = vhat.mean(0)
+    for h in range(w.q_heads):
+        assert rel_err(out[0, h], mean[h // 4]) <= 1e-4
+    assert np.allclose(lse, np.log(777), rtol=1e-5)
+
+
+def test_out_of_range_codes_are_flagged_not_trapped(api, gpu):
+    """Nc' = 16 with uint8 codes: a code >= 16 is clamped to 15 and recorded in the
+    workspace error word; the call itself completes."""
+    w = synth.WORKLOADS[0]
+    kcb, vcb = oracle_codebooks(w)
+    cfg = _cfg(api, w)
+    kc = synth.uniform_codes(w, True, 256)
+    vc = synth.uniform_codes(w, False, 256)
+    kc[17, 0, 0, 3] = 200
+    q = to_torch_q(synth.queries(w), w.q_dtype, gpu)
+    offs = torch.tensor([0, 256], dtype=torch.int64, device=gpu)
+    ws = api.attend_workspace(cfg, 1, 256, gpu)
+    out, _ = api.attend_decode(cfg, q, _codes_np_to_gpu(kc, gpu), _codes_np_to_gpu(vc, gpu), offs, 256,
+                               torch.from_numpy(kcb).to(gpu), torch.from_numpy(vcb).to(gpu),
+                               workspace=ws)
+    assert api.workspace_error(ws) == 1
+    kc2 = kc.copy()
+    kc2[17, 0, 0, 3] = 15
+    out2, _ = api.attend_decode(cfg, q, _codes_np_to_gpu(kc2, gpu), _codes_np_to_gpu(vc, gpu), offs,
+                                256, torch.from_numpy(kcb).to(gpu), torch.from_numpy(vcb).to(gpu),
+                                workspace=ws)
+    assert api.workspace_error(ws) == 0
+    # value histograms accumulate with shared-memory float atomics: equal up to rounding order
+    assert rel_err(out.cpu().numpy(), out2.cpu().numpy()) <= 1e-6
+
+
+def test_workspace_too_small_is_rejected(api, gpu):
+    w = synth.WORKLOADS[0]
+    cfg = _cfg(api, w)
+    ws = torch.empty(64, dtype=torch.uint8, device=gpu)
+    z = torch.zeros(1, w.q_heads, w.d, dtype=torch.float32, device=gpu)
+    codes = torch.zeros(256, 1, 1, 16, dtype=torch.uint8, device=gpu)
+    cb = torch.zeros(1, 16, 16, 8, dtype=torch.float32, device=gpu)
+    offs = torch.tensor([0, 256], dtype=torch.int64, device=gpu)
+    with pytest.raises(api.CommVQError) as e:
+        api.attend_decode(cfg, z, codes, codes, offs, 256, cb, cb, workspace=ws)
+    assert e.value.status == 4

@@ -1,0 +1,119 @@
+"""Encoder parity: CUDA codes must equal the oracle's bit for bit (ties to the lowest
+index), with the same near-tie count and the same fp32 residual."""
+import numpy as np
+import pytest
+import torch
+
+from decode_attention_commvq_b200 import synth
+from oracle import oracle as O
+from tests.helpers import oracle_codebooks
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def api():
+    from decode_attention_commvq_b200 import api as A
+    return A
+
+
+def _cfg(api, w):
+    return api.Config(d=w.d, g=w.g, R=w.R, n_codes=w.n_codes, q_heads=w.q_heads,
+                      kv_heads=w.kv_heads, rope_base=w.rope_base)
+
+
+def _run(api, cfg, x_np, cb_np, gpu, residual=False):
+    x = torch.from_numpy(x_np).to(gpu)
+    cb = torch.from_numpy(cb_np).to(gpu)
+    ties = torch.zeros(1, dtype=torch.int64, device=gpu)
+    res = torch.empty(x.shape, dtype=torch.float32, device=gpu) if residual else None
+    codes = api.encode(cfg, x, cb, near_ties=ties, residual_out=res)
+    torch.cuda.synchronize()
+    c = codes.cpu().numpy()
+    if cfg.code_bytes == 2:
+        c = c.view(np.uint16)
+    return c.astype(np.int64), int(ties.item()), (res.cpu().numpy() if residual else None)
+
+
+def _compare(api, cfg, x_np, cb_np, gpu, residual=True):
+    got, ties, res = _run(api, cfg, x_np, cb_np, gpu, residual)
+    want, want_ties, want_res = O.encode(x_np, cb_np, want_residual=True)
+    assert got.shape == want.shape
+    mism = np.argwhere(got != want)
+    assert mism.size == 0, f"{len(mism)} code mismatches, first at {mism[:5]}"
+    assert ties == want_ties
+    if residual:
+        assert np.array_equal(res.view(np.uint32), want_res.astype(np.float32).view(np.uint32))
+    return want_ties
+
+
+def test_encode_tiny_workload(api, gpu):
+    w = synth.WORKLOADS[0]
+    kcb, vcb = oracle_codebooks(w)
+    cfg = _cfg(api, w)
+    for key, cb in ((True, kcb), (False, vcb)):
+        x = synth.kv_cache_rows(w, key)          # fp32 rows
+        _compare(api, cfg, x, cb, gpu)
+
+
+@pytest.mark.parametrize("key", [True, False])
+def test_encode_2bit_layer_slice(api, gpu, key):
+    w = synth.WORKLOADS[1]
+    kcb, vcb = oracle_codebooks(w)
+    cfg = _cfg(api, w)
+    x = synth.kv_rows(w, key, T=1027)            # fp16, ragged tail vs 512-row blocks
+    _compare(api, cfg, x, kcb if key else vcb, gpu)
+
+
+def test_encode_1bit_layer_slice(api, gpu):
+    w = synth.WORKLOADS[2]
+    kcb, _ = oracle_codebooks(w)
+    cfg = _cfg(api, w)
+    x = synth.kv_rows(w, True, T=300)
+    _compare(api, cfg, x, kcb, gpu)
+
+
+def test_encode_full_workload_sampled_rows(api, gpu):
+    """The encode workload at full size (131072 x 8 rows of fp16 K): codes of a seeded
+    sample of rows are checked one by one against the oracle."""
+    w = synth.WORKLOADS[4]
+    kcb, _ = oracle_codebooks(w.with_(em_rows=4096, em_iters=2))
+    cfg = _cfg(api, w)
+    x = synth.encode_rows(w, True, w.encode_tokens)
+    got, _, _ = _run(api, cfg, x, kcb, gpu)
+    rng = np.random.default_rng(123)
+    toks = np.sort(rng.choice(w.encode_tokens, 512, replace=False))
+    toks = np.concatenate([toks, [0, w.encode_tokens - 1]])
+    want, _ = O.encode(x[toks], kcb)
+    assert np.array_equal(got[toks], want)
+
+
+def test_encode_uint16_codes_and_multi_tile(api, gpu):
+    rng = np.random.default_rng(7)
+    for Nc, R in ((300, 2), (1500, 1), (2, 3)):
+        cfg = api.Config(d=64, g=8, R=R, n_codes=Nc, q_heads=1, kv_heads=3)
+        cb = rng.standard_normal((R, 8, Nc, 8)).astype(np.float32)
+        x = rng.standard_normal((97, 3, 64)).astype(np.float16)
+        _compare(api, cfg, x, cb, gpu)
+
+
+def test_encode_ties_and_duplicates(api, gpu):
+    cfg = api.Config(d=16, g=8, R=1, n_codes=8, q_heads=1, kv_heads=1)
+    cb = np.zeros((1, 2, 8, 8), dtype=np.float32)
+    cb[0, :, 3] = 1.0
+    cb[0, :, 6] = 1.0        # duplicate of entry 3
+    cb[0, :, 0] = -2.0
+    x = np.ones((5, 1, 16), dtype=np.float32)
+    t = _compare(api, cfg, x, cb, gpu)
+    assert t == 10
+    got, _, _ = _run(api, cfg, x, cb, gpu)
+    assert np.all(got == 3)
+
+
+def test_encode_empty(api, gpu):
+    w = synth.WORKLOADS[1]
+    cfg = _cfg(api, w)
+    x = torch.empty((0, 8, 128), dtype=torch.float16, device=gpu)
+    cb = torch.zeros((2, 16, 256, 8), dtype=torch.float32, device=gpu)
+    codes = api.encode(cfg, x, cb)
+    assert codes.shape == (0, 8, 2, 16)
