@@ -64,8 +64,12 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_sha():
-    src = os.path.join(ROOT, "decode_attention_commvq_b200", "csrc", "attend_table.cu")
+KERNEL_SOURCES = {"attend_table_kernel": "attend_table.cu",
+                  "attend_scores_kernel+attend_values_kernel": "attend_mma.cu"}
+
+
+def kernel_source_sha(kernel: str):
+    src = os.path.join(ROOT, "decode_attention_commvq_b200", "csrc", KERNEL_SOURCES[kernel])
     with open(src, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
@@ -78,9 +82,21 @@ def recorded_traffic(kernel: str, workload_name: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel, {}).get(workload_name)
-    if not e or e.get("source_sha") != kernel_source_sha():
+    if not e or e.get("source_sha") != kernel_source_sha(kernel):
         return None
     return float(e["dram_bytes_per_launch"])
+
+
+def main_kernel(api, cfg, algo):
+    """Name of the kernel(s) the main events bracket for this shape and algorithm."""
+    run = algo
+    if algo == api.ATTN_AUTO:
+        mma_ok = cfg.R <= 2 and cfg.n_codes <= 256 and cfg.kv_heads in (1, 2, 4, 8) and \
+            cfg.q_heads % cfg.kv_heads == 0 and cfg.q_heads // cfg.kv_heads <= 8
+        run = api.ATTN_DECODE_MMA if mma_ok else api.ATTN_TABLE
+    if run == api.ATTN_DECODE_MMA:
+        return "attend_scores_kernel+attend_values_kernel", 4   # prep, scores, values, merge
+    return "attend_table_kernel", 2                             # table, merge
 
 
 # ---------------------------------------------------------------------------------------
@@ -138,6 +154,25 @@ class ClockSampler:
             return None
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------
+# multi-rank plumbing (replicas: no data-path collective)
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: one all-reduce (MAX) of a timing scalar."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, steps: int, units_per_step: int, ms_max: float) -> float:
+    """Whole-job units per second: every rank processes units_per_step per step."""
+    return world * steps * units_per_step / (ms_max / 1e3)
 
 
 # ---------------------------------------------------------------------------------------
@@ -217,7 +252,8 @@ def run_ours(args, w, rank, world, dev):
     with torch.cuda.graph(graph, stream=stream):
         for i in range(K):
             step(W + i, evs[i])
-    graph.replay()                   # one untimed replay (the graph's own upload)
+    with torch.cuda.stream(stream):
+        graph.replay()               # one untimed replay (the graph's own upload)
     torch.cuda.synchronize(dev)
 
     bus = None
@@ -232,27 +268,26 @@ def run_ours(args, w, rank, world, dev):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    t0.record(stream)
-    graph.replay()
-    t1.record(stream)
+    with torch.cuda.stream(stream):  # replay on the stream the events are recorded on
+        t0.record(stream)
+        graph.replay()
+        t1.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
     ms = t0.elapsed_time(t1)
     kern_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, dev)
     del graph
 
     # ---- e2e: one decode step through the API with host buffers -----------------------
     e2e = run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, ws, stream, dev, torch,
                   api, synth, world, dist)
 
-    value = world * K * total_T / (ms_max / 1e3)
+    value = job_throughput(world, K, total_T, ms_max)
     peak, peak_kind = measured_peaks()
+    kname, launches_per_step = main_kernel(api, cfg, args.algo)
     achieved = code_bytes / (kern_ms / 1e3) / 1e9
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
@@ -268,11 +303,11 @@ def run_ours(args, w, rank, world, dev):
         "compressed_cache_gbs": code_bytes * K / (ms_max / 1e3) / 1e9 * 1.0 / world * world,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
-                     "kernel": "attend_table_kernel", "algorithmic_bytes_per_launch": code_bytes,
+                     "kernel": kname, "algorithmic_bytes_per_launch": code_bytes,
                      "kernel_ms_mean": kern_ms,
-                     "traffic": recorded_traffic("attend_table_kernel", w.name)},
+                     "traffic": recorded_traffic(kname, w.name)},
         "e2e": e2e,
-        "gpu_launches": 2 * K,
+        "gpu_launches": launches_per_step * K,
         "clocks": clk,
     }
     return result
@@ -325,13 +360,9 @@ def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, ws, stream, 
         graph.replay()
         t1.record(stream)
         torch.cuda.synchronize(dev)
-    ms = t0.elapsed_time(t1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     del graph
-    return {"value": world * K * total_T / (ms / 1e3), "unit": UNIT,
+    return {"value": job_throughput(world, K, total_T, ms), "unit": UNIT,
             "h2d_bytes_per_step": int(q_h.numel() * q_h.element_size() + kv_h.numel() * kv_h.element_size()),
             "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()),
             "ms_per_step": ms / K,

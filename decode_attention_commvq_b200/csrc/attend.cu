@@ -32,36 +32,123 @@ constexpr size_t kHeaderBytes = 256;   // device error word + padding
 
 // Split-T merge (flash-decoding style log-sum-exp combine of the per-split partials):
 // out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, lse = (M + log2 L) ln 2.
-__global__ void __launch_bounds__(kD) combine_kernel(AttendArgs a, int S) {
+// One block per (sequence, head). The split weights are formed once in shared memory; then
+// each warp adds every 8th split's 128-float partial with one float4 per lane, so all the
+// block's loads are in flight together, and the 8 warp sums are added in a fixed order.
+constexpr int kCombineThreads = 256;
+constexpr int kMaxSplits = 4096;
+
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(AttendArgs a, int S) {
+  __shared__ float wts[kMaxSplits];
+  __shared__ float4 acc_s[kCombineThreads / 32][32];
+  __shared__ float red[kCombineThreads / 32];
   const int bh = blockIdx.x;
-  const int dim = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const Partial* p = a.partials + static_cast<int64_t>(bh) * S;
+
   float M = -INFINITY;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, p[s].m);
-  float L = 0.0f, acc = 0.0f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < S; ++s) {
-      const float w = exp2f(p[s].m - M);
-      L = fmaf(w, p[s].l, L);
-      acc = fmaf(w, p[s].o[dim], acc);
-    }
+  for (int s = tid; s < S; s += kCombineThreads) M = fmaxf(M, p[s].m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  M = red[0];
+#pragma unroll
+  for (int w = 1; w < kCombineThreads / 32; ++w) M = fmaxf(M, red[w]);
+  __syncthreads();
+
+  float L = 0.0f;
+  for (int s = tid; s < S; s += kCombineThreads) {
+    const float w = (M == -INFINITY) ? 0.0f : exp2f(p[s].m - M);
+    wts[s] = w;
+    L = fmaf(w, p[s].l, L);
   }
-  a.out[static_cast<int64_t>(bh) * kD + dim] = L > 0.0f ? acc / L : 0.0f;
-  if (a.lse && dim == 0)
-    a.lse[bh] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  if (lane == 0) red[warp] = L;
+  __syncthreads();
+  L = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kCombineThreads / 32; ++w) L += red[w];
+
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int s = warp; s < S; s += kCombineThreads / 32) {
+    const float w = wts[s];
+    const float4 o = reinterpret_cast<const float4*>(p[s].o)[lane];
+    acc.x = fmaf(w, o.x, acc.x);
+    acc.y = fmaf(w, o.y, acc.y);
+    acc.z = fmaf(w, o.z, acc.z);
+    acc.w = fmaf(w, o.w, acc.w);
+  }
+  acc_s[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float4 t = acc_s[0][lane];
+#pragma unroll
+    for (int w = 1; w < kCombineThreads / 32; ++w) {
+      const float4 u = acc_s[w][lane];
+      t.x += u.x;
+      t.y += u.y;
+      t.z += u.z;
+      t.w += u.w;
+    }
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    reinterpret_cast<float4*>(a.out + static_cast<int64_t>(bh) * kD)[lane] =
+        make_float4(t.x * inv, t.y * inv, t.z * inv, t.w * inv);
+    if (a.lse && lane == 0)
+      a.lse[bh] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+  }
 }
 
-int choose_splits(int B, int q_heads, int64_t max_T, const commvq_attend_options* opt) {
+// Algorithm actually run for a request (AUTO -> decode-and-rotate when it supports the shape).
+int resolve_algo(const commvq_config* cfg, const commvq_attend_options* opt) {
+  const int algo = opt ? opt->algo : COMMVQ_ATTN_AUTO;
+  if (algo != COMMVQ_ATTN_AUTO) return algo;
+  return mma_supported(cfg->R, cfg->q_heads, cfg->kv_heads, cfg->n_codes) ? COMMVQ_ATTN_DECODE_MMA
+                                                                          : COMMVQ_ATTN_TABLE;
+}
+
+// Split-T partitions per sequence. Table form: one CTA per (sequence, query head, split);
+// decode-and-rotate form: one CTA per (sequence, split) covering every head. Both aim at
+// one wave of CTAs on the SMs.
+int choose_splits(int algo, int B, int q_heads, int64_t max_T, const commvq_attend_options* opt) {
   if (opt && opt->splits > 0) return opt->splits;
   const DeviceInfo di = current_device_info();
   const int sms = di.sms > 0 ? di.sms : 148;
-  const int64_t units = static_cast<int64_t>(B) * q_heads;
-  int64_t S = units >= sms ? 1 : sms / units;
-  const int64_t by_len = (max_T + 511) / 512;
-  if (S > by_len) S = by_len;
+  int64_t S;
+  if (algo == COMMVQ_ATTN_DECODE_MMA) {
+    S = B >= sms ? 1 : sms / B;
+    const int64_t by_len = (max_T + 15) / 16;
+    if (S > by_len) S = by_len;
+  } else {
+    const int64_t units = static_cast<int64_t>(B) * q_heads;
+    S = units >= sms ? 1 : sms / units;
+    const int64_t by_len = (max_T + 511) / 512;
+    if (S > by_len) S = by_len;
+  }
   if (S < 1) S = 1;
-  if (S > 4096) S = 4096;
+  if (S > kMaxSplits) S = kMaxSplits;
   return static_cast<int>(S);
+}
+
+struct WorkspaceLayout {
+  size_t partials_off, kimg_off, vimg_off, scores_off, total;
+};
+
+WorkspaceLayout workspace_layout(const commvq_config* cfg, int algo, int B, int64_t max_T, int S) {
+  WorkspaceLayout L{};
+  L.partials_off = kHeaderBytes;
+  size_t end = L.partials_off + static_cast<size_t>(B) * cfg->q_heads * S * sizeof(Partial);
+  if (algo == COMMVQ_ATTN_DECODE_MMA) {
+    const size_t img = static_cast<size_t>(512) * cfg->n_codes;
+    L.kimg_off = round_up(end, 256);
+    L.vimg_off = round_up(L.kimg_off + img, 256);
+    L.scores_off = round_up(L.vimg_off + img, 256);
+    end = L.scores_off + static_cast<size_t>(B) * ((max_T + 15) / 16 * 16) * cfg->q_heads * sizeof(float);
+  }
+  L.total = round_up(end, 256);
+  return L;
 }
 
 // Shape checks shared by the workspace query and the call. Returns OK, INVALID or UNSUPPORTED.
@@ -86,8 +173,13 @@ using namespace commvq;
 extern "C" size_t commvq_attend_workspace_bytes(const commvq_config* cfg, int32_t B, int64_t max_T,
                                                 const commvq_attend_options* options) {
   if (check_config(cfg) != COMMVQ_OK || B < 0 || max_T < 0) return 0;
-  const int S = choose_splits(B > 0 ? B : 1, cfg->q_heads, max_T, options);
-  return kHeaderBytes + static_cast<size_t>(B) * cfg->q_heads * S * sizeof(Partial);
+  if (options && (options->splits < 0 || options->splits > kMaxSplits || options->algo < 0 || options->algo > 2))
+    return 0;
+  const int algo = resolve_algo(cfg, options);
+  if (algo == COMMVQ_ATTN_DECODE_MMA && !mma_supported(cfg->R, cfg->q_heads, cfg->kv_heads, cfg->n_codes))
+    return 0;
+  const int S = choose_splits(algo, B > 0 ? B : 1, cfg->q_heads, max_T, options);
+  return workspace_layout(cfg, algo, B, max_T, S).total;
 }
 
 extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const void* q,
@@ -103,7 +195,7 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
   if (q_dtype != COMMVQ_F32 && q_dtype != COMMVQ_F16 && q_dtype != COMMVQ_BF16)
     return COMMVQ_ERR_INVALID_ARG;
   const int algo = options ? options->algo : COMMVQ_ATTN_AUTO;
-  if (options && (options->splits < 0 || options->splits > 65535)) return COMMVQ_ERR_INVALID_ARG;
+  if (options && (options->splits < 0 || options->splits > kMaxSplits)) return COMMVQ_ERR_INVALID_ARG;
   if (algo != COMMVQ_ATTN_AUTO && algo != COMMVQ_ATTN_TABLE && algo != COMMVQ_ATTN_DECODE_MMA)
     return COMMVQ_ERR_INVALID_ARG;
   if (B == 0) return COMMVQ_OK;
@@ -114,16 +206,27 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
       !aligned(v_codebook, 16) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(seq_offsets, 8) ||
       !aligned(workspace, 256))
     return COMMVQ_ERR_INVALID_ARG;
+  if (algo == COMMVQ_ATTN_DECODE_MMA && !mma_supported(cfg->R, cfg->q_heads, cfg->kv_heads, cfg->n_codes))
+    return COMMVQ_ERR_UNSUPPORTED;
   const size_t need = commvq_attend_workspace_bytes(cfg, B, max_T, options);
   if (need == 0 || workspace_bytes < need) return COMMVQ_ERR_WORKSPACE;
 
   const DeviceInfo di = current_device_info();
   if (di.device < 0) return COMMVQ_ERR_CUDA;
-  if (algo == COMMVQ_ATTN_DECODE_MMA) return COMMVQ_ERR_UNSUPPORTED;
-  if (table_smem_bytes(cfg->R, cfg->n_codes) > di.smem_optin) return COMMVQ_ERR_UNSUPPORTED;
+  const int run = resolve_algo(cfg, options);
+  if (run == COMMVQ_ATTN_DECODE_MMA) {
+    if (!mma_supported(cfg->R, cfg->q_heads, cfg->kv_heads, cfg->n_codes)) return COMMVQ_ERR_UNSUPPORTED;
+    if (mma_scores_smem_bytes(cfg->R, cfg->kv_heads, cfg->n_codes) > di.smem_optin ||
+        mma_values_smem_bytes(cfg->R, cfg->kv_heads, cfg->q_heads, cfg->n_codes) > di.smem_optin)
+      return COMMVQ_ERR_UNSUPPORTED;
+  } else if (table_smem_bytes(cfg->R, cfg->n_codes) > di.smem_optin) {
+    return COMMVQ_ERR_UNSUPPORTED;
+  }
 
-  const int S = choose_splits(B, cfg->q_heads, max_T, options);
-  AttendArgs a;
+  const int S = choose_splits(run, B, cfg->q_heads, max_T, options);
+  const WorkspaceLayout L = workspace_layout(cfg, run, B, max_T, S);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  AttendArgs a{};
   a.k_codes = static_cast<const uint8_t*>(k_codes);
   a.v_codes = static_cast<const uint8_t*>(v_codes);
   a.seq_offsets = seq_offsets;
@@ -132,7 +235,14 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
   a.out = out;
   a.lse = lse;
   a.error_word = static_cast<int*>(workspace);
-  a.partials = reinterpret_cast<Partial*>(static_cast<unsigned char*>(workspace) + kHeaderBytes);
+  a.partials = reinterpret_cast<Partial*>(ws + L.partials_off);
+  if (run == COMMVQ_ATTN_DECODE_MMA) {
+    a.k_img = reinterpret_cast<const uint4*>(ws + L.kimg_off);
+    a.v_img = reinterpret_cast<const uint4*>(ws + L.vimg_off);
+    a.scores = reinterpret_cast<float*>(ws + L.scores_off);
+  }
+  a.main_start = options ? options->main_start : nullptr;
+  a.main_stop = options ? options->main_stop : nullptr;
   a.max_T = max_T;
   a.rope_base = cfg->rope_base;
   a.B = B;
@@ -143,23 +253,27 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(a.error_word, 0, sizeof(int), st) != cudaSuccess) return COMMVQ_ERR_CUDA;
-  // External records so the events keep their timestamps inside a captured CUDA graph too.
-  if (options && options->main_start &&
-      cudaEventRecordWithFlags(static_cast<cudaEvent_t>(options->main_start), st,
-                               cudaEventRecordExternal) != cudaSuccess)
-    return COMMVQ_ERR_CUDA;
-  commvq_status rc = launch_attend_table(a, q, q_dtype, S, st);
+  commvq_status rc;
+  if (run == COMMVQ_ATTN_DECODE_MMA) {
+    rc = launch_attend_mma(a, q, q_dtype, S, st);
+  } else {
+    // External records so the events keep their timestamps inside a captured CUDA graph too.
+    if (a.main_start && cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a.main_start), st,
+                                                 cudaEventRecordExternal) != cudaSuccess)
+      return COMMVQ_ERR_CUDA;
+    rc = launch_attend_table(a, q, q_dtype, S, st);
+    if (rc == COMMVQ_OK && a.main_stop &&
+        cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a.main_stop), st, cudaEventRecordExternal) !=
+            cudaSuccess)
+      return COMMVQ_ERR_CUDA;
+  }
   if (rc != COMMVQ_OK) return rc;
-  if (options && options->main_stop &&
-      cudaEventRecordWithFlags(static_cast<cudaEvent_t>(options->main_stop), st,
-                               cudaEventRecordExternal) != cudaSuccess)
-    return COMMVQ_ERR_CUDA;
   return launch_combine(a, S, st);
 }
 
 namespace commvq {
 commvq_status launch_combine(const AttendArgs& a, int S, cudaStream_t st) {
-  combine_kernel<<<a.B * a.q_heads, kD, 0, st>>>(a, S);
+  combine_kernel<<<a.B * a.q_heads, kCombineThreads, 0, st>>>(a, S);
   return launch_status();
 }
 }  // namespace commvq

@@ -25,6 +25,11 @@ struct AttendArgs {
   float* lse;
   Partial* partials;
   int* error_word;
+  float* scores;          // decode-and-rotate form: tile-blocked exp2-domain scores
+  const uint4* k_img;     // decode-and-rotate form: fp16 codebook images (see attend_mma.cu)
+  const uint4* v_img;
+  void* main_start;       // optional cudaEvent_t pair around the main kernel(s)
+  void* main_stop;
   int64_t max_T;
   double rope_base;
   int B;
@@ -35,6 +40,11 @@ struct AttendArgs {
 };
 
 size_t table_smem_bytes(int R, int n_codes);
+size_t mma_scores_smem_bytes(int R, int KV, int n_codes);
+size_t mma_values_smem_bytes(int R, int KV, int q_heads, int n_codes);
+bool mma_supported(int R, int q_heads, int kv_heads, int n_codes);
+commvq_status launch_attend_mma(const AttendArgs& a, const void* q, commvq_dtype qt, int splits,
+                                cudaStream_t st);
 commvq_status launch_attend_table(const AttendArgs& a, const void* q, commvq_dtype qt, int splits,
                                   cudaStream_t st);
 commvq_status launch_combine(const AttendArgs& a, int splits, cudaStream_t st);

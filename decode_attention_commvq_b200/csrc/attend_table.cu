@@ -61,6 +61,8 @@ attend_table_kernel(AttendArgs a, const QT* __restrict__ q) {
   float* sc = hist + static_cast<size_t>(R) * Nc * kGroups;                      // kChunk
   float* qs = sc + kChunk;                                                       // kD
   float* red = qs + kD;                                                          // 2 * 8
+  uint8_t* kbuf = reinterpret_cast<uint8_t*>(red + 16);        // [2][kChunk][R][16] key codes
+  uint8_t* vbuf = kbuf + 2 * kChunk * R * kGroups;             // [2][kChunk][R][16] value codes
 
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int S = gridDim.x;
@@ -114,17 +116,41 @@ attend_table_kernel(AttendArgs a, const QT* __restrict__ q) {
 #pragma unroll
   for (int i = 0; i < kPairs; ++i)
     theta[i] = pow(a.rope_base, -2.0 * static_cast<double>(j * kPairs + i) / kD);
-  const uint8_t* kc = a.k_codes;
-  const uint8_t* vc = a.v_codes;
   const int64_t code_row = static_cast<int64_t>(a.kv_heads) * R * kGroups;  // bytes per position
+  const uint8_t* kc = a.k_codes + row0 * code_row + static_cast<int64_t>(kvh) * R * kGroups;
+  const uint8_t* vc = a.v_codes + row0 * code_row + static_cast<int64_t>(kvh) * R * kGroups;
   int err = 0;
+
+  // Prefetch of one chunk's key and value codes (R 16-byte pieces per position and tensor).
+  auto issue = [&](int64_t c0, int stage) {
+    const int n = static_cast<int>(min(static_cast<int64_t>(kChunk), t_end - c0));
+    const int pieces = n * R;
+    for (int p = tid; p < 2 * pieces; p += kThreads) {
+      const int tensor = p >= pieces;
+      const int qp = p - tensor * pieces;
+      const int t = qp / R, r = qp - (qp / R) * R;
+      const uint8_t* src = (tensor ? vc : kc) + (c0 + t) * code_row + r * kGroups;
+      uint8_t* dst = (tensor ? vbuf : kbuf) + ((stage * kChunk + t) * R + r) * kGroups;
+      cp_async16(dst, src);
+    }
+    cp_async_commit();
+  };
 
   float m_run = -INFINITY;   // running max (exp2 domain)
   float l_run = 0.0f;        // this thread's share of the running sum
-  __syncthreads();
+  issue(t_begin, 0);
+  int stage = 0;
 
-  for (int64_t c0 = t_begin; c0 < t_end; c0 += kChunk) {
+  for (int64_t c0 = t_begin; c0 < t_end; c0 += kChunk, stage ^= 1) {
     const int n = static_cast<int>(min(static_cast<int64_t>(kChunk), t_end - c0));
+    if (c0 + kChunk < t_end)
+      issue(c0 + kChunk, stage ^ 1);
+    else
+      cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    const uint8_t* kchunk = kbuf + stage * kChunk * R * kGroups;
+    const uint8_t* vchunk = vbuf + stage * kChunk * R * kGroups;
 
     // ---- 2. scores of this chunk ----------------------------------------------------------
 #pragma unroll 2
@@ -133,7 +159,7 @@ attend_table_kernel(AttendArgs a, const QT* __restrict__ q) {
       float part_s = 0.0f;
       if (tl < n) {
         const int64_t t = c0 + tl;
-        const uint8_t* cp = kc + (row0 + t) * code_row + static_cast<int64_t>(kvh) * R * kGroups + j;
+        const uint8_t* cp = kchunk + tl * R * kGroups + j;
         float U[kPairs] = {0.f, 0.f, 0.f, 0.f}, W[kPairs] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int r = 0; r < R; ++r) {
@@ -198,9 +224,8 @@ attend_table_kernel(AttendArgs a, const QT* __restrict__ q) {
     for (int step = 0; step < 16; ++step) {
       const int tl = warp * 32 + step * 2 + slot;
       if (tl < n) {
-        const int64_t t = c0 + tl;
         const float p = sc[tl];
-        const uint8_t* cp = vc + (row0 + t) * code_row + static_cast<int64_t>(kvh) * R * kGroups + j;
+        const uint8_t* cp = vchunk + tl * R * kGroups + j;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           int code = cp[r * kGroups];
@@ -286,7 +311,7 @@ commvq_status launch_table_c(const AttendArgs& a, const void* q, commvq_dtype qt
 
 size_t table_smem_bytes(int R, int n_codes) {
   return static_cast<size_t>(R) * n_codes * (2 * 8 * 16 + kGroups * 4) +
-         (kChunk + kD + 16) * sizeof(float);
+         (kChunk + kD + 16) * sizeof(float) + static_cast<size_t>(4) * kChunk * R * kGroups;
 }
 
 commvq_status launch_attend_table(const AttendArgs& a, const void* q, commvq_dtype qt, int splits,

@@ -108,4 +108,16 @@ __device__ __forceinline__ void store_code(void* codes, int64_t at, int code, in
     static_cast<uint16_t*>(codes)[at] = static_cast<uint16_t>(code);
 }
 
+// Ampere-style asynchronous 16-byte global -> shared copies (bypass L1), used to prefetch
+// code chunks one step ahead of the compute that consumes them.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
 }  // namespace commvq

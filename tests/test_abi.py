@@ -89,9 +89,20 @@ def test_attend_rejects_bad_arguments(api):
 
 def test_workspace_sizes(api):
     cfg = _cfg(api)
-    one = api.attend_workspace_bytes(cfg, 1, 32768, splits=4)
+    one = api.attend_workspace_bytes(cfg, 1, 32768, algo=api.ATTN_TABLE, splits=4)
     assert one == 256 + 32 * 4 * 528
-    assert api.attend_workspace_bytes(cfg, 16, 8192, splits=1) == 256 + 16 * 32 * 528
+    assert api.attend_workspace_bytes(cfg, 16, 8192, algo=api.ATTN_TABLE, splits=1) == 256 + 16 * 32 * 528
+    # decode-and-rotate form: partials, two fp16 codebook images, the score buffer
+    mma = api.attend_workspace_bytes(cfg, 1, 32768, algo=api.ATTN_DECODE_MMA, splits=148)
+    part = 256 + 32 * 148 * 528
+    img = 512 * 256
+    want = -(-part // 256) * 256 + 2 * img + 32768 * 32 * 4
+    assert mma == -(-want // 256) * 256
+    assert api.attend_workspace_bytes(cfg, 1, 32768) == api.attend_workspace_bytes(
+        cfg, 1, 32768, algo=api.ATTN_DECODE_MMA)
+    # shapes the decode-and-rotate form does not take
+    assert api.attend_workspace_bytes(_cfg(api, R=3, n_codes=64), 1, 10, algo=api.ATTN_DECODE_MMA) == 0
+    assert api.attend_workspace_bytes(_cfg(api, R=3, n_codes=64), 1, 10) > 0   # AUTO -> table
     assert api.attend_workspace_bytes(_cfg(api, q_heads=30), 1, 10) == 0
     em = api.em_workspace_bytes(cfg, 65536)
     assert em >= 32 * 16 * 256 * (8 * 8 + 4)

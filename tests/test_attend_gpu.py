@@ -11,7 +11,7 @@ from tests.helpers import oracle_codebooks, q_as_f64, rel_err, to_torch_q, tol_f
 
 pytestmark = pytest.mark.gpu
 
-ALGOS = [1]   # table path
+ALGOS = [1, 2]   # table path, decode-and-rotate path
 
 
 @pytest.fixture(scope="module")
@@ -125,8 +125,12 @@ def test_split_count_invariance(api, gpu, algo):
     q = synth.queries(w)
     offs = w.offsets()
     outs = [_run(api, w, q, kc, vc, offs, kcb, vcb, gpu, algo, s)[0] for s in (1, 2, 5, 16)]
+    # The table path keeps softmax weights in fp32, so splits change only fp32 rounding. The
+    # decode-and-rotate path feeds the weights to the tensor cores in fp16 relative to each
+    # split's own maximum (rounding up to 2^-11 relative), so its bound is fp16's.
+    bound = 1e-5 if algo == 1 else 1e-3
     for o in outs[1:]:
-        assert rel_err(o, outs[0]) <= 1e-5
+        assert rel_err(o, outs[0]) <= bound
 
 
 @pytest.mark.parametrize("algo", ALGOS)
@@ -153,22 +157,27 @@ def test_degenerate_lengths(api, gpu, algo):
         assert np.allclose(out[1, h], vhat[h // 4], rtol=1e-3, atol=1e-3)
 
 
-def test_zero_query_gives_mean_value(api, gpu):
+@pytest.mark.parametrize("algo", ALGOS)
+def test_zero_query_gives_mean_value(api, gpu, algo):
     w = synth.WORKLOADS[1].with_(seq_len=777)
     kcb, vcb = oracle_codebooks(synth.WORKLOADS[1])
     offs = w.offsets()
     kc = synth.uniform_codes(w, True, 777)
     vc = synth.uniform_codes(w, False, 777)
     q = np.zeros((1, w.q_heads, w.d), dtype=np.uint16)    # bf16 zeros
-    out, lse = _run(api, w, q, kc, vc, offs, kcb, vcb, gpu)
+    out, lse = _run(api, w, q, kc, vc, offs, kcb, vcb, gpu, algo)
     vhat = O.decode(vc, vcb)                               # [T, Hkv, d]
     mean = vhat.mean(0)
+    # table path: fp32 value codebook; decode-and-rotate path: fp16 codebook entries
+    # (2^-12 relative rounding each, fixed per entry)
+    bound = 1e-4 if algo == 1 else 2e-3
     for h in range(w.q_heads):
-        assert rel_err(out[0, h], mean[h // 4]) <= 1e-4
+        assert rel_err(out[0, h], mean[h // 4]) <= bound
     assert np.allclose(lse, np.log(777), rtol=1e-5)
 
 
-def test_out_of_range_codes_are_flagged_not_trapped(api, gpu):
+@pytest.mark.parametrize("algo", ALGOS)
+def test_out_of_range_codes_are_flagged_not_trapped(api, gpu, algo):
     """Nc' = 16 with uint8 codes: a code >= 16 is clamped to 15 and recorded in the
     workspace error word; the call itself completes."""
     w = synth.WORKLOADS[0]
@@ -177,18 +186,20 @@ def test_out_of_range_codes_are_flagged_not_trapped(api, gpu):
     kc = synth.uniform_codes(w, True, 256)
     vc = synth.uniform_codes(w, False, 256)
     kc[17, 0, 0, 3] = 200
+    vc[40, 0, 0, 9] = 16
     q = to_torch_q(synth.queries(w), w.q_dtype, gpu)
     offs = torch.tensor([0, 256], dtype=torch.int64, device=gpu)
-    ws = api.attend_workspace(cfg, 1, 256, gpu)
+    ws = api.attend_workspace(cfg, 1, 256, gpu, algo=algo)
     out, _ = api.attend_decode(cfg, q, _codes_np_to_gpu(kc, gpu), _codes_np_to_gpu(vc, gpu), offs, 256,
                                torch.from_numpy(kcb).to(gpu), torch.from_numpy(vcb).to(gpu),
-                               workspace=ws)
+                               workspace=ws, algo=algo)
     assert api.workspace_error(ws) == 1
-    kc2 = kc.copy()
+    kc2, vc2 = kc.copy(), vc.copy()
     kc2[17, 0, 0, 3] = 15
-    out2, _ = api.attend_decode(cfg, q, _codes_np_to_gpu(kc2, gpu), _codes_np_to_gpu(vc, gpu), offs,
+    vc2[40, 0, 0, 9] = 15
+    out2, _ = api.attend_decode(cfg, q, _codes_np_to_gpu(kc2, gpu), _codes_np_to_gpu(vc2, gpu), offs,
                                 256, torch.from_numpy(kcb).to(gpu), torch.from_numpy(vcb).to(gpu),
-                                workspace=ws)
+                                workspace=ws, algo=algo)
     assert api.workspace_error(ws) == 0
     # value histograms accumulate with shared-memory float atomics: equal up to rounding order
     assert rel_err(out.cpu().numpy(), out2.cpu().numpy()) <= 1e-6
