@@ -22,8 +22,8 @@ ATTN_AUTO, ATTN_TABLE, ATTN_DECODE_MMA = 0, 1, 2
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "WORKSPACE", 5: "DEVICE_CHECK"}
 
 EXPORTS = ("commvq_encode", "commvq_attend_workspace_bytes", "commvq_attend_decode",
-           "commvq_em_workspace_bytes", "commvq_em_step", "commvq_workspace_error",
-           "commvq_status_string", "commvq_abi_version")
+           "commvq_attend_decode_noalloc", "commvq_em_workspace_bytes", "commvq_em_step",
+           "commvq_workspace_error", "commvq_status_string", "commvq_abi_version")
 
 
 class CConfig(ctypes.Structure):
@@ -58,6 +58,8 @@ def _load():
     lib.commvq_attend_workspace_bytes.restype = SZ
     lib.commvq_attend_decode.argtypes = [CP, P, I32, P, P, P, I32, I64, P, P, P, P, P, SZ, OP, P]
     lib.commvq_attend_decode.restype = I32
+    lib.commvq_attend_decode_noalloc.argtypes = [CP, P, I32, P, P, P, I32, I64, P, P, P, P, OP, P]
+    lib.commvq_attend_decode_noalloc.restype = I32
     lib.commvq_em_workspace_bytes.argtypes = [CP, I64]
     lib.commvq_em_workspace_bytes.restype = SZ
     lib.commvq_em_step.argtypes = [CP, P, I64, P, P, P, P, SZ, P]
@@ -180,6 +182,22 @@ def attend_decode(cfg: Config, q: torch.Tensor, k_codes: torch.Tensor, v_codes: 
                                     _ptr(k_codebook), _ptr(v_codebook), _ptr(out), _ptr(lse),
                                     _ptr(workspace), workspace.numel(), ctypes.byref(o),
                                     _stream(stream)), "commvq_attend_decode")
+    return out, lse
+
+
+def attend_decode_noalloc(cfg: Config, q: torch.Tensor, k_codes: torch.Tensor, v_codes: torch.Tensor,
+                          seq_offsets: torch.Tensor, max_T: int, k_codebook: torch.Tensor,
+                          v_codebook: torch.Tensor, out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                          algo: int = ATTN_AUTO, splits: int = 0, stream=None):
+    """commvq_attend_decode_noalloc: the library's fixed internal scratch instead of a
+    workspace (for callers that cannot allocate device memory). out/lse are caller-owned."""
+    cc = cfg.c()
+    o = _opts(algo, splits)
+    _check(LIB.commvq_attend_decode_noalloc(ctypes.byref(cc), _ptr(q), _DT[q.dtype], _ptr(k_codes),
+                                            _ptr(v_codes), _ptr(seq_offsets), int(q.shape[0]),
+                                            int(max_T), _ptr(k_codebook), _ptr(v_codebook), _ptr(out),
+                                            _ptr(lse), ctypes.byref(o), _stream(stream)),
+           "commvq_attend_decode_noalloc")
     return out, lse
 
 

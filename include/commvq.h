@@ -148,6 +148,32 @@ commvq_status commvq_attend_decode(const commvq_config* cfg, const void* q, comm
                                    size_t workspace_bytes, const commvq_attend_options* options,
                                    void* stream);
 
+/* commvq_attend_decode for callers that cannot allocate device memory -- for example a
+ * plugin inside a host framework that owns the device allocator, or a latency-critical loop
+ * where a cudaMalloc (which may synchronise the device) is not allowed. This call has no
+ * counterpart in the paper; it is a packaging variant of commvq_attend_decode.
+ * Arguments and results are those of commvq_attend_decode without workspace/workspace_bytes:
+ * the workspace is a fixed 32 MiB device array inside the library (every GPU that loads the
+ * library holds it until the process exits). No cudaMalloc, cudaFree or other allocating
+ * routine is called.
+ * - Limit: a request whose commvq_attend_workspace_bytes exceeds 32 MiB returns
+ *   COMMVQ_ERR_WORKSPACE without launching. (The 2-bit 32K layer needs ~7 MiB; the 1-bit
+ *   128K layer and a batch of 16 sequences of up to 8192 positions need ~19-20 MiB.)
+ * - Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call before any
+ *   stream capture.
+ * - Sharing: all calls on a device use the same array and it keeps the last call's
+ *   contents. Each call rewrites everything it reads, so results do not depend on earlier
+ *   calls, but calls that overlap on the GPU (different streams without ordering) race.
+ * - Device data checks: codes >= Nc' are still clamped, but the error word lives in the
+ *   internal array and is not reported by this entry point. */
+commvq_status commvq_attend_decode_noalloc(const commvq_config* cfg, const void* q,
+                                           commvq_dtype q_dtype, const void* k_codes,
+                                           const void* v_codes, const int64_t* seq_offsets,
+                                           int32_t B, int64_t max_T, const float* k_codebook,
+                                           const float* v_codebook, float* out, float* lse,
+                                           const commvq_attend_options* options, void* stream);
+
 /* Bytes of device workspace commvq_em_step needs for N rows. 0 for invalid input. */
 size_t commvq_em_workspace_bytes(const commvq_config* cfg, int64_t N);
 
