@@ -32,18 +32,21 @@ constexpr size_t kHeaderBytes = 256;   // device error word + padding
 
 // Split-T merge (flash-decoding style log-sum-exp combine of the per-split partials):
 // out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, lse = (M + log2 L) ln 2.
-// One block per (sequence, head). The split weights are formed once in shared memory; then
-// each warp adds every 8th split's 128-float partial with one float4 per lane, so all the
-// block's loads are in flight together, and the 8 warp sums are added in a fixed order.
+// Grid: (sequence x head, 4 quarters of the 128 output dims). Every block forms the split
+// weights in shared memory; then each of its 32 eight-lane groups adds every 32nd split's
+// 32-dim slice (one float4 per lane, all loads of a group issued together), and the 32
+// group sums are added in a fixed order.
 constexpr int kCombineThreads = 256;
+constexpr int kCombineQuarters = 4;
 constexpr int kMaxSplits = 4096;
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(AttendArgs a, int S) {
   __shared__ float wts[kMaxSplits];
-  __shared__ float4 acc_s[kCombineThreads / 32][32];
+  __shared__ float4 acc_s[kCombineThreads / 8][8];
   __shared__ float red[kCombineThreads / 32];
-  const int bh = blockIdx.x;
+  const int bh = blockIdx.x, quarter = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int grp = tid >> 3, gl = tid & 7;            // 32 groups of 8 lanes; lane gl -> 4 dims
   const Partial* p = a.partials + static_cast<int64_t>(bh) * S;
 
   float M = -INFINITY;
@@ -71,32 +74,41 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(AttendArgs a, 
 #pragma unroll
   for (int w = 0; w < kCombineThreads / 32; ++w) L += red[w];
 
+  constexpr int kGroupsPerBlock = kCombineThreads / 8;
+  const int dim4 = quarter * 8 + gl;                  // float4 index within o[128]
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int s = warp; s < S; s += kCombineThreads / 32) {
-    const float w = wts[s];
-    const float4 o = reinterpret_cast<const float4*>(p[s].o)[lane];
-    acc.x = fmaf(w, o.x, acc.x);
-    acc.y = fmaf(w, o.y, acc.y);
-    acc.z = fmaf(w, o.z, acc.z);
-    acc.w = fmaf(w, o.w, acc.w);
-  }
-  acc_s[warp][lane] = acc;
-  __syncthreads();
-  if (warp == 0) {
-    float4 t = acc_s[0][lane];
+  for (int s0 = grp; s0 < S; s0 += kGroupsPerBlock * 8) {
+    float4 o[8];
+    float w[8];
 #pragma unroll
-    for (int w = 1; w < kCombineThreads / 32; ++w) {
-      const float4 u = acc_s[w][lane];
+    for (int k = 0; k < 8; ++k) {
+      const int s = s0 + k * kGroupsPerBlock;
+      w[k] = s < S ? wts[s] : 0.0f;
+      o[k] = s < S ? reinterpret_cast<const float4*>(p[s].o)[dim4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      acc.x = fmaf(w[k], o[k].x, acc.x);
+      acc.y = fmaf(w[k], o[k].y, acc.y);
+      acc.z = fmaf(w[k], o[k].z, acc.z);
+      acc.w = fmaf(w[k], o[k].w, acc.w);
+    }
+  }
+  acc_s[grp][gl] = acc;
+  __syncthreads();
+  if (tid < 8) {
+    float4 t = acc_s[0][tid];
+    for (int g2 = 1; g2 < kGroupsPerBlock; ++g2) {
+      const float4 u = acc_s[g2][tid];
       t.x += u.x;
       t.y += u.y;
       t.z += u.z;
       t.w += u.w;
     }
     const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-    reinterpret_cast<float4*>(a.out + static_cast<int64_t>(bh) * kD)[lane] =
+    reinterpret_cast<float4*>(a.out + static_cast<int64_t>(bh) * kD)[quarter * 8 + tid] =
         make_float4(t.x * inv, t.y * inv, t.z * inv, t.w * inv);
-    if (a.lse && lane == 0)
+    if (a.lse && quarter == 0 && tid == 0)
       a.lse[bh] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
   }
 }
@@ -133,8 +145,9 @@ int choose_splits(int algo, int B, int q_heads, int64_t max_T, const commvq_atte
 }
 
 struct WorkspaceLayout {
-  size_t partials_off, kimg_off, vimg_off, scores_off, total;
+  size_t partials_off, kimg_off, vimg_off, phase_off, qfrag_off, base_off, scores_off, total;
 };
+constexpr size_t kPhaseBytes = 64 * sizeof(double) + 128 * 64 * 8 + 64 * 8;   // theta, rows, advance
 
 WorkspaceLayout workspace_layout(const commvq_config* cfg, int algo, int B, int64_t max_T, int S) {
   WorkspaceLayout L{};
@@ -144,7 +157,10 @@ WorkspaceLayout workspace_layout(const commvq_config* cfg, int algo, int B, int6
     const size_t img = static_cast<size_t>(512) * cfg->n_codes;
     L.kimg_off = round_up(end, 256);
     L.vimg_off = round_up(L.kimg_off + img, 256);
-    L.scores_off = round_up(L.vimg_off + img, 256);
+    L.phase_off = round_up(L.vimg_off + img, 256);
+    L.qfrag_off = round_up(L.phase_off + kPhaseBytes, 256);
+    L.base_off = round_up(L.qfrag_off + static_cast<size_t>(B) * cfg->kv_heads * 256 * 8, 256);
+    L.scores_off = round_up(L.base_off + static_cast<size_t>(B) * S * 64 * 8, 256);
     end = L.scores_off + static_cast<size_t>(B) * ((max_T + 15) / 16 * 16) * cfg->q_heads * sizeof(float);
   }
   L.total = round_up(end, 256);
@@ -240,6 +256,11 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
     a.k_img = reinterpret_cast<const uint4*>(ws + L.kimg_off);
     a.v_img = reinterpret_cast<const uint4*>(ws + L.vimg_off);
     a.scores = reinterpret_cast<float*>(ws + L.scores_off);
+    a.theta = reinterpret_cast<const double*>(ws + L.phase_off);
+    a.rowph = reinterpret_cast<const float2*>(ws + L.phase_off + 64 * sizeof(double));
+    a.advph = a.rowph + 128 * 64;
+    a.qfrag = reinterpret_cast<const uint2*>(ws + L.qfrag_off);
+    a.basetab = reinterpret_cast<const float2*>(ws + L.base_off);
   }
   a.main_start = options ? options->main_start : nullptr;
   a.main_stop = options ? options->main_stop : nullptr;
@@ -252,11 +273,11 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
   a.n_codes = cfg->n_codes;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(a.error_word, 0, sizeof(int), st) != cudaSuccess) return COMMVQ_ERR_CUDA;
   commvq_status rc;
   if (run == COMMVQ_ATTN_DECODE_MMA) {
-    rc = launch_attend_mma(a, q, q_dtype, S, st);
+    rc = launch_attend_mma(a, q, q_dtype, S, st);   // its prep kernel clears the error word
   } else {
+    if (cudaMemsetAsync(a.error_word, 0, sizeof(int), st) != cudaSuccess) return COMMVQ_ERR_CUDA;
     // External records so the events keep their timestamps inside a captured CUDA graph too.
     if (a.main_start && cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a.main_start), st,
                                                  cudaEventRecordExternal) != cudaSuccess)
@@ -273,7 +294,7 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
 
 namespace commvq {
 commvq_status launch_combine(const AttendArgs& a, int S, cudaStream_t st) {
-  combine_kernel<<<a.B * a.q_heads, kCombineThreads, 0, st>>>(a, S);
+  combine_kernel<<<dim3(a.B * a.q_heads, kCombineQuarters), kCombineThreads, 0, st>>>(a, S);
   return launch_status();
 }
 }  // namespace commvq

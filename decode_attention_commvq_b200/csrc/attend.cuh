@@ -28,6 +28,11 @@ struct AttendArgs {
   float* scores;          // decode-and-rotate form: tile-blocked exp2-domain scores
   const uint4* k_img;     // decode-and-rotate form: fp16 codebook images (see attend_mma.cu)
   const uint4* v_img;
+  const double* theta;    // decode-and-rotate form: RoPE tables written by its prep kernel
+  const float2* rowph;
+  const float2* advph;
+  const uint2* qfrag;     // decode-and-rotate form: per-call query fragments and split phasors
+  const float2* basetab;
   void* main_start;       // optional cudaEvent_t pair around the main kernel(s)
   void* main_stop;
   int64_t max_T;

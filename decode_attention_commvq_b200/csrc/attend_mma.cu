@@ -38,7 +38,7 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kTileT = 16;                 // positions per mma row block
 constexpr int kStageT = kWarps * kTileT;   // positions per pipeline stage
-constexpr int kRefresh = 16;               // phasor recurrence steps between fp64 refreshes
+constexpr int kRefresh = 16;               // phasor recurrence steps between exact refreshes
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -141,12 +141,75 @@ __device__ __forceinline__ int clamp_code(int c, int Nc, int& err) {
 }
 
 // ---------------------------------------------------------------------------------------
-// Codebook image: fp32 [R][16][Nc'][8] -> fp16 slots (see the file comment). blockIdx.y
-// selects the key (0) or value (1) codebook.
-__global__ void prep_codebook_kernel(const float* __restrict__ kcb, const float* __restrict__ vcb,
-                                     int R, int Nc, uint4* __restrict__ kimg, uint4* __restrict__ vimg) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;   // (v, j, c)
-  if (e >= 2 * kGroups * Nc) return;
+// Per-call preparation. blockIdx.y = 0 / 1: key / value codebook image, fp32 [R][16][Nc'][8]
+// -> fp16 slots (see the file comment). blockIdx.y = 2: RoPE tables, all from fp64:
+//   theta[p] = base^(-2p/d), row[delta][p] = e^{i delta theta_p} for the 128 rows of a stage,
+//   adv[p] = e^{i 128 theta_p} (one stage further).
+constexpr int kPhaseRows = kStageT;
+
+// blockIdx.y = 3: query fragments of every (sequence, KV head) in the scores kernel's mma
+// k-order (see attend_scores_kernel); blockIdx.y = 4: base phasor e^{i t_begin theta_p} of
+// every (sequence, split), from an fp64 angle.
+template <typename QT>
+__device__ __forceinline__ void prep_qfrag(const AttendArgs& a, const QT* q, int e) {
+  const int KV = a.kv_heads, G = a.q_heads / KV;
+  if (e >= a.B * KV * 256) return;
+  const int b = e / (KV * 256), r = e % (KV * 256);
+  const int kv = r >> 8, st = (r >> 5) & 7, ln = r & 31;
+  const int gg = ln >> 2, ii = ln & 3;
+  uint2 v = make_uint2(0u, 0u);
+  if (gg < G) {
+    const QT* qh = q + (static_cast<int64_t>(b) * a.q_heads + kv * G + gg) * kD;
+    const int d0 = 8 * (4 * (st >> 1) + ii) + 4 * (st & 1);
+    v.x = h2_as_u32(__floats2half2_rn(qval(qh, d0), qval(qh, d0 + 1)));
+    v.y = h2_as_u32(__floats2half2_rn(qval(qh, d0 + 2), qval(qh, d0 + 3)));
+  }
+  const_cast<uint2*>(a.qfrag)[e] = v;
+}
+
+__global__ void prep_kernel(AttendArgs a, int R, const void* __restrict__ q, int q_dtype, int S) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  const int Nc = a.n_codes;
+  if (e == 0 && blockIdx.y == 0) *a.error_word = 0;   // this call's device error word starts clear
+  if (blockIdx.y == 3) {
+    if (q_dtype == COMMVQ_F32) prep_qfrag(a, static_cast<const float*>(q), e);
+    else if (q_dtype == COMMVQ_F16) prep_qfrag(a, static_cast<const __half*>(q), e);
+    else prep_qfrag(a, static_cast<const __nv_bfloat16*>(q), e);
+    return;
+  }
+  if (blockIdx.y == 4) {
+    if (e >= a.B * S * (kD / 2)) return;
+    const int p = e % (kD / 2), bs = e / (kD / 2), s = bs % S, b = bs / S;
+    int64_t row0, t_begin, t_end;
+    split_range(a, b, s, S, row0, t_begin, t_end);
+    double sn, cs;
+    sincos(static_cast<double>(t_begin) * pow(a.rope_base, -2.0 * p / kD), &sn, &cs);
+    const_cast<float2*>(a.basetab)[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+    return;
+  }
+  const double rope_base = a.rope_base;
+  double* theta = const_cast<double*>(a.theta);
+  float2* rowph = const_cast<float2*>(a.rowph);
+  float2* advph = const_cast<float2*>(a.advph);
+  const float* kcb = a.k_codebook;
+  const float* vcb = a.v_codebook;
+  uint4* kimg = const_cast<uint4*>(a.k_img);
+  uint4* vimg = const_cast<uint4*>(a.v_img);
+  if (blockIdx.y == 2) {
+    if (e >= kPhaseRows * (kD / 2)) return;
+    const int delta = e / (kD / 2), p = e % (kD / 2);
+    const double th = pow(rope_base, -2.0 * p / kD);
+    double sn, cs;
+    sincos(static_cast<double>(delta) * th, &sn, &cs);
+    rowph[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+    if (delta == 0) {
+      theta[p] = th;
+      sincos(static_cast<double>(kStageT) * th, &sn, &cs);
+      advph[p] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+    }
+    return;
+  }
+  if (e >= 2 * kGroups * Nc) return;   // (v, j, c)
   const float* cb = blockIdx.y ? vcb : kcb;
   uint4* img = blockIdx.y ? vimg : kimg;
   const int c = e % Nc, vj = e / Nc, j = vj % kGroups, v = vj / kGroups;
@@ -170,16 +233,19 @@ __device__ __forceinline__ int slot(int v, int j, int c, int Nc) {
 // tile and, through the k-order of the mma, the 16 RoPE pairs of groups i, i+4, i+8, i+12:
 // k-step 2u+h of the mma covers pairs 2h and 2h+1 of group 4u+i, so one 16-byte gather
 // fills two k-steps of a row. The query fragments use the same k-order.
-template <int R, int KV, bool kCheck, typename QT>
+// NC: the entry count when it is 256 (compile-time; every uint8 code is valid), else 0
+// (run-time count, codes checked against it).
+template <int R, int KV, int NC, typename QT>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
+  constexpr bool kCheck = NC != 256;
   extern __shared__ __align__(16) unsigned char smem[];
-  const int Nc = a.n_codes;
+  const int Nc = NC ? NC : a.n_codes;
   const int G = a.q_heads / KV;
   uint4* cbk = reinterpret_cast<uint4*>(smem);                       // 32 * Nc slots
   uint2* qf = reinterpret_cast<uint2*>(cbk + 32 * Nc);               // [KV][8][32]
-  double* theta = reinterpret_cast<double*>(qf + KV * 8 * 32);       // [64]
-  float* red = reinterpret_cast<float*>(theta + 64);                 // [8 warps][KV*8]
+  float2* base = reinterpret_cast<float2*>(qf + KV * 8 * 32);       // [64] e^{i t0 theta_p}
+  float* red = reinterpret_cast<float*>(base + 64);                  // [8 warps][KV*8]
   uint8_t* stage_buf = reinterpret_cast<uint8_t*>(red + kWarps * KV * 8);   // [2][kStageT][KV][R][16]
   using SL = StageLayout<R, KV>;
   constexpr int kStageBytes = SL::kBytes;
@@ -196,50 +262,45 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
     return;
   }
 
-  // codebook image (async), query fragments, RoPE frequencies, first code stage
+  // Set-up is all asynchronous copies of what the prep kernel made: codebook image, query
+  // fragments of this sequence, base phasors of this split; then the first code stage.
   for (int p = tid; p < 32 * Nc; p += kThreads) cp_async16(cbk + p, a.k_img + p);
-  cp_async_commit();
-  for (int e = tid; e < KV * 8 * 32; e += kThreads) {
-    const int kv = e >> 8, st = (e >> 5) & 7, ln = e & 31;
-    const int gg = ln >> 2, ii = ln & 3;
-    uint2 v = make_uint2(0u, 0u);
-    if (gg < G) {
-      const QT* qh = q + (static_cast<int64_t>(b) * a.q_heads + kv * G + gg) * kD;
-      const int d0 = 8 * (4 * (st >> 1) + ii) + 4 * (st & 1);
-      v.x = h2_as_u32(__floats2half2_rn(qval(qh, d0), qval(qh, d0 + 1)));
-      v.y = h2_as_u32(__floats2half2_rn(qval(qh, d0 + 2), qval(qh, d0 + 3)));
-    }
-    qf[e] = v;
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(a.qfrag + static_cast<int64_t>(b) * KV * 256);
+    for (int p = tid; p < KV * 256 / 2; p += kThreads) cp_async16(reinterpret_cast<uint4*>(qf) + p, src + p);
+    const uint4* bsrc = reinterpret_cast<const uint4*>(a.basetab + (static_cast<int64_t>(b) * S + s) * (kD / 2));
+    if (tid < kD / 4) cp_async16(reinterpret_cast<uint4*>(base) + tid, bsrc + tid);
   }
-  if (tid < 64) theta[tid] = pow(a.rope_base, -2.0 * tid / kD);
+  cp_async_commit();
   issue_stage<R, KV>(stage_buf, a.k_codes, row0, t_begin, t_end);
   cp_async_commit();
-  __syncthreads();
+  (void)q;
 
   // Phasors of the thread's 16 pairs (k = 4u + m -> pair 4(4u+i) + m) at its two rows, and
-  // the per-iteration advance e^{i kStageT theta}.
+  // the per-iteration advance e^{i kStageT theta}. A refresh rebuilds them exactly from the
+  // stage's base phasor (fp64, in shared memory) times the row table of the prep kernel.
   float2 ph[2][16], adv[16];
-  auto refresh = [&](int64_t t_row0) {
+  auto load_rows = [&]() {   // e^{i delta theta_p} of the thread's two rows (delta < kStageT)
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+#pragma unroll
+      for (int rho = 0; rho < 2; ++rho)
+        ph[rho][k] = a.rowph[(warp * kTileT + g + 8 * rho) * (kD / 2) + 4 * (4 * (k >> 2) + i) + (k & 3)];
+  };
+  auto times_base = [&]() {  // ph <- base (this stage's e^{i t0 theta}) x row phasor
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
-      const double th = theta[4 * (4 * (k >> 2) + i) + (k & 3)];
+      const float2 bp = base[4 * (4 * (k >> 2) + i) + (k & 3)];
 #pragma unroll
       for (int rho = 0; rho < 2; ++rho) {
-        const double ang = static_cast<double>(t_row0 + g + 8 * rho) * th;
-        const double red_ang = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
-        float sn, cs;
-        sincosf(static_cast<float>(red_ang), &sn, &cs);
-        ph[rho][k] = make_float2(cs, sn);
+        const float2 rp = ph[rho][k];
+        ph[rho][k] = make_float2(fmaf(bp.x, rp.x, -bp.y * rp.y), fmaf(bp.x, rp.y, bp.y * rp.x));
       }
     }
   };
+  load_rows();   // global loads in flight while the asynchronous copies land
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const double ang = static_cast<double>(kStageT) * theta[4 * (4 * (k >> 2) + i) + (k & 3)];
-    float sn, cs;
-    sincosf(static_cast<float>(ang - 6.283185307179586 * rint(ang * 0.15915494309189535)), &sn, &cs);
-    adv[k] = make_float2(cs, sn);
-  }
+  for (int k = 0; k < 16; ++k) adv[k] = a.advph[4 * (4 * (k >> 2) + i) + (k & 3)];
 
   for (int e = tid; e < kWarps * KV * 8; e += kThreads) red[e] = -INFINITY;
   const int64_t n_tiles = (a.max_T + kTileT - 1) / kTileT;
@@ -251,12 +312,18 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
     if (t0 + kStageT < t_end)
       issue_stage<R, KV>(stage_buf + (stage ^ 1) * kStageBytes, a.k_codes, row0, t0 + kStageT, t_end);
     cp_async_commit();
+    if (it > 0 && it % kRefresh == 0 && tid < kD / 2) {   // later refresh: fp64 angle
+      double sn, cs;
+      sincos(static_cast<double>(t0) * a.theta[tid], &sn, &cs);
+      base[tid] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+    }
     cp_async_wait<1>();
     __syncthreads();
 
     const int64_t tt0 = t0 + warp * kTileT;        // this warp's tile
     if (it % kRefresh == 0) {
-      refresh(tt0);
+      if (it > 0) load_rows();
+      times_base();
     } else {
 #pragma unroll
       for (int k = 0; k < 16; ++k)
@@ -268,7 +335,8 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
     }
     if (tt0 < t_end) {
       const uint8_t* sb = stage_buf + stage * kStageBytes;
-      const bool valid0 = tt0 + g < t_end, valid1 = tt0 + g + 8 < t_end;
+      const int rem = static_cast<int>(min(static_cast<int64_t>(kTileT), t_end - tt0));  // valid rows
+      const bool valid0 = g < rem, valid1 = g + 8 < rem;
 #pragma unroll 1
       for (int kv = 0; kv < KV; ++kv) {
         uint4 cw[2][R];
@@ -363,11 +431,12 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
 // 16g+m, row g+8 is dim 16g+8+m) and positions 2i, 2i+1, 2i+8, 2i+9 of each tile, which are
 // exactly the positions of its P^T fragment, so probabilities go from the score buffer into
 // registers with no exchange. Warps are spread over KV heads (8/KV warps per head).
-template <int R, int KV, bool kCheck>
+template <int R, int KV, int NC>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_values_kernel(AttendArgs a) {
+  constexpr bool kCheck = NC != 256;
   extern __shared__ __align__(16) unsigned char smem[];
-  const int Nc = a.n_codes;
+  const int Nc = NC ? NC : a.n_codes;
   const int G = a.q_heads / KV;
   constexpr int kWpk = kWarps / KV;                  // warps per KV head
   using SL = StageLayout<R, KV>;
@@ -437,6 +506,7 @@ attend_values_kernel(AttendArgs a) {
     for (int tile = sub; tile < kWarps; tile += kWpk) {
       const int64_t tt0 = t0 + tile * kTileT;
       if (tt0 >= t_end) break;
+      const int rem = static_cast<int>(min(static_cast<int64_t>(kTileT), t_end - tt0));  // valid positions
       // probabilities of this thread's 4 positions for head column g
       const int tau[4] = {2 * i, 2 * i + 1, 2 * i + 8, 2 * i + 9};
       float p[4] = {0.f, 0.f, 0.f, 0.f};
@@ -445,7 +515,7 @@ attend_values_kernel(AttendArgs a) {
         const float sk[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          if (tt0 + tau[k] < t_end) p[k] = exp2f(sk[k] - m_h);
+          if (tau[k] < rem) p[k] = exp2f(sk[k] - m_h);
           lsum += p[k];
         }
       }
@@ -457,13 +527,15 @@ attend_values_kernel(AttendArgs a) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int tl = tile * kTileT + tau[k];
-        const bool valid = tt0 + tau[k] < t_end;
+        const bool valid = tau[k] < rem;
         uint32_t cwr[R];
 #pragma unroll
         for (int r = 0; r < R; ++r)
           cwr[r] = valid ? *reinterpret_cast<const uint32_t*>(sb + SL::offset(tl, kv * R + r) + 4 * (g >> 1))
                          : 0u;
-        // load order chosen per lane so that each 8-lane phase hits 8 different bank groups
+        // Load order chosen per lane so that each 8-lane phase of a gather hits 8 different
+        // bank groups: lane i reads group 2g + (i & 1) first and round/copy (i >> 1) first;
+        // odd lanes then swap the two sums back into (group 2g, group 2g+1).
         const int jA = 2 * g + odd, jB = 2 * g + (odd ^ 1);
         const int shA = sh + 8 * odd, shB = sh + 8 * (odd ^ 1);
         uint4 SA, SB;
@@ -557,23 +629,24 @@ attend_values_kernel(AttendArgs a) {
   }
 }
 
-template <int R, int KV, bool kCheck>
+template <int R, int KV, int NC>
 commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt, int S, cudaStream_t st) {
   const size_t smem_s = mma_scores_smem_bytes(R, KV, a.n_codes);
   const size_t smem_v = mma_values_smem_bytes(R, KV, a.q_heads, a.n_codes);
   dim3 grid(S, a.B);
   {
     const int n = 2 * kGroups * a.n_codes;
-    prep_codebook_kernel<<<dim3((n + kThreads - 1) / kThreads, 2), kThreads, 0, st>>>(
-        a.k_codebook, a.v_codebook, R, a.n_codes, const_cast<uint4*>(a.k_img),
-        const_cast<uint4*>(a.v_img));
+    int bx = max((n + kThreads - 1) / kThreads, (kPhaseRows * (kD / 2) + kThreads - 1) / kThreads);
+    bx = max(bx, (a.B * a.kv_heads * 256 + kThreads - 1) / kThreads);
+    bx = max(bx, (a.B * S * (kD / 2) + kThreads - 1) / kThreads);
+    prep_kernel<<<dim3(bx, 5), kThreads, 0, st>>>(a, R, q, static_cast<int>(qt), S);
   }
   if (a.main_start &&
       cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a.main_start), st, cudaEventRecordExternal) != cudaSuccess)
     return COMMVQ_ERR_CUDA;
 #define COMMVQ_LAUNCH_SCORES(T)                                                                      \
   {                                                                                                \
-    auto k = attend_scores_kernel<R, KV, kCheck, T>;                                               \
+    auto k = attend_scores_kernel<R, KV, NC, T>;                                               \
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s) != cudaSuccess) \
       return COMMVQ_ERR_CUDA;                                                                      \
     k<<<grid, kThreads, smem_s, st>>>(a, static_cast<const T*>(q));                                \
@@ -586,7 +659,7 @@ commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt,
   }
 #undef COMMVQ_LAUNCH_SCORES
   {
-    auto k = attend_values_kernel<R, KV, kCheck>;
+    auto k = attend_values_kernel<R, KV, NC>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_v) != cudaSuccess)
       return COMMVQ_ERR_CUDA;
     k<<<grid, kThreads, smem_v, st>>>(a);
@@ -599,8 +672,8 @@ commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt,
 
 template <int R, int KV>
 commvq_status launch_mma_r(const AttendArgs& a, const void* q, commvq_dtype qt, int S, cudaStream_t st) {
-  if (a.n_codes < 256) return launch_mma_rk<R, KV, true>(a, q, qt, S, st);
-  return launch_mma_rk<R, KV, false>(a, q, qt, S, st);
+  if (a.n_codes == 256) return launch_mma_rk<R, KV, 256>(a, q, qt, S, st);
+  return launch_mma_rk<R, KV, 0>(a, q, qt, S, st);
 }
 
 template <int R>
@@ -617,7 +690,7 @@ commvq_status launch_mma_kv(const AttendArgs& a, const void* q, commvq_dtype qt,
 }  // namespace
 
 size_t mma_scores_smem_bytes(int R, int KV, int n_codes) {
-  return static_cast<size_t>(512) * n_codes + static_cast<size_t>(KV) * 8 * 32 * 8 + 64 * 8 +
+  return static_cast<size_t>(512) * n_codes + static_cast<size_t>(KV) * 8 * 32 * 8 + 64 * sizeof(float2) +
          static_cast<size_t>(kWarps) * KV * 8 * 4 + static_cast<size_t>(2) * kStageT * KV * R * kGroups;
 }
 

@@ -15,7 +15,7 @@ namespace {
 
 constexpr int kRowsPerThread = 2;
 constexpr int kSub = kThreads * kRowsPerThread;   // rows assigned per pass
-constexpr int kChunkRows = 2048;                  // rows per CTA
+constexpr int kChunkRows = 512;                   // rows per CTA (4096 rows fill 128 CTAs)
 constexpr int kTile = 1024;                       // codebook entries staged per pass
 constexpr int kMaxCodes = 4096;
 

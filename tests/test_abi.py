@@ -96,7 +96,11 @@ def test_workspace_sizes(api):
     mma = api.attend_workspace_bytes(cfg, 1, 32768, algo=api.ATTN_DECODE_MMA, splits=148)
     part = 256 + 32 * 148 * 528
     img = 512 * 256
-    want = -(-part // 256) * 256 + 2 * img + 32768 * 32 * 4
+    phase = 64 * 8 + 128 * 64 * 8 + 64 * 8
+    qfrag = 1 * 8 * 256 * 8
+    base = 1 * 148 * 64 * 8
+    want = (-(-part // 256) * 256 + 2 * img + -(-phase // 256) * 256 + -(-qfrag // 256) * 256 +
+            -(-base // 256) * 256 + 32768 * 32 * 4)
     assert mma == -(-want // 256) * 256
     assert api.attend_workspace_bytes(cfg, 1, 32768) == api.attend_workspace_bytes(
         cfg, 1, 32768, algo=api.ATTN_DECODE_MMA)
