@@ -35,9 +35,16 @@
 namespace commvq {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kMmaThreads = 512;           // 16 warps per CTA, one CTA per SM
+constexpr int kMmaWarps = kMmaThreads / 32;
+constexpr int kTiles = 8;                  // mma row blocks per pipeline stage
 constexpr int kTileT = 16;                 // positions per mma row block
-constexpr int kStageT = kWarps * kTileT;   // positions per pipeline stage
+constexpr int kStageT = kTiles * kTileT;   // positions per pipeline stage
+
+// Barrier for a subset of the CTA's warps (ids 1..15; id 0 is __syncthreads).
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
+}
 constexpr int kRefresh = 16;               // phasor recurrence steps between exact refreshes
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -118,7 +125,7 @@ __device__ __forceinline__ void issue_stage(uint8_t* dst, const uint8_t* codes, 
   const int n = static_cast<int>(min(static_cast<int64_t>(kStageT), t_end - t0));
   const int pieces = n * SL::kPieces;
   const uint8_t* src = codes + (row0 + t0) * (SL::kPieces * 16);
-  for (int p = threadIdx.x; p < pieces; p += kThreads) {
+  for (int p = threadIdx.x; p < pieces; p += blockDim.x) {
     const int row = p / SL::kPieces, piece = p - row * SL::kPieces;
     cp_async16(dst + SL::offset(row, piece), src + p * 16);
   }
@@ -228,15 +235,33 @@ __device__ __forceinline__ int slot(int v, int j, int c, int Nc) {
   return ((v * 2 + (j >> 3)) * Nc + c) * 8 + ((j + 4 * v) & 7);
 }
 
+// Shared-memory loads at a byte offset from the start of the dynamic shared array.
+__device__ __forceinline__ uint4 lds128(const unsigned char* smem, uint32_t off) {
+  return *reinterpret_cast<const uint4*>(smem + off);
+}
+__device__ __forceinline__ uint2 lds64(const unsigned char* smem, uint32_t off) {
+  return *reinterpret_cast<const uint2*>(smem + off);
+}
+__device__ __forceinline__ uint32_t lds32(const unsigned char* smem, uint32_t off) {
+  return *reinterpret_cast<const uint32_t*>(smem + off);
+}
+// Byte b of w, zero-extended (one PRMT); sel = byte_sel(b).
+__device__ __forceinline__ uint32_t byte_sel(int b) { return 0x4440u | static_cast<uint32_t>(b); }
+__device__ __forceinline__ uint32_t take_byte(uint32_t w, uint32_t sel) { return __byte_perm(w, 0u, sel); }
+
 // ---------------------------------------------------------------------------------------
-// Scores. Thread (g = lane/4, i = lane%4) of a warp owns rows g and g+8 of its 16-position
-// tile and, through the k-order of the mma, the 16 RoPE pairs of groups i, i+4, i+8, i+12:
-// k-step 2u+h of the mma covers pairs 2h and 2h+1 of group 4u+i, so one 16-byte gather
-// fills two k-steps of a row. The query fragments use the same k-order.
+// Scores. A 16-position tile is shared by a pair of warps (tile = warp / 2, half = warp % 2).
+// Thread (g = lane/4, i = lane%4) owns rows g and g+8 of the tile and, through the k-order of
+// the mma, 8 RoPE pairs: k-step 2u+h covers pairs 2h and 2h+1 of group 4u+i, and half h of
+// the pair takes u = 2h and 2h+1 (groups i, 4+i or 8+i, 12+i). One 16-byte gather fills two
+// k-steps of a row. Each half accumulates a partial S over its 64 dimensions; the halves add
+// them through a small double-buffered exchange in shared memory, ordered by a named barrier
+// per warp pair. The query fragments use the same k-order. Splitting the pairs halves the
+// phasor registers, which lets 16 warps share an SM.
 // NC: the entry count when it is 256 (compile-time; every uint8 code is valid), else 0
 // (run-time count, codes checked against it).
 template <int R, int KV, int NC, typename QT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kMmaThreads, 1)
 attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
   constexpr bool kCheck = NC != 256;
   extern __shared__ __align__(16) unsigned char smem[];
@@ -245,29 +270,31 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
   uint4* cbk = reinterpret_cast<uint4*>(smem);                       // 32 * Nc slots
   uint2* qf = reinterpret_cast<uint2*>(cbk + 32 * Nc);               // [KV][8][32]
   float2* base = reinterpret_cast<float2*>(qf + KV * 8 * 32);       // [64] e^{i t0 theta_p}
-  float* red = reinterpret_cast<float*>(base + 64);                  // [8 warps][KV*8]
-  uint8_t* stage_buf = reinterpret_cast<uint8_t*>(red + kWarps * KV * 8);   // [2][kStageT][KV][R][16]
+  float* red = reinterpret_cast<float*>(base + 64);                  // [8 tiles][KV*8]
+  float4* xch = reinterpret_cast<float4*>(red + kTiles * KV * 8);    // [8 tiles][2][32]
+  uint8_t* stage_buf = reinterpret_cast<uint8_t*>(xch + kTiles * 2 * 32);   // [2][kStageT][KV][R][16]
   using SL = StageLayout<R, KV>;
   constexpr int kStageBytes = SL::kBytes;
 
   const int s = blockIdx.x, b = blockIdx.y, S = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tile = warp >> 1, half = warp & 1;
   const int g = lane >> 2, i = lane & 3, par = g & 1;
   int64_t row0, t_begin, t_end;
   split_range(a, b, s, S, row0, t_begin, t_end);
   Partial* part = a.partials + static_cast<int64_t>(b) * a.q_heads * S + s;   // + h * S
 
   if (t_begin >= t_end) {
-    for (int h = tid; h < a.q_heads; h += kThreads) part[static_cast<int64_t>(h) * S].m = -INFINITY;
+    for (int h = tid; h < a.q_heads; h += kMmaThreads) part[static_cast<int64_t>(h) * S].m = -INFINITY;
     return;
   }
 
   // Set-up is all asynchronous copies of what the prep kernel made: codebook image, query
   // fragments of this sequence, base phasors of this split; then the first code stage.
-  for (int p = tid; p < 32 * Nc; p += kThreads) cp_async16(cbk + p, a.k_img + p);
+  for (int p = tid; p < 32 * Nc; p += kMmaThreads) cp_async16(cbk + p, a.k_img + p);
   {
     const uint4* src = reinterpret_cast<const uint4*>(a.qfrag + static_cast<int64_t>(b) * KV * 256);
-    for (int p = tid; p < KV * 256 / 2; p += kThreads) cp_async16(reinterpret_cast<uint4*>(qf) + p, src + p);
+    for (int p = tid; p < KV * 256 / 2; p += kMmaThreads) cp_async16(reinterpret_cast<uint4*>(qf) + p, src + p);
     const uint4* bsrc = reinterpret_cast<const uint4*>(a.basetab + (static_cast<int64_t>(b) * S + s) * (kD / 2));
     if (tid < kD / 4) cp_async16(reinterpret_cast<uint4*>(base) + tid, bsrc + tid);
   }
@@ -276,21 +303,21 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
   cp_async_commit();
   (void)q;
 
-  // Phasors of the thread's 16 pairs (k = 4u + m -> pair 4(4u+i) + m) at its two rows, and
-  // the per-iteration advance e^{i kStageT theta}. A refresh rebuilds them exactly from the
-  // stage's base phasor (fp64, in shared memory) times the row table of the prep kernel.
-  float2 ph[2][16], adv[16];
-  auto load_rows = [&]() {   // e^{i delta theta_p} of the thread's two rows (delta < kStageT)
+  // Phasors of the thread's 8 pairs (k = 4 ul + m -> pair 4(4(2 half + ul) + i) + m) at its two
+  // rows, and the per-iteration advance e^{i kStageT theta}. A refresh rebuilds them exactly
+  // from the stage's base phasor (fp64 angle, in shared memory) times the prep row table.
+  auto pair_of = [&](int k) { return 4 * (4 * (2 * half + (k >> 2)) + i) + (k & 3); };
+  float2 ph[2][8], adv[8];
+  auto load_rows = [&]() {
 #pragma unroll
-    for (int k = 0; k < 16; ++k)
+    for (int k = 0; k < 8; ++k)
 #pragma unroll
-      for (int rho = 0; rho < 2; ++rho)
-        ph[rho][k] = a.rowph[(warp * kTileT + g + 8 * rho) * (kD / 2) + 4 * (4 * (k >> 2) + i) + (k & 3)];
+      for (int rho = 0; rho < 2; ++rho) ph[rho][k] = a.rowph[(tile * kTileT + g + 8 * rho) * (kD / 2) + pair_of(k)];
   };
-  auto times_base = [&]() {  // ph <- base (this stage's e^{i t0 theta}) x row phasor
+  auto times_base = [&]() {
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float2 bp = base[4 * (4 * (k >> 2) + i) + (k & 3)];
+    for (int k = 0; k < 8; ++k) {
+      const float2 bp = base[pair_of(k)];
 #pragma unroll
       for (int rho = 0; rho < 2; ++rho) {
         const float2 rp = ph[rho][k];
@@ -300,13 +327,23 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
   };
   load_rows();   // global loads in flight while the asynchronous copies land
 #pragma unroll
-  for (int k = 0; k < 16; ++k) adv[k] = a.advph[4 * (4 * (k >> 2) + i) + (k & 3)];
+  for (int k = 0; k < 8; ++k) adv[k] = a.advph[pair_of(k)];
 
-  for (int e = tid; e < kWarps * KV * 8; e += kThreads) red[e] = -INFINITY;
+  for (int e = tid; e < kTiles * KV * 8; e += kMmaThreads) red[e] = -INFINITY;
   const int64_t n_tiles = (a.max_T + kTileT - 1) / kTileT;
   const float scale = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
   int err = 0;
   int stage = 0, it = 0;
+  // Byte offsets of the thread's gathers: entry c of group 4u+i lives at g?[u - 2 half] + 128 c,
+  // gF in the v = par half of the image (first round / copy), gS in the other.
+  const uint32_t sel_i = byte_sel(i);
+  uint32_t gF[2], gS[2];
+#pragma unroll
+  for (int ul = 0; ul < 2; ++ul) {
+    const int j = 4 * (2 * half + ul) + i;
+    gF[ul] = static_cast<uint32_t>(slot(par, j, 0, Nc)) * 16;
+    gS[ul] = static_cast<uint32_t>(slot(par ^ 1, j, 0, Nc)) * 16;
+  }
 
   for (int64_t t0 = t_begin; t0 < t_end; t0 += kStageT, stage ^= 1, ++it) {
     if (t0 + kStageT < t_end)
@@ -320,66 +357,78 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
     cp_async_wait<1>();
     __syncthreads();
 
-    const int64_t tt0 = t0 + warp * kTileT;        // this warp's tile
+    const int64_t tt0 = t0 + tile * kTileT;        // this warp pair's tile
     if (it % kRefresh == 0) {
       if (it > 0) load_rows();
       times_base();
     } else {
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
+      for (int k = 0; k < 8; ++k)
 #pragma unroll
         for (int rho = 0; rho < 2; ++rho) {
           const float2 p = ph[rho][k], d = adv[k];
           ph[rho][k] = make_float2(fmaf(p.x, d.x, -p.y * d.y), fmaf(p.x, d.y, p.y * d.x));
         }
     }
-    if (tt0 < t_end) {
-      const uint8_t* sb = stage_buf + stage * kStageBytes;
+    if (tt0 < t_end) {   // uniform over the warp pair
+      const uint32_t sb = static_cast<uint32_t>(stage_buf - smem) + stage * kStageBytes;
       const int rem = static_cast<int>(min(static_cast<int64_t>(kTileT), t_end - tt0));  // valid rows
       const bool valid0 = g < rem, valid1 = g + 8 < rem;
 #pragma unroll 1
       for (int kv = 0; kv < KV; ++kv) {
-        uint4 cw[2][R];
+        // code words 2 half, 2 half + 1 (groups 8 half .. 8 half + 7) of each row; with two
+        // rounds, round `par` first (it pairs with the v = par half of the image)
+        uint2 cw[2][R];
 #pragma unroll
         for (int rho = 0; rho < 2; ++rho) {
           const bool valid = rho ? valid1 : valid0;
+          const int row = tile * kTileT + g + 8 * rho;
 #pragma unroll
-          for (int r = 0; r < R; ++r)
-            cw[rho][r] = valid ? *reinterpret_cast<const uint4*>(
-                                     sb + SL::offset(warp * kTileT + g + 8 * rho, kv * R + r))
-                               : make_uint4(0u, 0u, 0u, 0u);
+          for (int r = 0; r < R; ++r) {
+            const int piece = kv * R + (R == 2 ? (r ^ par) : r);
+            const uint32_t off = sb + SL::offset(row, piece) + 8 * half;
+            cw[rho][r] = valid ? lds64(smem, off) : make_uint2(0u, 0u);
+          }
         }
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = 4 * u + i;
+        for (int ul = 0; ul < 2; ++ul) {
+          const int u = 2 * half + ul;
           uint32_t A[2][4];
 #pragma unroll
           for (int rho = 0; rho < 2; ++rho) {
             uint4 e;
+            int c0 = static_cast<int>(take_byte(ul ? cw[rho][0].y : cw[rho][0].x, sel_i));
+            if (kCheck) c0 = clamp_code(c0, Nc, err);
             if (R == 2) {
-              const uint32_t w0 = word(cw[rho][0], u), w1 = word(cw[rho][R - 1], u);
-              int c_first = ((par ? w1 : w0) >> (8 * i)) & 0xff;    // round `par`
-              int c_second = ((par ? w0 : w1) >> (8 * i)) & 0xff;   // round 1 - par
-              if (kCheck) {
-                c_first = clamp_code(c_first, Nc, err);
-                c_second = clamp_code(c_second, Nc, err);
-              }
-              e = hadd2x4(cbk[slot(par, j, c_first, Nc)], cbk[slot(par ^ 1, j, c_second, Nc)]);
+              int c1 = static_cast<int>(take_byte(ul ? cw[rho][R - 1].y : cw[rho][R - 1].x, sel_i));
+              if (kCheck) c1 = clamp_code(c1, Nc, err);
+              e = hadd2x4(lds128(smem, gF[ul] + (c0 << 7)), lds128(smem, gS[ul] + (c1 << 7)));
             } else {
-              int c = (word(cw[rho][0], u) >> (8 * i)) & 0xff;
-              if (kCheck) c = clamp_code(c, Nc, err);
-              e = cbk[slot(par, j, c, Nc)];
+              e = lds128(smem, gF[ul] + (c0 << 7));
             }
-            A[0][rho] = rotate_pair(e.x, ph[rho][4 * u + 0]);
-            A[0][2 + rho] = rotate_pair(e.y, ph[rho][4 * u + 1]);
-            A[1][rho] = rotate_pair(e.z, ph[rho][4 * u + 2]);
-            A[1][2 + rho] = rotate_pair(e.w, ph[rho][4 * u + 3]);
+            A[0][rho] = rotate_pair(e.x, ph[rho][4 * ul + 0]);
+            A[0][2 + rho] = rotate_pair(e.y, ph[rho][4 * ul + 1]);
+            A[1][rho] = rotate_pair(e.z, ph[rho][4 * ul + 2]);
+            A[1][2 + rho] = rotate_pair(e.w, ph[rho][4 * ul + 3]);
           }
           const uint2 b0 = qf[(kv * 8 + 2 * u) * 32 + lane];
           const uint2 b1 = qf[(kv * 8 + 2 * u + 1) * 32 + lane];
           mma16816(acc, A[0][0], A[0][1], A[0][2], A[0][3], b0.x, b0.y);
           mma16816(acc, A[1][0], A[1][1], A[1][2], A[1][3], b1.x, b1.y);
+        }
+        // Add the two halves' partial S: half 1 writes, both meet at the pair's barrier,
+        // half 0 reads. The buffer alternates with kv, so half 1 can run one kv ahead.
+        float4* xs = xch + (tile * 2 + (kv & 1)) * 32 + lane;
+        if (half) *xs = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        named_barrier_sync(1 + tile, 64);
+        if (half) continue;
+        {
+          const float4 o = *xs;
+          acc[0] += o.x;
+          acc[1] += o.y;
+          acc[2] += o.z;
+          acc[3] += o.w;
         }
         // acc: rows g (c0, c1) and g+8 (c2, c3); columns 2i, 2i+1 = query heads kv*G + col.
         const int64_t tau = tt0 / kTileT;
@@ -401,7 +450,7 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
           m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
         }
         if (g == 0) {
-          float* rw = red + warp * KV * 8 + kv * 8 + 2 * i;
+          float* rw = red + tile * KV * 8 + kv * 8 + 2 * i;
           rw[0] = fmaxf(rw[0], m0);
           rw[1] = fmaxf(rw[1], m1);
         }
@@ -410,13 +459,13 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
     __syncthreads();
   }
 
-  // split maxima: each warp kept its own row of maxima; take the max over warps
-  for (int e = tid; e < KV * 8; e += kThreads) {
+  // split maxima: the half-0 warp of each tile kept a row of maxima; take the max over tiles
+  for (int e = tid; e < KV * 8; e += kMmaThreads) {
     const int kv = e >> 3, col = e & 7;
     if (col >= G) continue;
     float v = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) v = fmaxf(v, red[w * KV * 8 + e]);
+    for (int w = 0; w < kTiles; ++w) v = fmaxf(v, red[w * KV * 8 + e]);
     part[static_cast<int64_t>(kv * G + col) * S].m = v;
   }
   if (kCheck) {
@@ -430,22 +479,24 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
 // Thread (g, i) owns value dims 16g..16g+15 (groups 2g, 2g+1; mma row g of m-tile m is dim
 // 16g+m, row g+8 is dim 16g+8+m) and positions 2i, 2i+1, 2i+8, 2i+9 of each tile, which are
 // exactly the positions of its P^T fragment, so probabilities go from the score buffer into
-// registers with no exchange. Warps are spread over KV heads (8/KV warps per head).
+// registers with no exchange. Warps are spread over KV heads (16/KV warps per head, each
+// taking every (16/KV)-th tile of a stage); the A fragments are built one position pair at a
+// time to stay within the 128 registers that 16 warps per SM allow.
 template <int R, int KV, int NC>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kMmaThreads, 1)
 attend_values_kernel(AttendArgs a) {
   constexpr bool kCheck = NC != 256;
   extern __shared__ __align__(16) unsigned char smem[];
   const int Nc = NC ? NC : a.n_codes;
   const int G = a.q_heads / KV;
-  constexpr int kWpk = kWarps / KV;                  // warps per KV head
+  constexpr int kWpk = kMmaWarps / KV;               // warps per KV head
   using SL = StageLayout<R, KV>;
   uint4* cbv = reinterpret_cast<uint4*>(smem);
   uint8_t* stage_buf = reinterpret_cast<uint8_t*>(cbv + 32 * Nc);
   constexpr int kStageBytes = SL::kBytes;
-  const int score_stage_bytes = (kStageT / kTileT) * a.q_heads * 16 * 4;   // 8 tiles x Hq x 16 floats
+  const int score_stage_bytes = kTiles * a.q_heads * 16 * 4;   // 8 tiles x Hq x 16 floats
   uint8_t* score_buf = stage_buf + 2 * kStageBytes;
-  float* xred = reinterpret_cast<float*>(stage_buf);  // reused after the loop: [kWarps][32][33]
+  float* xred = reinterpret_cast<float*>(stage_buf);  // reused after the loop: [warps][32][33]
 
   const int s = blockIdx.x, b = blockIdx.y, S = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -456,7 +507,7 @@ attend_values_kernel(AttendArgs a) {
   Partial* part = a.partials + static_cast<int64_t>(b) * a.q_heads * S + s;
 
   if (t_begin >= t_end) {
-    for (int e = tid; e < a.q_heads * (kD + 1); e += kThreads) {
+    for (int e = tid; e < a.q_heads * (kD + 1); e += kMmaThreads) {
       const int h = e / (kD + 1), d = e % (kD + 1);
       if (d < kD)
         part[static_cast<int64_t>(h) * S].o[d] = 0.0f;
@@ -474,9 +525,9 @@ attend_values_kernel(AttendArgs a) {
     const int pieces = static_cast<int>((tau1 - tau0) * a.q_heads * 4);
     const uint8_t* src = reinterpret_cast<const uint8_t*>(
         a.scores + score_index(b, tau0, 0, 0, 0, 0, n_tiles, KV, G));
-    for (int p = tid; p < pieces; p += kThreads) cp_async16(dst + p * 16, src + p * 16);
+    for (int p = tid; p < pieces; p += kMmaThreads) cp_async16(dst + p * 16, src + p * 16);
   };
-  for (int p = tid; p < 32 * Nc; p += kThreads) cp_async16(cbv + p, a.v_img + p);
+  for (int p = tid; p < 32 * Nc; p += kMmaThreads) cp_async16(cbv + p, a.v_img + p);
   cp_async_commit();
   issue_stage<R, KV>(stage_buf, a.v_codes, row0, t_begin, t_end);
   issue_scores(score_buf, t_begin);
@@ -489,8 +540,30 @@ attend_values_kernel(AttendArgs a) {
   float lsum = 0.0f;
   int err = 0;
   const int odd = i & 1, vsel = (i >> 1) & 1;
-  const int sh = 16 * (g & 1);                       // groups 2g, 2g+1 inside their code word
   int stage = 0;
+  // Per-thread constants. Lane i reads group jA = 2g + (i & 1) before jB = 2g + 1 - (i & 1)
+  // and image half vsel = (i >> 1) before the other, so each 8-lane phase of a gather hits 8
+  // bank groups; odd lanes swap the sums back. gA[x], gB[x]: byte offset of entry 0 of jA/jB
+  // in the x-th half read; cw_off[k][x]: offset of the code word (groups 2g, 2g+1) of
+  // position tau[k] in a tile, for the round read x-th.
+  const int jA = 2 * g + odd, jB = 2 * g + (odd ^ 1);
+  const uint32_t selA = byte_sel(jA & 3), selB = byte_sel(jB & 3);
+  uint32_t gA[R], gB[R], cw_off[4][R];
+#pragma unroll
+  for (int x = 0; x < R; ++x) {
+    gA[x] = static_cast<uint32_t>(slot(vsel ^ x, jA, 0, Nc)) * 16;
+    gB[x] = static_cast<uint32_t>(slot(vsel ^ x, jB, 0, Nc)) * 16;
+  }
+  {
+    const int tau4[4] = {2 * i, 2 * i + 1, 2 * i + 8, 2 * i + 9};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int x = 0; x < R; ++x) {
+        const int r = (R == 2) ? (vsel ^ x) : 0;
+        cw_off[k][x] = static_cast<uint32_t>(SL::offset(tau4[k], kv * R + r) + 4 * (g >> 1));
+      }
+  }
 
   for (int64_t t0 = t_begin; t0 < t_end; t0 += kStageT, stage ^= 1) {
     if (t0 + kStageT < t_end) {
@@ -500,10 +573,10 @@ attend_values_kernel(AttendArgs a) {
     cp_async_commit();
     cp_async_wait<1>();
     __syncthreads();
-    const uint8_t* sb = stage_buf + stage * kStageBytes;
+    const uint32_t sb = static_cast<uint32_t>(stage_buf - smem) + stage * kStageBytes;
     const float* ssc = reinterpret_cast<const float*>(score_buf + stage * score_stage_bytes);
 
-    for (int tile = sub; tile < kWarps; tile += kWpk) {
+    for (int tile = sub; tile < kTiles; tile += kWpk) {
       const int64_t tt0 = t0 + tile * kTileT;
       if (tt0 >= t_end) break;
       const int rem = static_cast<int>(min(static_cast<int64_t>(kTileT), t_end - tt0));  // valid positions
@@ -522,62 +595,49 @@ attend_values_kernel(AttendArgs a) {
       const uint32_t b0 = h2_as_u32(__floats2half2_rn(p[0], p[1]));
       const uint32_t b1 = h2_as_u32(__floats2half2_rn(p[2], p[3]));
 
-      // decoded groups 2g (E0) and 2g+1 (E1) of the 4 positions
-      uint4 E0[4], E1[4];
+      // A fragments of the 8 m-tiles: row g = dim 16g+m (group 2g, element m), row g+8 = dim
+      // 16g+8+m (group 2g+1, element m); register 2*pr (+1) holds positions of pair pr
+      // ((2i, 2i+1) or (2i+8, 2i+9)) for row g (g+8).
+      const uint32_t sbt = sb + tile * kTileT * SL::kPieces * 16;
+      uint32_t A[8][4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int tl = tile * kTileT + tau[k];
-        const bool valid = tau[k] < rem;
-        uint32_t cwr[R];
+      for (int pr = 0; pr < 2; ++pr) {
+        uint4 E0[2], E1[2];   // decoded groups 2g and 2g+1 of the pair's two positions
 #pragma unroll
-        for (int r = 0; r < R; ++r)
-          cwr[r] = valid ? *reinterpret_cast<const uint32_t*>(sb + SL::offset(tl, kv * R + r) + 4 * (g >> 1))
-                         : 0u;
-        // Load order chosen per lane so that each 8-lane phase of a gather hits 8 different
-        // bank groups: lane i reads group 2g + (i & 1) first and round/copy (i >> 1) first;
-        // odd lanes then swap the two sums back into (group 2g, group 2g+1).
-        const int jA = 2 * g + odd, jB = 2 * g + (odd ^ 1);
-        const int shA = sh + 8 * odd, shB = sh + 8 * (odd ^ 1);
-        uint4 SA, SB;
-        if (R == 2) {
-          const uint32_t wv = vsel ? cwr[R - 1] : cwr[0], wo = vsel ? cwr[0] : cwr[R - 1];
-          int cA0 = (wv >> shA) & 0xff, cB0 = (wv >> shB) & 0xff;
-          int cA1 = (wo >> shA) & 0xff, cB1 = (wo >> shB) & 0xff;
+        for (int k2 = 0; k2 < 2; ++k2) {
+          const int k = 2 * pr + k2;
+          const bool valid = tau[k] < rem;
+          // the code word of groups 2g, 2g+1; with two rounds, round vsel first
+          const uint32_t w0 = valid ? lds32(smem, sbt + cw_off[k][0]) : 0u;
+          int cA0 = static_cast<int>(take_byte(w0, selA)), cB0 = static_cast<int>(take_byte(w0, selB));
           if (kCheck) {
             cA0 = clamp_code(cA0, Nc, err);
             cB0 = clamp_code(cB0, Nc, err);
-            cA1 = clamp_code(cA1, Nc, err);
-            cB1 = clamp_code(cB1, Nc, err);
           }
-          const uint4 L0 = cbv[slot(vsel, jA, cA0, Nc)];
-          const uint4 L1 = cbv[slot(vsel, jB, cB0, Nc)];
-          const uint4 L2 = cbv[slot(vsel ^ 1, jA, cA1, Nc)];
-          const uint4 L3 = cbv[slot(vsel ^ 1, jB, cB1, Nc)];
-          SA = hadd2x4(L0, L2);
-          SB = hadd2x4(L1, L3);
-        } else {
-          int cA = (cwr[0] >> shA) & 0xff, cB = (cwr[0] >> shB) & 0xff;
-          if (kCheck) {
-            cA = clamp_code(cA, Nc, err);
-            cB = clamp_code(cB, Nc, err);
+          uint4 SA = lds128(smem, gA[0] + (cA0 << 7));
+          uint4 SB = lds128(smem, gB[0] + (cB0 << 7));
+          if (R == 2) {
+            const uint32_t w1 = valid ? lds32(smem, sbt + cw_off[k][R - 1]) : 0u;
+            int cA1 = static_cast<int>(take_byte(w1, selA)), cB1 = static_cast<int>(take_byte(w1, selB));
+            if (kCheck) {
+              cA1 = clamp_code(cA1, Nc, err);
+              cB1 = clamp_code(cB1, Nc, err);
+            }
+            SA = hadd2x4(SA, lds128(smem, gA[R - 1] + (cA1 << 7)));
+            SB = hadd2x4(SB, lds128(smem, gB[R - 1] + (cB1 << 7)));
           }
-          SA = cbv[slot(vsel, jA, cA, Nc)];
-          SB = cbv[slot(vsel, jB, cB, Nc)];
+          E0[k2] = odd ? SB : SA;
+          E1[k2] = odd ? SA : SB;
         }
-        E0[k] = odd ? SB : SA;
-        E1[k] = odd ? SA : SB;
-      }
-      // A fragments of the 8 m-tiles: row g = dim 16g+m (E0 element m), row g+8 = dim
-      // 16g+8+m (E1 element m); columns = positions (2i, 2i+1) and (2i+8, 2i+9).
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const unsigned sel = (m & 1) ? 0x7632u : 0x5410u;
-        const uint32_t a0 = __byte_perm(word(E0[0], m >> 1), word(E0[1], m >> 1), sel);
-        const uint32_t a1 = __byte_perm(word(E1[0], m >> 1), word(E1[1], m >> 1), sel);
-        const uint32_t a2 = __byte_perm(word(E0[2], m >> 1), word(E0[3], m >> 1), sel);
-        const uint32_t a3 = __byte_perm(word(E1[2], m >> 1), word(E1[3], m >> 1), sel);
-        mma16816(O[m], a0, a1, a2, a3, b0, b1);
+        for (int m = 0; m < 8; ++m) {
+          const unsigned sel = (m & 1) ? 0x7632u : 0x5410u;
+          A[m][2 * pr] = __byte_perm(word(E0[0], m >> 1), word(E0[1], m >> 1), sel);
+          A[m][2 * pr + 1] = __byte_perm(word(E1[0], m >> 1), word(E1[1], m >> 1), sel);
+        }
       }
+#pragma unroll
+      for (int m = 0; m < 8; ++m) mma16816(O[m], A[m][0], A[m][1], A[m][2], A[m][3], b0, b1);
     }
     __syncthreads();
   }
@@ -649,7 +709,7 @@ commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt,
     auto k = attend_scores_kernel<R, KV, NC, T>;                                               \
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s) != cudaSuccess) \
       return COMMVQ_ERR_CUDA;                                                                      \
-    k<<<grid, kThreads, smem_s, st>>>(a, static_cast<const T*>(q));                                \
+    k<<<grid, kMmaThreads, smem_s, st>>>(a, static_cast<const T*>(q));                             \
   }
   switch (qt) {
     case COMMVQ_F32: COMMVQ_LAUNCH_SCORES(float) break;
@@ -662,7 +722,7 @@ commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt,
     auto k = attend_values_kernel<R, KV, NC>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_v) != cudaSuccess)
       return COMMVQ_ERR_CUDA;
-    k<<<grid, kThreads, smem_v, st>>>(a);
+    k<<<grid, kMmaThreads, smem_v, st>>>(a);
   }
   if (a.main_stop &&
       cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a.main_stop), st, cudaEventRecordExternal) != cudaSuccess)
@@ -691,15 +751,18 @@ commvq_status launch_mma_kv(const AttendArgs& a, const void* q, commvq_dtype qt,
 
 size_t mma_scores_smem_bytes(int R, int KV, int n_codes) {
   return static_cast<size_t>(512) * n_codes + static_cast<size_t>(KV) * 8 * 32 * 8 + 64 * sizeof(float2) +
-         static_cast<size_t>(kWarps) * KV * 8 * 4 + static_cast<size_t>(2) * kStageT * KV * R * kGroups;
+         static_cast<size_t>(kTiles) * KV * 8 * 4 + static_cast<size_t>(kTiles) * 2 * 32 * 16 +
+         static_cast<size_t>(2) * kStageT * KV * R * kGroups;
 }
 
 size_t mma_values_smem_bytes(int R, int KV, int q_heads, int n_codes) {
-  size_t stages = static_cast<size_t>(2) * kStageT * KV * R * kGroups;
-  const size_t xred = static_cast<size_t>(kWarps) * 32 * 33 * 4;
-  if (KV < kWarps && stages < xred) stages = xred;
-  const size_t scores = static_cast<size_t>(2) * (kStageT / kTileT) * q_heads * 16 * 4;
-  return static_cast<size_t>(512) * n_codes + stages + scores;
+  // code stages and score stages; after the loop the same bytes hold the per-warp partial
+  // sums when several warps share a KV head
+  size_t stages = static_cast<size_t>(2) * kStageT * KV * R * kGroups +
+                  static_cast<size_t>(2) * kTiles * q_heads * 16 * 4;
+  const size_t xred = static_cast<size_t>(kMmaWarps) * 32 * 33 * 4;
+  if (KV < kMmaWarps && stages < xred) stages = xred;
+  return static_cast<size_t>(512) * n_codes + stages;
 }
 
 bool mma_supported(int R, int q_heads, int kv_heads, int n_codes) {

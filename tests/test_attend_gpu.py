@@ -216,3 +216,47 @@ def test_workspace_too_small_is_rejected(api, gpu):
     with pytest.raises(api.CommVQError) as e:
         api.attend_decode(cfg, z, codes, codes, offs, 256, cb, cb, workspace=ws)
     assert e.value.status == 4
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_long_split_refreshes_phasors(api, gpu, algo):
+    """One split of 4500 positions: the decode-and-rotate path advances its phasors by
+    recurrence and rebuilds them exactly every 16 stages (2048 positions)."""
+    w, kc, vc, kcb, vcb = _encoded_inputs(synth.WORKLOADS[1], T=4500)
+    q = synth.queries(w)
+    offs = w.offsets()
+    out, lse = _run(api, w, q, kc, vc, offs, kcb, vcb, gpu, algo, splits=1)
+    ref, ref_lse = O.attend_codes(q_as_f64(w, q), kc, vc, offs, kcb, vcb, w.rope_base)
+    assert rel_err(out, ref) <= tol_for(w)
+    assert np.allclose(lse, ref_lse, rtol=1e-3, atol=5e-3)
+
+
+SHAPES = [
+    # (q_heads, kv_heads, R, n_codes, q_dtype)
+    (32, 8, 2, 256, "f16"),
+    (32, 8, 2, 256, "f32"),
+    (8, 8, 2, 256, "bf16"),     # no grouping
+    (16, 2, 2, 256, "bf16"),    # 8 query heads per KV head
+    (8, 4, 1, 256, "bf16"),
+    (4, 1, 2, 64, "bf16"),      # smaller codebook: run-time entry count, codes checked
+    (6, 2, 1, 100, "f32"),
+]
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "q%d_kv%d_R%d_N%d_%s" % s)
+def test_shapes_and_query_types(api, gpu, algo, shape):
+    Hq, Hkv, R, Nc, qdt = shape
+    w = synth.WORKLOADS[1].with_(q_heads=Hq, kv_heads=Hkv, R=R, n_codes=Nc, q_dtype=qdt,
+                                 batch=3, ragged=(100, 700), codebook="normal")
+    kcb = synth.normal_codebook(w, True)
+    vcb = synth.normal_codebook(w, False)
+    offs = w.offsets()
+    total = int(offs[-1])
+    kc = synth.uniform_codes(w, True, total)
+    vc = synth.uniform_codes(w, False, total)
+    q = synth.queries(w)
+    out, lse = _run(api, w, q, kc, vc, offs, kcb, vcb, gpu, algo)
+    ref, ref_lse = O.attend_codes(q_as_f64(w, q), kc, vc, offs, kcb, vcb, w.rope_base)
+    assert rel_err(out, ref) <= tol_for(w)
+    assert np.allclose(lse, ref_lse, rtol=1e-3, atol=5e-3)
