@@ -23,6 +23,7 @@ STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "WORKSPACE"
 
 EXPORTS = ("commvq_encode", "commvq_attend_workspace_bytes", "commvq_attend_decode",
            "commvq_attend_decode_noalloc", "commvq_em_workspace_bytes", "commvq_em_step",
+           "commvq_em_step_soft",
            "commvq_workspace_error", "commvq_status_string", "commvq_abi_version")
 
 
@@ -64,6 +65,8 @@ def _load():
     lib.commvq_em_workspace_bytes.restype = SZ
     lib.commvq_em_step.argtypes = [CP, P, I64, P, P, P, P, SZ, P]
     lib.commvq_em_step.restype = I32
+    lib.commvq_em_step_soft.argtypes = [CP, P, I64, P, ctypes.c_float, P, P, SZ, P]
+    lib.commvq_em_step_soft.restype = I32
     lib.commvq_workspace_error.argtypes = [P, ctypes.POINTER(I32), P]
     lib.commvq_workspace_error.restype = I32
     lib.commvq_status_string.argtypes = [I32]
@@ -220,6 +223,23 @@ def em_step(cfg: Config, rows: torch.Tensor, codebook_round: torch.Tensor,
     _check(LIB.commvq_em_step(ctypes.byref(cc), _ptr(rows), int(N), _ptr(codebook_round),
                               _ptr(codes_out), _ptr(sse_out), _ptr(workspace), workspace.numel(),
                               _stream(stream)), "commvq_em_step")
+    return codebook_round
+
+
+def em_step_soft(cfg: Config, rows: torch.Tensor, codebook_round: torch.Tensor, tau: float,
+                 sse_out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                 stream=None):
+    """commvq_em_step_soft: soft-assignment EM step at temperature tau, in place."""
+    N = rows.shape[0]
+    if workspace is None:
+        n = em_workspace_bytes(cfg, N)
+        if n == 0:
+            raise CommVQError(1, "commvq_em_workspace_bytes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=rows.device)
+    cc = cfg.c()
+    _check(LIB.commvq_em_step_soft(ctypes.byref(cc), _ptr(rows), int(N), _ptr(codebook_round),
+                                   float(tau), _ptr(sse_out), _ptr(workspace), workspace.numel(),
+                                   _stream(stream)), "commvq_em_step_soft")
     return codebook_round
 
 

@@ -417,12 +417,14 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
           mma16816(acc, A[0][0], A[0][1], A[0][2], A[0][3], b0.x, b0.y);
           mma16816(acc, A[1][0], A[1][1], A[1][2], A[1][3], b1.x, b1.y);
         }
-        // Add the two halves' partial S: half 1 writes, both meet at the pair's barrier,
-        // half 0 reads. The buffer alternates with kv, so half 1 can run one kv ahead.
+        // Add the two halves' partial S. For even kv half 1 hands its partial to half 0, for
+        // odd kv the reverse, so the finishing work (stores, maxima) alternates between the
+        // two warps. The buffer alternates with kv, so the handing half can run one kv ahead.
+        const int finisher = kv & 1;
         float4* xs = xch + (tile * 2 + (kv & 1)) * 32 + lane;
-        if (half) *xs = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        if (half != finisher) *xs = make_float4(acc[0], acc[1], acc[2], acc[3]);
         named_barrier_sync(1 + tile, 64);
-        if (half) continue;
+        if (half != finisher) continue;
         {
           const float4 o = *xs;
           acc[0] += o.x;
@@ -459,7 +461,8 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
     __syncthreads();
   }
 
-  // split maxima: the half-0 warp of each tile kept a row of maxima; take the max over tiles
+  // split maxima: each tile's warp pair kept a row of maxima (entries of even kv heads written
+  // by half 0, odd by half 1); take the max over tiles
   for (int e = tid; e < KV * 8; e += kMmaThreads) {
     const int kv = e >> 3, col = e & 7;
     if (col >= G) continue;

@@ -8,6 +8,8 @@
 // partials in chunk order and writes (float)(sum / count), keeping entries that no row
 // chose; it also reduces the SSE partials in a fixed order. The whole step is therefore
 // deterministic run to run.
+#include <math.h>
+
 #include "common.cuh"
 
 namespace commvq {
@@ -19,18 +21,26 @@ constexpr int kChunkRows = 512;                   // rows per CTA (4096 rows fil
 constexpr int kTile = 1024;                       // codebook entries staged per pass
 constexpr int kMaxCodes = 4096;
 
+constexpr int kSoftChunkRows = 256;               // rows per CTA of the soft step
+
+// Workspace regions, sized for the larger chunk count of the two steps: per (chunk, group,
+// entry) fp64 sums of g scalars, then 8 bytes (int32 counts of the hard step or fp64 weight
+// sums of the soft step), then per (chunk, group) fp64 SSE partials.
 struct EmLayout {
-  int64_t chunks;
+  int64_t chunks;        // hard-step chunks
+  int64_t soft_chunks;   // soft-step chunks
   size_t sums_off, counts_off, sse_off, total;
 };
 
 EmLayout em_layout(int64_t N, int G, int Nc) {
   EmLayout L;
   L.chunks = (N + kChunkRows - 1) / kChunkRows;
+  L.soft_chunks = (N + kSoftChunkRows - 1) / kSoftChunkRows;
+  const int64_t cap = L.soft_chunks > L.chunks ? L.soft_chunks : L.chunks;
   L.sums_off = 0;
-  L.counts_off = round_up(L.sums_off + sizeof(double) * L.chunks * G * Nc * kG, 256);
-  L.sse_off = round_up(L.counts_off + sizeof(int32_t) * L.chunks * G * Nc, 256);
-  L.total = round_up(L.sse_off + sizeof(double) * L.chunks * G, 256);
+  L.counts_off = round_up(L.sums_off + sizeof(double) * cap * G * Nc * kG, 256);
+  L.sse_off = round_up(L.counts_off + sizeof(double) * cap * G * Nc, 256);
+  L.total = round_up(L.sse_off + sizeof(double) * cap * G, 256);
   return L;
 }
 
@@ -151,6 +161,132 @@ em_update_kernel(int64_t chunks, int G, int Nc, float* __restrict__ cb, const do
   }
 }
 
+// Soft assignment (one step at temperature tau): responsibilities w = exp(-(d - d_min)/tau)/Z
+// over a group's entries, with the encoder's exact fp32 distances. Phase 1 (row threads)
+// streams the codebook once per row keeping the running minimum and the partition sum
+// (rescaled when the minimum drops); phase 2 (entry threads) recomputes the same distances
+// against the chunk's rows, staged in shared memory, and accumulates w x and w in fp64 in row
+// order. Distances, minima and weights are fp32; sums are fp64.
+__global__ void __launch_bounds__(kThreads)
+em_soft_assign_kernel(const float* __restrict__ rows, int64_t N, int d, int Nc,
+                      const float* __restrict__ cb, float tau, double* __restrict__ psum,
+                      double* __restrict__ pw, double* __restrict__ psse) {
+  __shared__ float4 tile[kTile * 2];
+  __shared__ float4 xs[kSoftChunkRows * 2];
+  __shared__ float dmin_s[kSoftChunkRows];
+  __shared__ float zinv_s[kSoftChunkRows];
+  __shared__ double red[kThreads];
+  const int G = d / kG;
+  const int j = blockIdx.y;
+  const int64_t chunk = blockIdx.x;
+  const int64_t base = chunk * kSoftChunkRows;
+  const int rows_here = static_cast<int>(min(static_cast<int64_t>(kSoftChunkRows), N - base));
+  const float* sub_cb = cb + static_cast<int64_t>(j) * Nc * kG;
+  const float inv_tau = 1.0f / tau;
+
+  // phase 1: one row per thread
+  const int li = threadIdx.x;
+  float x[kG];
+  const bool valid = li < rows_here;
+  if (valid) {
+    load_row8(rows + (base + li) * d + j * kG, x);
+    xs[2 * li] = make_float4(x[0], x[1], x[2], x[3]);
+    xs[2 * li + 1] = make_float4(x[4], x[5], x[6], x[7]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < kG; ++k) x[k] = 0.0f;
+  }
+  float m = __int_as_float(0x7f800000), Z = 0.0f;
+  for (int c0 = 0; c0 < Nc; c0 += kTile) {
+    const int n = min(kTile, Nc - c0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < 2 * n; e += kThreads)
+      tile[e] = __ldg(reinterpret_cast<const float4*>(sub_cb + static_cast<int64_t>(c0) * kG) + e);
+    __syncthreads();
+    for (int c = 0; c < n; ++c) {
+      const float4 lo = tile[2 * c], hi = tile[2 * c + 1];
+      Nearest nb;
+      nearest_init(nb);
+      nearest_step<false>(nb, x, lo, hi, 0);
+      const float dist = nb.best;
+      if (dist < m) {
+        Z = Z * expf((dist - m) * inv_tau) + 1.0f;
+        m = dist;
+      } else {
+        Z += expf((m - dist) * inv_tau);
+      }
+    }
+  }
+  if (valid) {
+    dmin_s[li] = m;
+    zinv_s[li] = 1.0f / Z;
+  }
+  red[threadIdx.x] = valid ? static_cast<double>(m) : 0.0;
+  __syncthreads();
+  for (int w = kThreads / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) psse[chunk * G + j] = red[0];
+
+  // phase 2: one entry per thread, rows in order
+  for (int c = threadIdx.x; c < Nc; c += kThreads) {
+    float e_c[kG];
+    load_row8(sub_cb + static_cast<int64_t>(c) * kG, e_c);
+    const float4 lo = make_float4(e_c[0], e_c[1], e_c[2], e_c[3]);
+    const float4 hi = make_float4(e_c[4], e_c[5], e_c[6], e_c[7]);
+    double acc[kG];
+#pragma unroll
+    for (int k = 0; k < kG; ++k) acc[k] = 0.0;
+    double wsum = 0.0;
+    for (int r = 0; r < rows_here; ++r) {
+      const float4 a = xs[2 * r], b = xs[2 * r + 1];
+      const float xr[kG] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      Nearest nb;
+      nearest_init(nb);
+      nearest_step<false>(nb, xr, lo, hi, 0);
+      const float w = expf((dmin_s[r] - nb.best) * inv_tau) * zinv_s[r];
+      if (w == 0.0f) continue;
+      const double wd = static_cast<double>(w);
+      wsum += wd;
+#pragma unroll
+      for (int k = 0; k < kG; ++k) acc[k] = fma(wd, static_cast<double>(xr[k]), acc[k]);
+    }
+    const int64_t at = (chunk * G + j) * Nc + c;
+#pragma unroll
+    for (int k = 0; k < kG; ++k) psum[at * kG + k] = acc[k];
+    pw[at] = wsum;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+em_soft_update_kernel(int64_t chunks, int G, int Nc, float* __restrict__ cb, const double* __restrict__ psum,
+                      const double* __restrict__ pw, const double* __restrict__ psse,
+                      double* __restrict__ sse_out) {
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;   // j * Nc + c
+  if (e < static_cast<int64_t>(G) * Nc) {
+    double acc[kG];
+#pragma unroll
+    for (int k = 0; k < kG; ++k) acc[k] = 0.0;
+    double wsum = 0.0;
+    for (int64_t ch = 0; ch < chunks; ++ch) {
+      const int64_t at = ch * G * Nc + e;
+      wsum += pw[at];
+#pragma unroll
+      for (int k = 0; k < kG; ++k) acc[k] += psum[at * kG + k];
+    }
+    if (wsum > 0.0) {
+#pragma unroll
+      for (int k = 0; k < kG; ++k) cb[e * kG + k] = __double2float_rn(acc[k] / wsum);
+    }
+  }
+  if (sse_out && blockIdx.x == 0 && threadIdx.x == 0) {
+    double s = 0.0;
+    for (int64_t i = 0; i < chunks * G; ++i) s += psse[i];
+    *sse_out = s;
+  }
+}
+
 }  // namespace
 }  // namespace commvq
 
@@ -162,7 +298,7 @@ static commvq_status em_check(const commvq_config* cfg, int64_t N) {
   if (d <= 0 || g <= 0 || d % g || g % 2 || Nc < 1 || Nc > 65536 || N < 1) return COMMVQ_ERR_INVALID_ARG;
   if (cfg->code_bytes != (Nc <= 256 ? 1 : 2)) return COMMVQ_ERR_INVALID_ARG;
   if (g != kG || Nc > kMaxCodes) return COMMVQ_ERR_UNSUPPORTED;
-  if ((N + kChunkRows - 1) / kChunkRows > INT32_MAX) return COMMVQ_ERR_UNSUPPORTED;
+  if ((N + kSoftChunkRows - 1) / kSoftChunkRows > INT32_MAX) return COMMVQ_ERR_UNSUPPORTED;
   return COMMVQ_OK;
 }
 
@@ -195,5 +331,32 @@ extern "C" commvq_status commvq_em_step(const commvq_config* cfg, const float* r
   if (rc != COMMVQ_OK) return rc;
   const unsigned g2 = static_cast<unsigned>((static_cast<int64_t>(G) * Nc + kThreads - 1) / kThreads);
   em_update_kernel<<<g2, kThreads, 0, st>>>(L.chunks, G, Nc, codebook_round, psum, pcnt, psse, sse_out);
+  return launch_status();
+}
+
+extern "C" commvq_status commvq_em_step_soft(const commvq_config* cfg, const float* rows, int64_t N,
+                                             float* codebook_round, float tau, double* sse_out,
+                                             void* workspace, size_t workspace_bytes, void* stream) {
+  const commvq_status cs = em_check(cfg, N);
+  if (cs != COMMVQ_OK) return cs;
+  if (!(tau > 0.0f) || !isfinite(tau)) return COMMVQ_ERR_INVALID_ARG;
+  if (!rows || !codebook_round || !workspace) return COMMVQ_ERR_INVALID_ARG;
+  if (!aligned(rows, 16) || !aligned(codebook_round, 16) || !aligned(sse_out, 8) || !aligned(workspace, 256))
+    return COMMVQ_ERR_INVALID_ARG;
+  const int G = cfg->d / kG, Nc = cfg->n_codes;
+  const EmLayout L = em_layout(N, G, Nc);
+  if (workspace_bytes < L.total) return COMMVQ_ERR_WORKSPACE;
+  const int64_t chunks = L.soft_chunks;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  double* psum = reinterpret_cast<double*>(ws + L.sums_off);
+  double* pw = reinterpret_cast<double*>(ws + L.counts_off);
+  double* psse = reinterpret_cast<double*>(ws + L.sse_off);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  em_soft_assign_kernel<<<dim3(static_cast<unsigned>(chunks), G), kThreads, 0, st>>>(
+      rows, N, cfg->d, Nc, codebook_round, tau, psum, pw, psse);
+  commvq_status rc = launch_status();
+  if (rc != COMMVQ_OK) return rc;
+  const unsigned g2 = static_cast<unsigned>((static_cast<int64_t>(G) * Nc + kThreads - 1) / kThreads);
+  em_soft_update_kernel<<<g2, kThreads, 0, st>>>(chunks, G, Nc, codebook_round, psum, pw, psse, sse_out);
   return launch_status();
 }

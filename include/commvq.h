@@ -174,7 +174,8 @@ commvq_status commvq_attend_decode_noalloc(const commvq_config* cfg, const void*
                                            const float* v_codebook, float* out, float* lse,
                                            const commvq_attend_options* options, void* stream);
 
-/* Bytes of device workspace commvq_em_step needs for N rows. 0 for invalid input. */
+/* Bytes of device workspace commvq_em_step and commvq_em_step_soft need for N rows. 0 for
+ * invalid input. */
 size_t commvq_em_workspace_bytes(const commvq_config* cfg, int64_t N);
 
 /* One EM step for one residual round's codebook (review: codebook fit by EM, Algorithm 1
@@ -198,6 +199,21 @@ size_t commvq_em_workspace_bytes(const commvq_config* cfg, int64_t N);
 commvq_status commvq_em_step(const commvq_config* cfg, const float* rows, int64_t N,
                              float* codebook_round, void* codes_out, double* sse_out,
                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* One soft-assignment EM step at temperature tau (review, "Assumptions & free parameters":
+ * the paper stabilises its EM with soft assignment and annealing; lowering tau from call to
+ * call is the annealing). For each (row n, group j), with the encoder's fp32 distances d_c
+ * against the input codebook and d_min = min_c d_c:
+ *   w_c = exp(-(d_c - d_min) / tau) / sum_c' exp(-(d_c' - d_min) / tau)        (fp32),
+ *   entry (j, c) = (float)(sum_n w_c x_n / sum_n w_c) with fp64 sums; an entry whose weight
+ *   sum is 0 keeps its value.
+ * sse_out: sum over (row, group) of d_min (the hard distortion against the input codebook).
+ * tau must be finite and > 0 (COMMVQ_ERR_INVALID_ARG otherwise); as tau -> 0 the step tends
+ * to commvq_em_step. Arguments, workspace (commvq_em_workspace_bytes covers both steps) and
+ * limits are those of commvq_em_step. Deterministic run to run. */
+commvq_status commvq_em_step_soft(const commvq_config* cfg, const float* rows, int64_t N,
+                                  float* codebook_round, float tau, double* sse_out,
+                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /* The device error word in an attention workspace: synchronises `stream`, copies the word
  * to the host and writes it to *device_error (0 = none; bit 0 = a code >= Nc' was seen

@@ -334,3 +334,62 @@ int oracle_values_hist(const double* p, const int32_t* codes, int64_t code_strid
   free(H);
   return ORACLE_OK;
 }
+
+/* One soft-assignment EM step with temperature tau (review, "Assumptions & free
+ * parameters": the paper stabilises its EM with soft assignment and annealing; the caller
+ * lowers tau from step to step). For each (row n, group j), with the encoder's fp32
+ * distances d_c and d_min = min_c d_c:
+ *   w_c = exp(-(d_c - d_min) / tau) / sum_c' exp(-(d_c' - d_min) / tau)      (fp64),
+ * and each entry becomes (float)(sum_n w x / sum_n w); an entry whose weight sum is 0 keeps
+ * its value. sse_out = sum over (row, group) of d_min (fp64, the hard distortion against the
+ * input codebook). tau must be > 0 (tau -> 0 gives the hard step when there are no ties). */
+int oracle_em_soft_step(const float* rows, int64_t N, int d, int g, int n_codes, float* cb, double tau,
+                        double* sse_out) {
+  if (!valid_shape(d, g, 1, n_codes) || N < 0 || !rows || !cb || !(tau > 0.0)) return ORACLE_BAD_ARG;
+  const int G = d / g;
+  double* sum = (double*)calloc((size_t)G * n_codes * g, sizeof(double));
+  double* wsum = (double*)calloc((size_t)G * n_codes, sizeof(double));
+  double* w = (double*)malloc(sizeof(double) * (size_t)n_codes);
+  float* dist = (float*)malloc(sizeof(float) * (size_t)n_codes);
+  if (!sum || !wsum || !w || !dist) { free(sum); free(wsum); free(w); free(dist); return ORACLE_NO_MEM; }
+  double sse = 0.0;
+  for (int64_t n = 0; n < N; ++n)
+    for (int j = 0; j < G; ++j) {
+      const float* x = rows + n * d + (int64_t)j * g;
+      const float* sub = cb + (int64_t)j * n_codes * g;
+      float dmin = INFINITY;
+      for (int c = 0; c < n_codes; ++c) {
+        float acc = 0.0f;
+        for (int k = 0; k < g; ++k) {
+          float e = x[k] - sub[(int64_t)c * g + k];
+          acc = fmaf(e, e, acc);
+        }
+        dist[c] = acc;
+        if (acc < dmin) dmin = acc;
+      }
+      sse += (double)dmin;
+      double Z = 0.0;
+      for (int c = 0; c < n_codes; ++c) {
+        w[c] = exp(-((double)dist[c] - (double)dmin) / tau);
+        Z += w[c];
+      }
+      for (int c = 0; c < n_codes; ++c) {
+        const double wc = w[c] / Z;
+        if (wc == 0.0) continue;
+        wsum[(int64_t)j * n_codes + c] += wc;
+        for (int k = 0; k < g; ++k) sum[((int64_t)j * n_codes + c) * g + k] += wc * (double)x[k];
+      }
+    }
+  for (int j = 0; j < G; ++j)
+    for (int c = 0; c < n_codes; ++c) {
+      const double m = wsum[(int64_t)j * n_codes + c];
+      if (!(m > 0.0)) continue;
+      for (int k = 0; k < g; ++k) {
+        const int64_t at = ((int64_t)j * n_codes + c) * g + k;
+        cb[at] = (float)(sum[at] / m);
+      }
+    }
+  free(sum); free(wsum); free(w); free(dist);
+  if (sse_out) *sse_out = sse;
+  return ORACLE_OK;
+}

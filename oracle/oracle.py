@@ -47,8 +47,9 @@ def lib():
         _lib.oracle_attend.argtypes = [P, P, P, P, I, I, I, I, ctypes.c_double, P, P]
         _lib.oracle_em_step.argtypes = [P, I64, I, I, I, P, P, P]
         _lib.oracle_values_hist.argtypes = [P, P, I64, I64, I, I, I, I, P, P, P]
+        _lib.oracle_em_soft_step.argtypes = [P, I64, I, I, I, P, ctypes.c_double, P]
         for f in ("oracle_encode", "oracle_decode", "oracle_scores_plain", "oracle_scores_table",
-                  "oracle_attend", "oracle_em_step", "oracle_values_hist"):
+                  "oracle_attend", "oracle_em_step", "oracle_values_hist", "oracle_em_soft_step"):
             getattr(_lib, f).restype = ctypes.c_int
     return _lib
 
@@ -183,6 +184,18 @@ def em_step(rows: np.ndarray, cb_round: np.ndarray):
     _check(lib().oracle_em_step(_p(rf), N, d, g, Nc, _p(cb), _p(codes), ctypes.byref(sse)),
            "em_step")
     return cb, codes, float(sse.value)
+
+
+def em_soft_step(rows: np.ndarray, cb_round: np.ndarray, tau: float):
+    """One soft-assignment EM step at temperature tau. Returns (new codebook, sse)."""
+    G, Nc, g = cb_round.shape
+    d = G * g
+    rf = _c(rows, np.float32)
+    cb = _c(cb_round, np.float32).copy()
+    sse = ctypes.c_double(0.0)
+    _check(lib().oracle_em_soft_step(_p(rf), rf.shape[0], d, g, Nc, _p(cb), float(tau),
+                                     ctypes.byref(sse)), "em_soft_step")
+    return cb, float(sse.value)
 
 
 def forgy_init(rows: np.ndarray, idx: np.ndarray, g: int) -> np.ndarray:

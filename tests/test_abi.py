@@ -131,3 +131,11 @@ def test_encode_and_em_reject_bad_arguments(api):
     assert em(ctypes.byref(cc), P(FAKE), 100, P(FAKE), None, None, P(FAKE), 16, None) == 4
     c3 = _cfg(api, n_codes=5000).c()
     assert em(ctypes.byref(c3), P(FAKE), 100, P(FAKE), None, None, P(FAKE), 1 << 30, None) == UNSUP
+
+
+def test_soft_em_rejects_bad_temperature(api):
+    P = ctypes.c_void_p
+    cc = _cfg(api).c()
+    f = api.LIB.commvq_em_step_soft
+    for tau in (0.0, -1.0, float("nan"), float("inf")):
+        assert f(ctypes.byref(cc), P(FAKE), 100, P(FAKE), tau, None, P(FAKE), 1 << 30, None) == 1

@@ -83,3 +83,48 @@ def test_em_step_deterministic(api, gpu):
     b = _gpu_step(api, cfg, rows, cb, gpu)
     assert np.array_equal(a[0].view(np.uint32), b[0].view(np.uint32))
     assert a[2] == b[2]
+
+
+def _gpu_soft(api, cfg, rows, cb_round, tau, gpu):
+    r = torch.from_numpy(rows).to(gpu)
+    cb = torch.from_numpy(cb_round.copy()).to(gpu)
+    sse = torch.zeros(1, dtype=torch.float64, device=gpu)
+    api.em_step_soft(cfg, r, cb, tau, sse_out=sse)
+    torch.cuda.synchronize()
+    return cb.cpu().numpy(), float(sse.item())
+
+
+@pytest.mark.parametrize("tau", [0.5, 4.0, 40.0])
+def test_soft_em_step_matches_oracle(api, gpu, tau):
+    """Soft assignment at three temperatures on the 2-bit layer's key fitting rows."""
+    w = synth.WORKLOADS[1]
+    cfg = api.Config(d=128, g=8, R=1, n_codes=256, q_heads=32, kv_heads=8)
+    rows = synth.fit_rows(w, True)
+    cb = O.forgy_init(rows, synth.forgy_indices(w, True, 0, rows.shape[0]), 8)
+    got, sse = _gpu_soft(api, cfg, rows, cb, tau, gpu)
+    want, want_sse = O.em_soft_step(rows, cb, tau)
+    scale = np.abs(want).max()
+    assert np.abs(got - want).max() <= 2e-5 * scale
+    assert abs(sse - want_sse) <= 1e-12 * abs(want_sse)
+
+
+def test_soft_em_cold_limit_is_the_hard_step(api, gpu):
+    w = synth.WORKLOADS[1]
+    cfg = api.Config(d=128, g=8, R=1, n_codes=256, q_heads=32, kv_heads=8)
+    rows = synth.fit_rows(w, False)
+    cb = O.forgy_init(rows, synth.forgy_indices(w, False, 0, rows.shape[0]), 8)
+    soft, _ = _gpu_soft(api, cfg, rows, cb, 1e-30, gpu)
+    hard, _, _ = O.em_step(rows, cb)
+    assert _ulp_diff(soft, hard) <= 1
+
+
+def test_soft_em_deterministic_and_small_codebooks(api, gpu):
+    rng = np.random.default_rng(9)
+    cfg = api.Config(d=32, g=8, R=1, n_codes=300, q_heads=1, kv_heads=1)
+    rows = rng.standard_normal((777, 32)).astype(np.float32)
+    cb = rng.standard_normal((4, 300, 8)).astype(np.float32)
+    a, sa = _gpu_soft(api, cfg, rows, cb, 2.0, gpu)
+    b, sb = _gpu_soft(api, cfg, rows, cb, 2.0, gpu)
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32)) and sa == sb
+    want, _ = O.em_soft_step(rows, cb, 2.0)
+    assert np.abs(a - want).max() <= 2e-5 * np.abs(want).max()

@@ -448,3 +448,50 @@ def test_em_separated_clusters_converge_to_means():
     for c in range(Nc):
         mean = rows[labels == c].astype(np.float64).mean(0)
         assert np.allclose(cb[0, c], mean, rtol=0, atol=1e-5)
+
+
+# ----------------------------------------------------------------------------------------
+# soft-assignment EM step (annealing): limits and brute force
+
+def test_soft_em_zero_temperature_is_the_hard_step():
+    rng = np.random.default_rng(51)
+    rows = rng.standard_normal((300, 32)).astype(np.float32)
+    cb = rng.standard_normal((4, 20, 8)).astype(np.float32)
+    hard, _, sse_h = O.em_step(rows, cb)
+    soft, sse_s = O.em_soft_step(rows, cb, 1e-30)
+    assert np.array_equal(hard, soft)
+    assert sse_h == sse_s
+
+
+def test_soft_em_infinite_temperature_is_the_global_mean():
+    rng = np.random.default_rng(52)
+    rows = rng.standard_normal((200, 16)).astype(np.float32)
+    cb = rng.standard_normal((2, 7, 8)).astype(np.float32)
+    soft, _ = O.em_soft_step(rows, cb, 1e30)
+    mean = rows.astype(np.float64).reshape(200, 2, 8).mean(0)
+    for c in range(7):
+        assert np.allclose(soft[:, c], mean, rtol=0, atol=1e-6)
+
+
+def test_soft_em_brute_force():
+    rng = np.random.default_rng(53)
+    N, G, Nc, g, tau = 30, 2, 5, 8, 0.7
+    rows = rng.standard_normal((N, G * g)).astype(np.float32)
+    cb = rng.standard_normal((G, Nc, g)).astype(np.float32)
+    soft, sse = O.em_soft_step(rows, cb, tau)
+    want = cb.astype(np.float64).copy()
+    want_sse = 0.0
+    for j in range(G):
+        num = np.zeros((Nc, g)); den = np.zeros(Nc)
+        for n in range(N):
+            x = rows[n, j * g:(j + 1) * g]
+            _, dists = brute_nearest(x, cb[j])
+            dd = np.array([float(v) for v in dists])
+            want_sse += dd.min()
+            w = np.exp(-(dd - dd.min()) / tau)
+            w /= w.sum()
+            num += w[:, None] * x.astype(np.float64)[None, :]
+            den += w
+        want[j] = num / den[:, None]
+    assert np.allclose(soft, want.astype(np.float32), rtol=1e-6, atol=1e-7)
+    assert sse == pytest.approx(want_sse, rel=1e-12)
