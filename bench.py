@@ -1,9 +1,12 @@
 """Decode-attention benchmark over a CommVQ-compressed KV cache on B200.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME]
+                    [--path fused|naive]
 
 One step is one commvq_attend_decode over the whole workload (all heads of one layer,
-every cached position). The default workload is the LLaMA-3.1-8B-shaped 2-bit layer:
+every cached position). With --path naive a step is the comparator the CommVQ review measures
+against instead: commvq_decompress of the whole cache into dense 16-bit rows, then
+commvq_dense_decode over them. The default workload is the LLaMA-3.1-8B-shaped 2-bit layer:
 batch 1, 32 query / 8 KV heads, d = 128, T = 32768, R = 2, g = 8, Nc' = 256. Inputs are
 seeded synthetic rows, codebooks fit on the GPU by the library's EM step, codes made by
 the library's encoder. Under torchrun each rank runs its own replica (weak scaling; the
@@ -42,6 +45,12 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--algo", type=int, default=0)
     ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--path", default="fused", choices=["fused", "naive"],
+                    help="fused: attention on the codes; naive: decompress the cache to dense "
+                         "16-bit rows, then dense flash-decoding (the review's comparator)")
+    ap.add_argument("--naive-dtype", default="bf16", choices=["bf16", "f16"])
+    ap.add_argument("--unprepared", action="store_true",
+                    help="rebuild the codebook images and RoPE tables in every step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-heads", type=int, default=8, help="query heads in the oracle sample")
     return ap.parse_args()
@@ -65,7 +74,8 @@ def measured_peaks():
 
 
 KERNEL_SOURCES = {"attend_table_kernel": "attend_table.cu",
-                  "attend_scores_kernel+attend_values_kernel": "attend_mma.cu"}
+                  "attend_scores_kernel+attend_values_kernel": "attend_mma.cu",
+                  "dense_decode_kernel": "naive.cu"}
 
 
 def kernel_source_sha(kernel: str):
@@ -95,7 +105,7 @@ def main_kernel(api, cfg, algo):
             cfg.q_heads % cfg.kv_heads == 0 and cfg.q_heads // cfg.kv_heads <= 8
         run = api.ATTN_DECODE_MMA if mma_ok else api.ATTN_TABLE
     if run == api.ATTN_DECODE_MMA:
-        return "attend_scores_kernel+attend_values_kernel", 4   # prep, scores, values, merge
+        return "attend_scores_kernel+attend_values_kernel", 3   # scores, values, merge
     return "attend_table_kernel", 2                             # table, merge
 
 
@@ -226,16 +236,39 @@ def run_ours(args, w, rank, world, dev):
     n_copies = max(1, math.ceil(3 * l2 / code_bytes))
     kcs = [kc] + [kc.clone() for _ in range(n_copies - 1)]
     vcs = [vc] + [vc.clone() for _ in range(n_copies - 1)]
-    ws = api.attend_workspace(cfg, w.batch, max_T, dev, args.algo, args.splits)
     out = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32, device=dev)
     lse = torch.empty((w.batch, w.q_heads), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
     K, W = args.steps, args.warmup
+    naive = args.path == "naive"
+    if naive:
+        ndt = torch.bfloat16 if args.naive_dtype == "bf16" else torch.float16
+        k_rows = torch.empty((total_T, w.kv_heads, w.d), dtype=ndt, device=dev)
+        v_rows = torch.empty_like(k_rows)
+        ws = torch.empty(api.decompress_workspace_bytes(cfg, max_T), dtype=torch.uint8, device=dev)
+        ws_dense = torch.empty(api.dense_decode_workspace_bytes(cfg, w.batch, max_T, args.splits),
+                               dtype=torch.uint8, device=dev)
+    else:
+        ws = api.attend_workspace(cfg, w.batch, max_T, dev, args.algo, args.splits)
+        # the layer's codebook-dependent state (fp16 images, RoPE tables), once per layer
+        api.attend_prepare(cfg, w.batch, max_T, kcb, vcb, ws, args.algo, args.splits, stream)
+    prepared = not naive and not args.unprepared
+
+    def attend(kc_i, vc_i, q_i, out_i, lse_i, events=None, prep=None):
+        if naive:
+            api.decompress(cfg, kc_i, vc_i, offs, max_T, kcb, vcb, k_out=k_rows, v_out=v_rows,
+                           workspace=ws, stream=stream)
+            api.dense_decode(cfg, q_i, k_rows, v_rows, offs, max_T, out=out_i, lse=lse_i,
+                             workspace=ws_dense, splits=args.splits, want_lse=lse_i is not None,
+                             stream=stream, main_events=events)
+        else:
+            api.attend_decode(cfg, q_i, kc_i, vc_i, offs, max_T, kcb, vcb, out=out_i, lse=lse_i,
+                              workspace=ws, algo=args.algo, splits=args.splits,
+                              want_lse=lse_i is not None, stream=stream, main_events=events,
+                              prepared=prepared if prep is None else prep)
 
     def step(i, events=None):
-        api.attend_decode(cfg, q, kcs[i % n_copies], vcs[i % n_copies], offs, max_T, kcb, vcb,
-                          out=out, lse=lse, workspace=ws, algo=args.algo, splits=args.splits,
-                          stream=stream, main_events=events)
+        attend(kcs[i % n_copies], vcs[i % n_copies], q, out, lse, events)
 
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(K)]
@@ -248,10 +281,13 @@ def run_ours(args, w, rank, world, dev):
     torch.cuda.synchronize(dev)
     assert api.workspace_error(ws, stream) == 0
 
+    # The timed graph holds only the steps: event nodes between kernels inside a graph cost
+    # time of their own. The main-kernel times come from the same steps launched directly,
+    # where the library records the events around its own launches.
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for i in range(K):
-            step(W + i, evs[i])
+            step(W + i)
     with torch.cuda.stream(stream):
         graph.replay()               # one untimed replay (the graph's own upload)
     torch.cuda.synchronize(dev)
@@ -277,18 +313,67 @@ def run_ours(args, w, rank, world, dev):
         dist.barrier()
     clk = clocks.stop()
     ms = t0.elapsed_time(t1)
-    kern_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
     ms_max = max_over_ranks(ms, world, dev)
+    with torch.cuda.stream(stream):
+        for i in range(K):
+            step(W + i, evs[i])
+    torch.cuda.synchronize(dev)
+    kern_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
     del graph
+    extra = {}
+    if not naive:   # the same steps with the codebook-dependent state rebuilt every step
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=stream):
+            for i in range(K):
+                attend(kcs[i % n_copies], vcs[i % n_copies], q, out, lse, prep=False)
+        with torch.cuda.stream(stream):
+            g2.replay()
+            torch.cuda.synchronize(dev)
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            g2.replay()
+            a1.record(stream)
+        torch.cuda.synchronize(dev)
+        extra = {"prepared_state": {"reused_across_steps": prepared,
+                                    "ms_per_step_rebuilding_it": a0.elapsed_time(a1) / K}}
+        del g2
+    if naive:   # the decompress half alone, for the breakdown
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=stream):
+            for i in range(K):
+                api.decompress(cfg, kcs[i % n_copies], vcs[i % n_copies], offs, max_T, kcb, vcb,
+                               k_out=k_rows, v_out=v_rows, workspace=ws, stream=stream)
+        with torch.cuda.stream(stream):
+            g2.replay()
+            torch.cuda.synchronize(dev)
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            g2.replay()
+            a1.record(stream)
+        torch.cuda.synchronize(dev)
+        dec_ms = a0.elapsed_time(a1) / K
+        del g2
+        dense_bytes = 2 * k_rows.numel() * k_rows.element_size()
+        extra = {"naive": {"rows_dtype": args.naive_dtype, "decompress_ms": dec_ms,
+                           "decompress_gbs": (code_bytes + dense_bytes) / (dec_ms / 1e3) / 1e9,
+                           "dense_kernel_ms": kern_ms,
+                           "dense_rows_bytes": dense_bytes}}
 
     # ---- e2e: one decode step through the API with host buffers -----------------------
-    e2e = run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, ws, stream, dev, torch,
+    e2e = run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, attend, stream, dev, torch,
                   api, synth, world, dist)
 
     value = job_throughput(world, K, total_T, ms_max)
     peak, peak_kind = measured_peaks()
-    kname, launches_per_step = main_kernel(api, cfg, args.algo)
-    achieved = code_bytes / (kern_ms / 1e3) / 1e9
+    if naive:
+        kname, launches_per_step = "dense_decode_kernel", 4   # decompress prep, decompress, dense, merge
+        alg_bytes = 2 * k_rows.numel() * k_rows.element_size()
+    else:
+        kname, launches_per_step = main_kernel(api, cfg, args.algo)
+        if not prepared and kname.startswith("attend_scores"):
+            launches_per_step += 1   # the prep kernel
+        alg_bytes = code_bytes
+    achieved = alg_bytes / (kern_ms / 1e3) / 1e9
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak",
@@ -296,24 +381,30 @@ def run_ours(args, w, rank, world, dev):
         "config": {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
                    "d": w.d, "T": total_T, "R": w.R, "g": w.g, "n_codes": w.n_codes,
                    "q_dtype": w.q_dtype, "parallelism": f"replicas{world}",
-                   "algo": args.algo, "splits": args.splits,
+                   "path": args.path, "algo": args.algo, "splits": args.splits,
                    "l2_defence": f"rotating {n_copies} cache copies ({n_copies * code_bytes / 2**20:.0f} MiB "
                                  f">= 3x L2 {l2 / 2**20:.0f} MiB)",
-                   "timing": "K steps in one CUDA graph, CUDA events on the launch stream"},
+                   "timing": "K steps in one CUDA graph, CUDA events on the launch stream; main-kernel "
+                             "times from the same K steps launched directly, events recorded by the "
+                             "library around its main kernels",
+                   "codebook_state": ("fp16 codebook images and RoPE tables prepared once per layer "
+                                      "(commvq_attend_prepare), reused by every step") if prepared
+                   else "rebuilt inside every step"},
         "compressed_cache_gbs": code_bytes * K / (ms_max / 1e3) / 1e9 * 1.0 / world * world,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
-                     "kernel": kname, "algorithmic_bytes_per_launch": code_bytes,
+                     "kernel": kname, "algorithmic_bytes_per_launch": alg_bytes,
                      "kernel_ms_mean": kern_ms,
                      "traffic": recorded_traffic(kname, w.name)},
         "e2e": e2e,
         "gpu_launches": launches_per_step * K,
         "clocks": clk,
     }
+    result.update(extra)
     return result
 
 
-def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, ws, stream, dev, torch, api,
+def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, attend, stream, dev, torch, api,
             synth, world, dist):
     """Per step: pinned host -> device copy of the step's query and the new position's K/V
     rows, encode of the new position into the cache (position T-1 of sequence 0), decode
@@ -338,8 +429,7 @@ def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, ws, stream, 
         kv_d.copy_(kv_h, non_blocking=True)
         api.encode(cfg, kv_d[0], kcb, codes=kc[last:last + 1], stream=stream)
         api.encode(cfg, kv_d[1], vcb, codes=vc[last:last + 1], stream=stream)
-        api.attend_decode(cfg, qv, kc, vc, offs, max_T, kcb, vcb, out=out_d, workspace=ws,
-                          want_lse=False, stream=stream, algo=args.algo, splits=args.splits)
+        attend(kc, vc, qv, out_d, None)
         out_h.copy_(out_d, non_blocking=True)
 
     with torch.cuda.stream(stream):

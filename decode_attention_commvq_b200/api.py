@@ -18,12 +18,14 @@ LIB_PATH = os.path.join(_PKG, "libcommvq_b200.so")
 
 F32, F16, BF16 = 0, 1, 2
 ATTN_AUTO, ATTN_TABLE, ATTN_DECODE_MMA = 0, 1, 2
+ATTEND_PREPARED = 1
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "WORKSPACE", 5: "DEVICE_CHECK"}
 
-EXPORTS = ("commvq_encode", "commvq_attend_workspace_bytes", "commvq_attend_decode",
+EXPORTS = ("commvq_encode", "commvq_attend_workspace_bytes", "commvq_attend_decode", "commvq_attend_prepare",
            "commvq_attend_decode_noalloc", "commvq_em_workspace_bytes", "commvq_em_step",
-           "commvq_em_step_soft",
+           "commvq_em_step_soft", "commvq_decompress_workspace_bytes", "commvq_decompress",
+           "commvq_dense_decode_workspace_bytes", "commvq_dense_decode",
            "commvq_workspace_error", "commvq_status_string", "commvq_abi_version")
 
 
@@ -36,7 +38,8 @@ class CConfig(ctypes.Structure):
 
 class CAttendOptions(ctypes.Structure):
     _fields_ = [("algo", ctypes.c_int32), ("splits", ctypes.c_int32),
-                ("main_start", ctypes.c_void_p), ("main_stop", ctypes.c_void_p)]
+                ("main_start", ctypes.c_void_p), ("main_stop", ctypes.c_void_p),
+                ("flags", ctypes.c_int32)]
 
 
 class CommVQError(RuntimeError):
@@ -59,6 +62,8 @@ def _load():
     lib.commvq_attend_workspace_bytes.restype = SZ
     lib.commvq_attend_decode.argtypes = [CP, P, I32, P, P, P, I32, I64, P, P, P, P, P, SZ, OP, P]
     lib.commvq_attend_decode.restype = I32
+    lib.commvq_attend_prepare.argtypes = [CP, I32, I64, P, P, P, SZ, OP, P]
+    lib.commvq_attend_prepare.restype = I32
     lib.commvq_attend_decode_noalloc.argtypes = [CP, P, I32, P, P, P, I32, I64, P, P, P, P, OP, P]
     lib.commvq_attend_decode_noalloc.restype = I32
     lib.commvq_em_workspace_bytes.argtypes = [CP, I64]
@@ -67,6 +72,14 @@ def _load():
     lib.commvq_em_step.restype = I32
     lib.commvq_em_step_soft.argtypes = [CP, P, I64, P, ctypes.c_float, P, P, SZ, P]
     lib.commvq_em_step_soft.restype = I32
+    lib.commvq_decompress_workspace_bytes.argtypes = [CP, I64]
+    lib.commvq_decompress_workspace_bytes.restype = SZ
+    lib.commvq_decompress.argtypes = [CP, P, P, P, I32, I64, P, P, I32, P, P, P, SZ, P]
+    lib.commvq_decompress.restype = I32
+    lib.commvq_dense_decode_workspace_bytes.argtypes = [CP, I32, I64, OP]
+    lib.commvq_dense_decode_workspace_bytes.restype = SZ
+    lib.commvq_dense_decode.argtypes = [CP, P, I32, P, P, I32, P, I32, I64, P, P, P, SZ, OP, P]
+    lib.commvq_dense_decode.restype = I32
     lib.commvq_workspace_error.argtypes = [P, ctypes.POINTER(I32), P]
     lib.commvq_workspace_error.restype = I32
     lib.commvq_status_string.argtypes = [I32]
@@ -142,8 +155,8 @@ def encode(cfg: Config, x: torch.Tensor, codebook: torch.Tensor, codes: Optional
     return codes
 
 
-def _opts(algo: int, splits: int, events=None) -> CAttendOptions:
-    o = CAttendOptions(int(algo), int(splits), None, None)
+def _opts(algo: int, splits: int, events=None, flags: int = 0) -> CAttendOptions:
+    o = CAttendOptions(int(algo), int(splits), None, None, int(flags))
     if events is not None:
         o.main_start = ctypes.c_void_p(events[0].cuda_event)
         o.main_stop = ctypes.c_void_p(events[1].cuda_event)
@@ -168,9 +181,10 @@ def attend_decode(cfg: Config, q: torch.Tensor, k_codes: torch.Tensor, v_codes: 
                   v_codebook: torch.Tensor, out: Optional[torch.Tensor] = None,
                   lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                   algo: int = ATTN_AUTO, splits: int = 0, want_lse: bool = True, stream=None,
-                  main_events=None):
+                  main_events=None, prepared: bool = False):
     """commvq_attend_decode: returns (out [B, q_heads, d] f32, lse [B, q_heads] f32 or None).
-    main_events: optional (start, stop) torch.cuda.Event pair recorded around the main kernel."""
+    main_events: optional (start, stop) torch.cuda.Event pair recorded around the main kernel.
+    prepared: the workspace holds this layer's prepared state (attend_prepare)."""
     B = q.shape[0]
     if out is None:
         out = torch.empty((B, cfg.q_heads, cfg.d), dtype=torch.float32, device=q.device)
@@ -179,7 +193,7 @@ def attend_decode(cfg: Config, q: torch.Tensor, k_codes: torch.Tensor, v_codes: 
     if workspace is None:
         workspace = attend_workspace(cfg, B, max_T, q.device, algo, splits)
     cc = cfg.c()
-    o = _opts(algo, splits, main_events)
+    o = _opts(algo, splits, main_events, ATTEND_PREPARED if prepared else 0)
     _check(LIB.commvq_attend_decode(ctypes.byref(cc), _ptr(q), _DT[q.dtype], _ptr(k_codes),
                                     _ptr(v_codes), _ptr(seq_offsets), int(B), int(max_T),
                                     _ptr(k_codebook), _ptr(v_codebook), _ptr(out), _ptr(lse),
@@ -188,14 +202,26 @@ def attend_decode(cfg: Config, q: torch.Tensor, k_codes: torch.Tensor, v_codes: 
     return out, lse
 
 
+def attend_prepare(cfg: Config, B: int, max_T: int, k_codebook: torch.Tensor, v_codebook: torch.Tensor,
+                   workspace: torch.Tensor, algo: int = ATTN_AUTO, splits: int = 0, stream=None):
+    """commvq_attend_prepare: writes the codebook-dependent state into the workspace once, for
+    later attend_decode(..., prepared=True) calls with the same shapes and codebooks."""
+    cc = cfg.c()
+    o = _opts(algo, splits)
+    _check(LIB.commvq_attend_prepare(ctypes.byref(cc), int(B), int(max_T), _ptr(k_codebook), _ptr(v_codebook),
+                                     _ptr(workspace), workspace.numel(), ctypes.byref(o), _stream(stream)),
+           "commvq_attend_prepare")
+    return workspace
+
+
 def attend_decode_noalloc(cfg: Config, q: torch.Tensor, k_codes: torch.Tensor, v_codes: torch.Tensor,
                           seq_offsets: torch.Tensor, max_T: int, k_codebook: torch.Tensor,
                           v_codebook: torch.Tensor, out: torch.Tensor, lse: Optional[torch.Tensor] = None,
-                          algo: int = ATTN_AUTO, splits: int = 0, stream=None):
+                          algo: int = ATTN_AUTO, splits: int = 0, stream=None, prepared: bool = False):
     """commvq_attend_decode_noalloc: the library's fixed internal scratch instead of a
     workspace (for callers that cannot allocate device memory). out/lse are caller-owned."""
     cc = cfg.c()
-    o = _opts(algo, splits)
+    o = _opts(algo, splits, None, ATTEND_PREPARED if prepared else 0)
     _check(LIB.commvq_attend_decode_noalloc(ctypes.byref(cc), _ptr(q), _DT[q.dtype], _ptr(k_codes),
                                             _ptr(v_codes), _ptr(seq_offsets), int(q.shape[0]),
                                             int(max_T), _ptr(k_codebook), _ptr(v_codebook), _ptr(out),
@@ -241,6 +267,68 @@ def em_step_soft(cfg: Config, rows: torch.Tensor, codebook_round: torch.Tensor, 
                                    float(tau), _ptr(sse_out), _ptr(workspace), workspace.numel(),
                                    _stream(stream)), "commvq_em_step_soft")
     return codebook_round
+
+
+def decompress_workspace_bytes(cfg: Config, max_T: int) -> int:
+    cc = cfg.c()
+    return int(LIB.commvq_decompress_workspace_bytes(ctypes.byref(cc), int(max_T)))
+
+
+def decompress(cfg: Config, k_codes: torch.Tensor, v_codes: torch.Tensor, seq_offsets: torch.Tensor,
+               max_T: int, k_codebook: torch.Tensor, v_codebook: torch.Tensor,
+               out_dtype=torch.bfloat16, k_out: Optional[torch.Tensor] = None,
+               v_out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+               stream=None):
+    """commvq_decompress: codes [total_T, kv_heads, R, d/g] -> dense rows (k rotated, v),
+    each [total_T, kv_heads, d] of out_dtype (bf16 or f16)."""
+    N = k_codes.shape[0]
+    shape = (N, cfg.kv_heads, cfg.d)
+    if k_out is None:
+        k_out = torch.empty(shape, dtype=out_dtype, device=k_codes.device)
+    if v_out is None:
+        v_out = torch.empty(shape, dtype=out_dtype, device=k_codes.device)
+    if workspace is None:
+        n = decompress_workspace_bytes(cfg, max_T)
+        if n == 0:
+            raise CommVQError(1, "commvq_decompress_workspace_bytes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=k_codes.device)
+    cc = cfg.c()
+    _check(LIB.commvq_decompress(ctypes.byref(cc), _ptr(k_codes), _ptr(v_codes), _ptr(seq_offsets),
+                                 int(seq_offsets.numel() - 1), int(max_T), _ptr(k_codebook),
+                                 _ptr(v_codebook), _DT[k_out.dtype], _ptr(k_out), _ptr(v_out),
+                                 _ptr(workspace), workspace.numel(), _stream(stream)), "commvq_decompress")
+    return k_out, v_out
+
+
+def dense_decode_workspace_bytes(cfg: Config, B: int, max_T: int, splits: int = 0) -> int:
+    cc = cfg.c()
+    o = _opts(ATTN_AUTO, splits)
+    return int(LIB.commvq_dense_decode_workspace_bytes(ctypes.byref(cc), int(B), int(max_T), ctypes.byref(o)))
+
+
+def dense_decode(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_offsets: torch.Tensor,
+                 max_T: int, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, splits: int = 0, want_lse: bool = True,
+                 stream=None, main_events=None):
+    """commvq_dense_decode over dense rows k, v [total_T, kv_heads, d] (bf16 or f16; keys
+    already rotated). Returns (out [B, q_heads, d] f32, lse [B, q_heads] f32 or None)."""
+    B = q.shape[0]
+    if out is None:
+        out = torch.empty((B, cfg.q_heads, cfg.d), dtype=torch.float32, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, cfg.q_heads), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = dense_decode_workspace_bytes(cfg, B, max_T, splits)
+        if n == 0:
+            raise CommVQError(1, "commvq_dense_decode_workspace_bytes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    cc = cfg.c()
+    o = _opts(ATTN_AUTO, splits, main_events)
+    _check(LIB.commvq_dense_decode(ctypes.byref(cc), _ptr(q), _DT[q.dtype], _ptr(k), _ptr(v), _DT[k.dtype],
+                                   _ptr(seq_offsets), int(B), int(max_T), _ptr(out), _ptr(lse),
+                                   _ptr(workspace), workspace.numel(), ctypes.byref(o), _stream(stream)),
+           "commvq_dense_decode")
+    return out, lse
 
 
 def workspace_error(workspace: torch.Tensor, stream=None) -> int:

@@ -32,84 +32,93 @@ constexpr size_t kHeaderBytes = 256;   // device error word + padding
 
 // Split-T merge (flash-decoding style log-sum-exp combine of the per-split partials):
 // out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, lse = (M + log2 L) ln 2.
-// Grid: (sequence x head, 4 quarters of the 128 output dims). Every block forms the split
-// weights in shared memory; then each of its 32 eight-lane groups adds every 32nd split's
-// 32-dim slice (one float4 per lane, all loads of a group issued together), and the 32
-// group sums are added in a fixed order.
+// Grid: (sequence x head, 4 quarters of the 128 output dims), 256 threads = 32 groups of 8
+// lanes. Lane gl of group grp owns float4 gl of the quarter's 32 dims and the splits grp,
+// grp + 32, ...; it issues the loads of (m, l, its float4 of o) for 8 splits at a time before
+// any arithmetic, folds them in with a running maximum, and the 32 groups are merged in a
+// fixed order through shared memory, so one call's result does not depend on timing.
 constexpr int kCombineThreads = 256;
 constexpr int kCombineQuarters = 4;
+constexpr int kCombineGroups = kCombineThreads / 8;
+constexpr int kCombinePer = 8;   // splits per lane per pass
 constexpr int kMaxSplits = 4096;
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(AttendArgs a, int S) {
-  __shared__ float wts[kMaxSplits];
-  __shared__ float4 acc_s[kCombineThreads / 8][8];
-  __shared__ float red[kCombineThreads / 32];
+  __shared__ float4 acc_s[kCombineGroups][8];
+  __shared__ float ml_s[kCombineGroups][2];
   const int bh = blockIdx.x, quarter = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int grp = tid >> 3, gl = tid & 7;            // 32 groups of 8 lanes; lane gl -> 4 dims
+  const int tid = threadIdx.x, grp = tid >> 3, gl = tid & 7;
   const Partial* p = a.partials + static_cast<int64_t>(bh) * S;
+  const int dim4 = quarter * 8 + gl;   // float4 index within o[128]
 
-  float M = -INFINITY;
-  for (int s = tid; s < S; s += kCombineThreads) M = fmaxf(M, p[s].m);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if (lane == 0) red[warp] = M;
-  __syncthreads();
-  M = red[0];
-#pragma unroll
-  for (int w = 1; w < kCombineThreads / 32; ++w) M = fmaxf(M, red[w]);
-  __syncthreads();
-
-  float L = 0.0f;
-  for (int s = tid; s < S; s += kCombineThreads) {
-    const float w = (M == -INFINITY) ? 0.0f : exp2f(p[s].m - M);
-    wts[s] = w;
-    L = fmaf(w, p[s].l, L);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  if (lane == 0) red[warp] = L;
-  __syncthreads();
-  L = 0.0f;
-#pragma unroll
-  for (int w = 0; w < kCombineThreads / 32; ++w) L += red[w];
-
-  constexpr int kGroupsPerBlock = kCombineThreads / 8;
-  const int dim4 = quarter * 8 + gl;                  // float4 index within o[128]
+  float M = -INFINITY, L = 0.0f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = grp; s0 < S; s0 += kGroupsPerBlock * 8) {
-    float4 o[8];
-    float w[8];
+  for (int s0 = grp; s0 < S; s0 += kCombineGroups * kCombinePer) {
+    float m[kCombinePer], l[kCombinePer];
+    float4 o[kCombinePer];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int s = s0 + k * kGroupsPerBlock;
-      w[k] = s < S ? wts[s] : 0.0f;
-      o[k] = s < S ? reinterpret_cast<const float4*>(p[s].o)[dim4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < kCombinePer; ++k) {
+      const int s = s0 + k * kCombineGroups;
+      if (s < S) {
+        const float2 ml = *reinterpret_cast<const float2*>(&p[s].m);
+        m[k] = ml.x;
+        l[k] = ml.y;
+        o[k] = reinterpret_cast<const float4*>(p[s].o)[dim4];
+      } else {
+        m[k] = -INFINITY;
+        l[k] = 0.0f;
+        o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
+    float mx = M;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      acc.x = fmaf(w[k], o[k].x, acc.x);
-      acc.y = fmaf(w[k], o[k].y, acc.y);
-      acc.z = fmaf(w[k], o[k].z, acc.z);
-      acc.w = fmaf(w[k], o[k].w, acc.w);
+    for (int k = 0; k < kCombinePer; ++k) mx = fmaxf(mx, m[k]);
+    if (mx == -INFINITY) continue;   // only empty splits so far
+    const float sc = exp2f(M - mx);
+    acc.x *= sc;
+    acc.y *= sc;
+    acc.z *= sc;
+    acc.w *= sc;
+    L *= sc;
+#pragma unroll
+    for (int k = 0; k < kCombinePer; ++k) {
+      const float w = exp2f(m[k] - mx);
+      acc.x = fmaf(w, o[k].x, acc.x);
+      acc.y = fmaf(w, o[k].y, acc.y);
+      acc.z = fmaf(w, o[k].z, acc.z);
+      acc.w = fmaf(w, o[k].w, acc.w);
+      L = fmaf(w, l[k], L);
     }
+    M = mx;
   }
   acc_s[grp][gl] = acc;
+  if (gl == 0) {
+    ml_s[grp][0] = M;
+    ml_s[grp][1] = L;
+  }
   __syncthreads();
   if (tid < 8) {
-    float4 t = acc_s[0][tid];
-    for (int g2 = 1; g2 < kGroupsPerBlock; ++g2) {
-      const float4 u = acc_s[g2][tid];
-      t.x += u.x;
-      t.y += u.y;
-      t.z += u.z;
-      t.w += u.w;
+    float Mg = -INFINITY;
+#pragma unroll
+    for (int g2 = 0; g2 < kCombineGroups; ++g2) Mg = fmaxf(Mg, ml_s[g2][0]);
+    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+    float Lt = 0.0f;
+    if (Mg != -INFINITY) {
+      for (int g2 = 0; g2 < kCombineGroups; ++g2) {
+        const float w = exp2f(ml_s[g2][0] - Mg);
+        const float4 u = acc_s[g2][tid];
+        t.x = fmaf(w, u.x, t.x);
+        t.y = fmaf(w, u.y, t.y);
+        t.z = fmaf(w, u.z, t.z);
+        t.w = fmaf(w, u.w, t.w);
+        Lt = fmaf(w, ml_s[g2][1], Lt);
+      }
     }
-    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    const float inv = Lt > 0.0f ? 1.0f / Lt : 0.0f;
     reinterpret_cast<float4*>(a.out + static_cast<int64_t>(bh) * kD)[quarter * 8 + tid] =
         make_float4(t.x * inv, t.y * inv, t.z * inv, t.w * inv);
     if (a.lse && quarter == 0 && tid == 0)
-      a.lse[bh] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+      a.lse[bh] = Lt > 0.0f ? (Mg + log2f(Lt)) * 0.6931471805599453f : -INFINITY;
   }
 }
 
@@ -145,7 +154,7 @@ int choose_splits(int algo, int B, int q_heads, int64_t max_T, const commvq_atte
 }
 
 struct WorkspaceLayout {
-  size_t partials_off, kimg_off, vimg_off, phase_off, qfrag_off, base_off, scores_off, total;
+  size_t partials_off, kimg_off, vimg_off, phase_off, scores_off, total;
 };
 constexpr size_t kPhaseBytes = 64 * sizeof(double) + 128 * 64 * 8 + 64 * 8;   // theta, rows, advance
 
@@ -158,9 +167,7 @@ WorkspaceLayout workspace_layout(const commvq_config* cfg, int algo, int B, int6
     L.kimg_off = round_up(end, 256);
     L.vimg_off = round_up(L.kimg_off + img, 256);
     L.phase_off = round_up(L.vimg_off + img, 256);
-    L.qfrag_off = round_up(L.phase_off + kPhaseBytes, 256);
-    L.base_off = round_up(L.qfrag_off + static_cast<size_t>(B) * cfg->kv_heads * 256 * 8, 256);
-    L.scores_off = round_up(L.base_off + static_cast<size_t>(B) * S * 64 * 8, 256);
+    L.scores_off = round_up(L.phase_off + kPhaseBytes, 256);
     end = L.scores_off + static_cast<size_t>(B) * ((max_T + 15) / 16 * 16) * cfg->q_heads * sizeof(float);
   }
   L.total = round_up(end, 256);
@@ -257,10 +264,8 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
     a.v_img = reinterpret_cast<const uint4*>(ws + L.vimg_off);
     a.scores = reinterpret_cast<float*>(ws + L.scores_off);
     a.theta = reinterpret_cast<const double*>(ws + L.phase_off);
-    a.rowph = reinterpret_cast<const float2*>(ws + L.phase_off + 64 * sizeof(double));
-    a.advph = a.rowph + 128 * 64;
-    a.qfrag = reinterpret_cast<const uint2*>(ws + L.qfrag_off);
-    a.basetab = reinterpret_cast<const float2*>(ws + L.base_off);
+    a.rowph = reinterpret_cast<const float4*>(ws + L.phase_off + 64 * sizeof(double));
+    a.advph = a.rowph + 128 * 32;
   }
   a.main_start = options ? options->main_start : nullptr;
   a.main_stop = options ? options->main_stop : nullptr;
@@ -273,9 +278,17 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
   a.n_codes = cfg->n_codes;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool prepared = options && (options->flags & COMMVQ_ATTEND_PREPARED);
   commvq_status rc;
   if (run == COMMVQ_ATTN_DECODE_MMA) {
-    rc = launch_attend_mma(a, q, q_dtype, S, st);   // its prep kernel clears the error word
+    if (!prepared) {
+      rc = launch_attend_prep(a, st);   // also clears the error word
+      if (rc != COMMVQ_OK) return rc;
+    } else if (cfg->n_codes < 256 &&   // codes can be out of range: this call's word starts clear
+               cudaMemsetAsync(a.error_word, 0, sizeof(int), st) != cudaSuccess) {
+      return COMMVQ_ERR_CUDA;
+    }
+    rc = launch_attend_mma(a, q, q_dtype, S, st);
   } else {
     if (cudaMemsetAsync(a.error_word, 0, sizeof(int), st) != cudaSuccess) return COMMVQ_ERR_CUDA;
     // External records so the events keep their timestamps inside a captured CUDA graph too.
@@ -290,6 +303,54 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
   }
   if (rc != COMMVQ_OK) return rc;
   return launch_combine(a, S, st);
+}
+
+extern "C" commvq_status commvq_attend_prepare(const commvq_config* cfg, int32_t B, int64_t max_T,
+                                               const float* k_codebook, const float* v_codebook,
+                                               void* workspace, size_t workspace_bytes,
+                                               const commvq_attend_options* options, void* stream) {
+  const commvq_status cs = check_config(cfg);
+  if (cs != COMMVQ_OK) return cs;
+  if (B < 0 || max_T < 0) return COMMVQ_ERR_INVALID_ARG;
+  const int algo = options ? options->algo : COMMVQ_ATTN_AUTO;
+  if (options && (options->splits < 0 || options->splits > kMaxSplits)) return COMMVQ_ERR_INVALID_ARG;
+  if (algo != COMMVQ_ATTN_AUTO && algo != COMMVQ_ATTN_TABLE && algo != COMMVQ_ATTN_DECODE_MMA)
+    return COMMVQ_ERR_INVALID_ARG;
+  if (B == 0) return COMMVQ_OK;
+  if (B > 65535) return COMMVQ_ERR_UNSUPPORTED;
+  if (!k_codebook || !v_codebook || !workspace) return COMMVQ_ERR_INVALID_ARG;
+  if (!aligned(k_codebook, 16) || !aligned(v_codebook, 16) || !aligned(workspace, 256))
+    return COMMVQ_ERR_INVALID_ARG;
+  if (algo == COMMVQ_ATTN_DECODE_MMA && !mma_supported(cfg->R, cfg->q_heads, cfg->kv_heads, cfg->n_codes))
+    return COMMVQ_ERR_UNSUPPORTED;
+  const size_t need = commvq_attend_workspace_bytes(cfg, B, max_T, options);
+  if (need == 0 || workspace_bytes < need) return COMMVQ_ERR_WORKSPACE;
+  const DeviceInfo di = current_device_info();
+  if (di.device < 0) return COMMVQ_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int run = resolve_algo(cfg, options);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  if (run != COMMVQ_ATTN_DECODE_MMA)
+    return cudaMemsetAsync(workspace, 0, sizeof(int), st) == cudaSuccess ? COMMVQ_OK : COMMVQ_ERR_CUDA;
+  const int S = choose_splits(run, B, cfg->q_heads, max_T, options);
+  const WorkspaceLayout L = workspace_layout(cfg, run, B, max_T, S);
+  AttendArgs a{};
+  a.k_codebook = k_codebook;
+  a.v_codebook = v_codebook;
+  a.error_word = static_cast<int*>(workspace);
+  a.k_img = reinterpret_cast<const uint4*>(ws + L.kimg_off);
+  a.v_img = reinterpret_cast<const uint4*>(ws + L.vimg_off);
+  a.theta = reinterpret_cast<const double*>(ws + L.phase_off);
+  a.rowph = reinterpret_cast<const float4*>(ws + L.phase_off + 64 * sizeof(double));
+  a.advph = a.rowph + 128 * 32;
+  a.max_T = max_T;
+  a.rope_base = cfg->rope_base;
+  a.B = B;
+  a.q_heads = cfg->q_heads;
+  a.kv_heads = cfg->kv_heads;
+  a.R = cfg->R;
+  a.n_codes = cfg->n_codes;
+  return launch_attend_prep(a, st);
 }
 
 namespace commvq {
@@ -323,4 +384,4 @@ extern "C" const char* commvq_status_string(commvq_status s) {
   }
 }
 
-extern "C" int32_t commvq_abi_version(void) { return 1; }
+extern "C" int32_t commvq_abi_version(void) { return 2; }

@@ -28,11 +28,11 @@ struct AttendArgs {
   float* scores;          // decode-and-rotate form: tile-blocked exp2-domain scores
   const uint4* k_img;     // decode-and-rotate form: fp16 codebook images (see attend_mma.cu)
   const uint4* v_img;
-  const double* theta;    // decode-and-rotate form: RoPE tables written by its prep kernel
-  const float2* rowph;
-  const float2* advph;
-  const uint2* qfrag;     // decode-and-rotate form: per-call query fragments and split phasors
-  const float2* basetab;
+  // decode-and-rotate form: RoPE tables written by its prep kernel. Phasor rows hold, per
+  // pair of RoPE pairs (p, p+1) with p even, one float4 (cos p, cos p+1, sin p, sin p+1).
+  const double* theta;
+  const float4* rowph;    // [128 offsets][32]
+  const float4* advph;    // [32]
   void* main_start;       // optional cudaEvent_t pair around the main kernel(s)
   void* main_stop;
   int64_t max_T;
@@ -48,6 +48,7 @@ size_t table_smem_bytes(int R, int n_codes);
 size_t mma_scores_smem_bytes(int R, int KV, int n_codes);
 size_t mma_values_smem_bytes(int R, int KV, int q_heads, int n_codes);
 bool mma_supported(int R, int q_heads, int kv_heads, int n_codes);
+commvq_status launch_attend_prep(const AttendArgs& a, cudaStream_t st);
 commvq_status launch_attend_mma(const AttendArgs& a, const void* q, commvq_dtype qt, int splits,
                                 cudaStream_t st);
 commvq_status launch_attend_table(const AttendArgs& a, const void* q, commvq_dtype qt, int splits,

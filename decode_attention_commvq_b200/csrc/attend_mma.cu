@@ -41,10 +41,6 @@ constexpr int kTiles = 8;                  // mma row blocks per pipeline stage
 constexpr int kTileT = 16;                 // positions per mma row block
 constexpr int kStageT = kTiles * kTileT;   // positions per pipeline stage
 
-// Barrier for a subset of the CTA's warps (ids 1..15; id 0 is __syncthreads).
-__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
-}
 constexpr int kRefresh = 16;               // phasor recurrence steps between exact refreshes
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -72,12 +68,33 @@ __device__ __forceinline__ uint32_t word(const uint4& v, int k) {
   return k == 0 ? v.x : (k == 1 ? v.y : (k == 2 ? v.z : v.w));
 }
 
-// Rotate the stored pair (a, b) (one half2) by the phasor (cos, sin) in fp32; fp16 result.
-__device__ __forceinline__ uint32_t rotate_pair(uint32_t ab, float2 ph) {
-  const float2 f = __half22float2(u32_as_h2(ab));
-  const float x = fmaf(f.x, ph.x, -f.y * ph.y);
-  const float y = fmaf(f.x, ph.y, f.y * ph.x);
-  return h2_as_u32(__floats2half2_rn(x, y));
+// f32(h) - x for an fp16 value h, in one instruction (sm_100 mixed-precision subtract); exact
+// when h is x rounded to fp16.
+__device__ __forceinline__ float sub_h_f(__half h, float x) {
+  float d;
+  asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(__half_as_ushort(h)), "f"(x));
+  return d;
+}
+
+// Rotate two stored pairs (a0, b0), (a1, b1) (half2 words w0, w1) by their phasors, packed as
+// c = (cos 0, cos 1), s = (sin 0, sin 1), in fp32: x = a cos - b sin, y = a sin + b cos.
+// Each rotated pair leaves as two fp16 pairs: hi = (x, y) rounded (h0, h1) and the negated
+// rounding error nlo = hi - (x, y) rounded (n0, n1), so hi - nlo carries x and y to about
+// 2^-22 relative and a product with an fp16 query loses nothing to the fp16 operand type.
+__device__ __forceinline__ void rotate_two(uint32_t w0, uint32_t w1, f32x2 c, f32x2 s, uint32_t& h0,
+                                           uint32_t& h1, uint32_t& n0, uint32_t& n1) {
+  const float2 f0 = __half22float2(u32_as_h2(w0));
+  const float2 f1 = __half22float2(u32_as_h2(w1));
+  float c0, c1, s0, s1;
+  unpack2(c, c0, c1);
+  unpack2(s, s0, s1);
+  const float x0 = fmaf(f0.x, c0, -f0.y * s0), y0 = fmaf(f0.x, s0, f0.y * c0);
+  const float x1 = fmaf(f1.x, c1, -f1.y * s1), y1 = fmaf(f1.x, s1, f1.y * c1);
+  const __half2 p0 = __floats2half2_rn(x0, y0), p1 = __floats2half2_rn(x1, y1);
+  h0 = h2_as_u32(p0);
+  h1 = h2_as_u32(p1);
+  n0 = h2_as_u32(__floats2half2_rn(sub_h_f(__low2half(p0), x0), sub_h_f(__high2half(p0), y0)));
+  n1 = h2_as_u32(__floats2half2_rn(sub_h_f(__low2half(p1), x1), sub_h_f(__high2half(p1), y1)));
 }
 
 template <typename QT>
@@ -148,56 +165,21 @@ __device__ __forceinline__ int clamp_code(int c, int Nc, int& err) {
 }
 
 // ---------------------------------------------------------------------------------------
-// Per-call preparation. blockIdx.y = 0 / 1: key / value codebook image, fp32 [R][16][Nc'][8]
-// -> fp16 slots (see the file comment). blockIdx.y = 2: RoPE tables, all from fp64:
-//   theta[p] = base^(-2p/d), row[delta][p] = e^{i delta theta_p} for the 128 rows of a stage,
-//   adv[p] = e^{i 128 theta_p} (one stage further).
+// Preparation (once per codebook pair; see commvq_attend_prepare). blockIdx.y = 0 / 1: key /
+// value codebook image, fp32 [R][16][Nc'][8] -> fp16 slots (see the file comment).
+// blockIdx.y = 2: RoPE tables, all from fp64: theta[p] = base^(-2p/d),
+// row[delta][p] = e^{i delta theta_p} for the 128 rows of a stage, adv[p] = e^{i 128 theta_p}
+// (one stage further).
 constexpr int kPhaseRows = kStageT;
 
-// blockIdx.y = 3: query fragments of every (sequence, KV head) in the scores kernel's mma
-// k-order (see attend_scores_kernel); blockIdx.y = 4: base phasor e^{i t_begin theta_p} of
-// every (sequence, split), from an fp64 angle.
-template <typename QT>
-__device__ __forceinline__ void prep_qfrag(const AttendArgs& a, const QT* q, int e) {
-  const int KV = a.kv_heads, G = a.q_heads / KV;
-  if (e >= a.B * KV * 256) return;
-  const int b = e / (KV * 256), r = e % (KV * 256);
-  const int kv = r >> 8, st = (r >> 5) & 7, ln = r & 31;
-  const int gg = ln >> 2, ii = ln & 3;
-  uint2 v = make_uint2(0u, 0u);
-  if (gg < G) {
-    const QT* qh = q + (static_cast<int64_t>(b) * a.q_heads + kv * G + gg) * kD;
-    const int d0 = 8 * (4 * (st >> 1) + ii) + 4 * (st & 1);
-    v.x = h2_as_u32(__floats2half2_rn(qval(qh, d0), qval(qh, d0 + 1)));
-    v.y = h2_as_u32(__floats2half2_rn(qval(qh, d0 + 2), qval(qh, d0 + 3)));
-  }
-  const_cast<uint2*>(a.qfrag)[e] = v;
-}
-
-__global__ void prep_kernel(AttendArgs a, int R, const void* __restrict__ q, int q_dtype, int S) {
+__global__ void prep_kernel(AttendArgs a, int R) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   const int Nc = a.n_codes;
-  if (e == 0 && blockIdx.y == 0) *a.error_word = 0;   // this call's device error word starts clear
-  if (blockIdx.y == 3) {
-    if (q_dtype == COMMVQ_F32) prep_qfrag(a, static_cast<const float*>(q), e);
-    else if (q_dtype == COMMVQ_F16) prep_qfrag(a, static_cast<const __half*>(q), e);
-    else prep_qfrag(a, static_cast<const __nv_bfloat16*>(q), e);
-    return;
-  }
-  if (blockIdx.y == 4) {
-    if (e >= a.B * S * (kD / 2)) return;
-    const int p = e % (kD / 2), bs = e / (kD / 2), s = bs % S, b = bs / S;
-    int64_t row0, t_begin, t_end;
-    split_range(a, b, s, S, row0, t_begin, t_end);
-    double sn, cs;
-    sincos(static_cast<double>(t_begin) * pow(a.rope_base, -2.0 * p / kD), &sn, &cs);
-    const_cast<float2*>(a.basetab)[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
-    return;
-  }
+  if (e == 0 && blockIdx.y == 0) *a.error_word = 0;   // the device error word starts clear
   const double rope_base = a.rope_base;
   double* theta = const_cast<double*>(a.theta);
-  float2* rowph = const_cast<float2*>(a.rowph);
-  float2* advph = const_cast<float2*>(a.advph);
+  float4* rowph = const_cast<float4*>(a.rowph);
+  float4* advph = const_cast<float4*>(a.advph);
   const float* kcb = a.k_codebook;
   const float* vcb = a.v_codebook;
   uint4* kimg = const_cast<uint4*>(a.k_img);
@@ -208,11 +190,11 @@ __global__ void prep_kernel(AttendArgs a, int R, const void* __restrict__ q, int
     const double th = pow(rope_base, -2.0 * p / kD);
     double sn, cs;
     sincos(static_cast<double>(delta) * th, &sn, &cs);
-    rowph[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+    put_phasor(rowph + delta * (kD / 4), p, cs, sn);
     if (delta == 0) {
       theta[p] = th;
       sincos(static_cast<double>(kStageT) * th, &sn, &cs);
-      advph[p] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+      put_phasor(advph, p, cs, sn);
     }
     return;
   }
@@ -239,9 +221,6 @@ __device__ __forceinline__ int slot(int v, int j, int c, int Nc) {
 __device__ __forceinline__ uint4 lds128(const unsigned char* smem, uint32_t off) {
   return *reinterpret_cast<const uint4*>(smem + off);
 }
-__device__ __forceinline__ uint2 lds64(const unsigned char* smem, uint32_t off) {
-  return *reinterpret_cast<const uint2*>(smem + off);
-}
 __device__ __forceinline__ uint32_t lds32(const unsigned char* smem, uint32_t off) {
   return *reinterpret_cast<const uint32_t*>(smem + off);
 }
@@ -250,35 +229,35 @@ __device__ __forceinline__ uint32_t byte_sel(int b) { return 0x4440u | static_ca
 __device__ __forceinline__ uint32_t take_byte(uint32_t w, uint32_t sel) { return __byte_perm(w, 0u, sel); }
 
 // ---------------------------------------------------------------------------------------
-// Scores. A 16-position tile is shared by a pair of warps (tile = warp / 2, half = warp % 2).
-// Thread (g = lane/4, i = lane%4) owns rows g and g+8 of the tile and, through the k-order of
-// the mma, 8 RoPE pairs: k-step 2u+h covers pairs 2h and 2h+1 of group 4u+i, and half h of
-// the pair takes u = 2h and 2h+1 (groups i, 4+i or 8+i, 12+i). One 16-byte gather fills two
-// k-steps of a row. Each half accumulates a partial S over its 64 dimensions; the halves add
-// them through a small double-buffered exchange in shared memory, ordered by a named barrier
-// per warp pair. The query fragments use the same k-order. Splitting the pairs halves the
-// phasor registers, which lets 16 warps share an SM.
+// Scores. Warp w takes the 8 positions 8w .. 8w+7 of each 128-position stage, over all 128
+// dimensions, for every KV head in turn; there is no exchange between warps. Thread
+// (g = lane/4, i = lane%4) owns position row g; the mma rows 8..15 are zero (the tensor pipe
+// has room to spare). Through the k-order of the mma the thread owns 16 RoPE pairs: k-step
+// 2u+h covers pairs 2h and 2h+1 of group 4u+i (u = 0..3), so one 16-byte gather of group 4u+i
+// fills k-steps 2u and 2u+1 of the row. The query fragments use the same k-order.
 // NC: the entry count when it is 256 (compile-time; every uint8 code is valid), else 0
 // (run-time count, codes checked against it).
 template <int R, int KV, int NC, typename QT>
 __global__ void __launch_bounds__(kMmaThreads, 1)
 attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
   constexpr bool kCheck = NC != 256;
+  constexpr int kRows = 8;                                           // positions per warp and stage
+  static_assert(kMmaWarps * kRows == kStageT, "stage split");
   extern __shared__ __align__(16) unsigned char smem[];
   const int Nc = NC ? NC : a.n_codes;
   const int G = a.q_heads / KV;
   uint4* cbk = reinterpret_cast<uint4*>(smem);                       // 32 * Nc slots
   uint2* qf = reinterpret_cast<uint2*>(cbk + 32 * Nc);               // [KV][8][32]
-  float2* base = reinterpret_cast<float2*>(qf + KV * 8 * 32);       // [64] e^{i t0 theta_p}
-  float* red = reinterpret_cast<float*>(base + 64);                  // [8 tiles][KV*8]
-  float4* xch = reinterpret_cast<float4*>(red + kTiles * KV * 8);    // [8 tiles][2][32]
-  uint8_t* stage_buf = reinterpret_cast<uint8_t*>(xch + kTiles * 2 * 32);   // [2][kStageT][KV][R][16]
+  float4* base = reinterpret_cast<float4*>(qf + KV * 8 * 32);       // [32] e^{i t0 theta_p}, packed
+  float4* advs = base + 32;                                          // [32] e^{i kStageT theta_p}, packed
+  float* red = reinterpret_cast<float*>(advs + 32);                  // [16 warps][KV*8]
+  float4* base_all = reinterpret_cast<float4*>(red + kMmaWarps * KV * 8);   // [16 warps][32] refreshes
+  uint8_t* stage_all = reinterpret_cast<uint8_t*>(base_all + kMmaWarps * 32);   // [16 warps][2][8 rows][KV R][16]
   using SL = StageLayout<R, KV>;
-  constexpr int kStageBytes = SL::kBytes;
+  constexpr int kWarpStage = kRows * SL::kPieces * 16;                // one warp's rows of one stage
 
   const int s = blockIdx.x, b = blockIdx.y, S = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int tile = warp >> 1, half = warp & 1;
   const int g = lane >> 2, i = lane & 3, par = g & 1;
   int64_t row0, t_begin, t_end;
   split_range(a, b, s, S, row0, t_begin, t_end);
@@ -289,162 +268,169 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
     return;
   }
 
-  // Set-up is all asynchronous copies of what the prep kernel made: codebook image, query
-  // fragments of this sequence, base phasors of this split; then the first code stage.
-  for (int p = tid; p < 32 * Nc; p += kMmaThreads) cp_async16(cbk + p, a.k_img + p);
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(a.qfrag + static_cast<int64_t>(b) * KV * 256);
-    for (int p = tid; p < KV * 256 / 2; p += kMmaThreads) cp_async16(reinterpret_cast<uint4*>(qf) + p, src + p);
-    const uint4* bsrc = reinterpret_cast<const uint4*>(a.basetab + (static_cast<int64_t>(b) * S + s) * (kD / 2));
-    if (tid < kD / 4) cp_async16(reinterpret_cast<uint4*>(base) + tid, bsrc + tid);
-  }
-  cp_async_commit();
-  issue_stage<R, KV>(stage_buf, a.k_codes, row0, t_begin, t_end);
-  cp_async_commit();
-  (void)q;
-
-  // Phasors of the thread's 8 pairs (k = 4 ul + m -> pair 4(4(2 half + ul) + i) + m) at its two
-  // rows, and the per-iteration advance e^{i kStageT theta}. A refresh rebuilds them exactly
-  // from the stage's base phasor (fp64 angle, in shared memory) times the prep row table.
-  auto pair_of = [&](int k) { return 4 * (4 * (2 * half + (k >> 2)) + i) + (k & 3); };
-  float2 ph[2][8], adv[8];
-  auto load_rows = [&]() {
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-#pragma unroll
-      for (int rho = 0; rho < 2; ++rho) ph[rho][k] = a.rowph[(tile * kTileT + g + 8 * rho) * (kD / 2) + pair_of(k)];
-  };
-  auto times_base = [&]() {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float2 bp = base[pair_of(k)];
-#pragma unroll
-      for (int rho = 0; rho < 2; ++rho) {
-        const float2 rp = ph[rho][k];
-        ph[rho][k] = make_float2(fmaf(bp.x, rp.x, -bp.y * rp.y), fmaf(bp.x, rp.y, bp.y * rp.x));
-      }
+  // Each warp streams its own rows: the 8 rows 8w..8w+7 of every 128-position stage, into a
+  // private double buffer (XOR-swizzled pieces, as StageLayout), with no CTA barrier in the loop.
+  uint8_t* wstage = stage_all + warp * 2 * kWarpStage;
+  auto issue_rows = [&](int buf, int64_t t0) {
+    const int64_t r0 = t0 + warp * kRows;
+    const int n = static_cast<int>(min(static_cast<int64_t>(kRows), t_end - r0));
+    const uint8_t* src = a.k_codes + (row0 + r0) * (SL::kPieces * 16);
+    for (int p = lane; p < n * SL::kPieces; p += 32) {
+      const int row = p / SL::kPieces, piece = p - row * SL::kPieces;
+      cp_async16(wstage + buf * kWarpStage + SL::offset(row, piece), src + p * 16);
     }
   };
-  load_rows();   // global loads in flight while the asynchronous copies land
-#pragma unroll
-  for (int k = 0; k < 8; ++k) adv[k] = a.advph[pair_of(k)];
+  // Set-up: asynchronous copies of the prepared codebook image and advance phasors, then the
+  // warp's first rows; meanwhile the query fragments and the split's base phasor are formed.
+  for (int p = tid; p < 32 * Nc; p += kMmaThreads) cp_async16(cbk + p, a.k_img + p);
+  if (tid < kD / 4) cp_async16(reinterpret_cast<uint4*>(advs) + tid, reinterpret_cast<const uint4*>(a.advph) + tid);
+  cp_async_commit();
+  if (t_begin + warp * kRows < t_end) issue_rows(0, t_begin);
+  cp_async_commit();
+  // Query fragments of this sequence in the mma k-order: entry (kv, k-step st, lane) holds, for
+  // head column lane/4, the dims of pairs 2(st&1) and 2(st&1)+1 of group 4(st>>1) + lane%4, fp16.
+  for (int e = tid; e < KV * 256; e += kMmaThreads) {
+    const int kv = e >> 8, st = (e >> 5) & 7, ln = e & 31, gg = ln >> 2, ii = ln & 3;
+    uint2 v = make_uint2(0u, 0u);
+    if (gg < G) {
+      const QT* qh = q + (static_cast<int64_t>(b) * a.q_heads + kv * G + gg) * kD;
+      const int d0 = 8 * (4 * (st >> 1) + ii) + 4 * (st & 1);
+      v.x = h2_as_u32(__floats2half2_rn(qval(qh, d0), qval(qh, d0 + 1)));
+      v.y = h2_as_u32(__floats2half2_rn(qval(qh, d0 + 2), qval(qh, d0 + 3)));
+    }
+    qf[e] = v;
+  }
+  if (tid >= kD / 2 && tid < kD) {   // base phasor e^{i t_begin theta_p}, fp64 angle
+    double sn, cs;
+    sincos(static_cast<double>(t_begin) * a.theta[tid - kD / 2], &sn, &cs);
+    put_phasor(base, tid - kD / 2, cs, sn);
+  }
 
-  for (int e = tid; e < kTiles * KV * 8; e += kMmaThreads) red[e] = -INFINITY;
+  // Phasors of the thread's 16 pairs at its row, packed two pairs per register pair: entry
+  // qq = 2u + h holds pairs 2h, 2h+1 of group 4u+i, i.e. packed table entry 2(4u+i) + h. A
+  // refresh rebuilds them exactly from the stage's base phasor (fp64 angle, in shared memory;
+  // the split's first, then the warp's own) times the prep row table; in between they advance
+  // by e^{i kStageT theta} per stage.
+  auto quad_of = [&](int qq) { return 2 * (4 * (qq >> 1) + i) + (qq & 1); };
+  f32x2 pc[8], ps[8];
+  const int srow = warp * kRows + g;                                 // row within the stage
+  auto load_rows = [&]() {
+#pragma unroll
+    for (int qq = 0; qq < 8; ++qq) load_phasor(a.rowph[srow * (kD / 4) + quad_of(qq)], pc[qq], ps[qq]);
+  };
+  load_rows();   // global loads in flight while the asynchronous copies land
+
+  for (int e = tid; e < kMmaWarps * KV * 8; e += kMmaThreads) red[e] = -INFINITY;
   const int64_t n_tiles = (a.max_T + kTileT - 1) / kTileT;
   const float scale = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
   int err = 0;
   int stage = 0, it = 0;
-  // Byte offsets of the thread's gathers: entry c of group 4u+i lives at g?[u - 2 half] + 128 c,
-  // gF in the v = par half of the image (first round / copy), gS in the other.
+  // Byte offsets of the thread's gathers: entry c of group 4u+i lives at gF[u] + 128 c in the
+  // v = par half of the image (first round / copy) and gS[u] + 128 c in the other half.
   const uint32_t sel_i = byte_sel(i);
-  uint32_t gF[2], gS[2];
+  uint32_t gF[4], gS[4];
 #pragma unroll
-  for (int ul = 0; ul < 2; ++ul) {
-    const int j = 4 * (2 * half + ul) + i;
-    gF[ul] = static_cast<uint32_t>(slot(par, j, 0, Nc)) * 16;
-    gS[ul] = static_cast<uint32_t>(slot(par ^ 1, j, 0, Nc)) * 16;
+  for (int u = 0; u < 4; ++u) {
+    gF[u] = static_cast<uint32_t>(slot(par, 4 * u + i, 0, Nc)) * 16;
+    gS[u] = static_cast<uint32_t>(slot(par ^ 1, 4 * u + i, 0, Nc)) * 16;
   }
+  // The row's record: piece kv R + r sits at 16 ((kv R + r) ^ swz), swz = the row's low bits.
+  const int swz = g & SL::kSwz;
+  const uint32_t cw_lane = static_cast<uint32_t>(g * SL::kPieces * 16);
+  // score buffer slot of this row: 16-position tile, values-kernel quad g/2, k = (g&1) + 2 (w&1)
+  const int sc_k = (g & 1) + 2 * (warp & 1);
+  float* red_w = red + warp * KV * 8;
 
-  for (int64_t t0 = t_begin; t0 < t_end; t0 += kStageT, stage ^= 1, ++it) {
-    if (t0 + kStageT < t_end)
-      issue_stage<R, KV>(stage_buf + (stage ^ 1) * kStageBytes, a.k_codes, row0, t0 + kStageT, t_end);
+  auto times_base = [&](const float4* bt) {
+#pragma unroll
+    for (int qq = 0; qq < 8; ++qq) {
+      f32x2 bc, bs;
+      load_phasor(bt[quad_of(qq)], bc, bs);
+      cmul2(pc[qq], ps[qq], bc, bs);
+    }
+  };
+  cp_async_wait<1>();   // the image (every thread's share) is in; the warp's rows may still land
+  __syncthreads();
+  times_base(base);
+  float4* base_w = base_all + warp * 32;
+
+  for (int64_t t0 = t_begin; t0 + warp * kRows < t_end; t0 += kStageT, stage ^= 1, ++it) {
+    if (t0 + kStageT + warp * kRows < t_end) issue_rows(stage ^ 1, t0 + kStageT);
     cp_async_commit();
-    if (it > 0 && it % kRefresh == 0 && tid < kD / 2) {   // later refresh: fp64 angle
-      double sn, cs;
-      sincos(static_cast<double>(t0) * a.theta[tid], &sn, &cs);
-      base[tid] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+    if (it > 0) {
+      if (it % kRefresh == 0) {   // the warp's own refresh: fp64 angles of all 64 pairs
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          double sn, cs;
+          sincos(static_cast<double>(t0) * a.theta[lane + 32 * h], &sn, &cs);
+          put_phasor(base_w, lane + 32 * h, cs, sn);
+        }
+        __syncwarp();
+        load_rows();
+        times_base(base_w);
+      } else {
+#pragma unroll
+        for (int qq = 0; qq < 8; ++qq) {
+          f32x2 dc, ds;
+          load_phasor(advs[quad_of(qq)], dc, ds);
+          cmul2(pc[qq], ps[qq], dc, ds);
+        }
+      }
     }
     cp_async_wait<1>();
-    __syncthreads();
-
-    const int64_t tt0 = t0 + tile * kTileT;        // this warp pair's tile
-    if (it % kRefresh == 0) {
-      if (it > 0) load_rows();
-      times_base();
-    } else {
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-#pragma unroll
-        for (int rho = 0; rho < 2; ++rho) {
-          const float2 p = ph[rho][k], d = adv[k];
-          ph[rho][k] = make_float2(fmaf(p.x, d.x, -p.y * d.y), fmaf(p.x, d.y, p.y * d.x));
-        }
-    }
-    if (tt0 < t_end) {   // uniform over the warp pair
-      const uint32_t sb = static_cast<uint32_t>(stage_buf - smem) + stage * kStageBytes;
-      const int rem = static_cast<int>(min(static_cast<int64_t>(kTileT), t_end - tt0));  // valid rows
-      const bool valid0 = g < rem, valid1 = g + 8 < rem;
+    __syncwarp();
+    const int64_t pos = t0 + warp * kRows + g;
+    {
+      const bool valid = pos < t_end;
+      const uint32_t cwb = static_cast<uint32_t>(wstage - smem) + stage * kWarpStage + cw_lane;
+      const int64_t tau = pos / kTileT;
 #pragma unroll 1
       for (int kv = 0; kv < KV; ++kv) {
-        // code words 2 half, 2 half + 1 (groups 8 half .. 8 half + 7) of each row; with two
-        // rounds, round `par` first (it pairs with the v = par half of the image)
-        uint2 cw[2][R];
+        // the row's code pieces of this KV head, round `par` first (it pairs with the v = par
+        // image half). With 256 entries every byte is a valid code, so rows past the end read
+        // stale codes whose scores are neither stored nor counted; with fewer entries they read 0.
+        uint4 cw[R];
 #pragma unroll
-        for (int rho = 0; rho < 2; ++rho) {
-          const bool valid = rho ? valid1 : valid0;
-          const int row = tile * kTileT + g + 8 * rho;
-#pragma unroll
-          for (int r = 0; r < R; ++r) {
-            const int piece = kv * R + (R == 2 ? (r ^ par) : r);
-            const uint32_t off = sb + SL::offset(row, piece) + 8 * half;
-            cw[rho][r] = valid ? lds64(smem, off) : make_uint2(0u, 0u);
-          }
+        for (int r = 0; r < R; ++r) {
+          const int rr = (R == 2) ? (r ^ par) : r;
+          const uint32_t off = cwb + static_cast<uint32_t>(((kv * R + rr) ^ swz) * 16);
+          cw[r] = (kCheck && !valid) ? make_uint4(0u, 0u, 0u, 0u) : lds128(smem, off);
         }
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};    // q . hi
+        float accn[4] = {0.f, 0.f, 0.f, 0.f};   // q . nlo
 #pragma unroll
-        for (int ul = 0; ul < 2; ++ul) {
-          const int u = 2 * half + ul;
-          uint32_t A[2][4];
-#pragma unroll
-          for (int rho = 0; rho < 2; ++rho) {
-            uint4 e;
-            int c0 = static_cast<int>(take_byte(ul ? cw[rho][0].y : cw[rho][0].x, sel_i));
-            if (kCheck) c0 = clamp_code(c0, Nc, err);
-            if (R == 2) {
-              int c1 = static_cast<int>(take_byte(ul ? cw[rho][R - 1].y : cw[rho][R - 1].x, sel_i));
-              if (kCheck) c1 = clamp_code(c1, Nc, err);
-              e = hadd2x4(lds128(smem, gF[ul] + (c0 << 7)), lds128(smem, gS[ul] + (c1 << 7)));
-            } else {
-              e = lds128(smem, gF[ul] + (c0 << 7));
-            }
-            A[0][rho] = rotate_pair(e.x, ph[rho][4 * ul + 0]);
-            A[0][2 + rho] = rotate_pair(e.y, ph[rho][4 * ul + 1]);
-            A[1][rho] = rotate_pair(e.z, ph[rho][4 * ul + 2]);
-            A[1][2 + rho] = rotate_pair(e.w, ph[rho][4 * ul + 3]);
+        for (int u = 0; u < 4; ++u) {
+          uint4 e;
+          int c0 = static_cast<int>(take_byte(word(cw[0], u), sel_i));
+          if (kCheck) c0 = clamp_code(c0, Nc, err);
+          if (R == 2) {
+            int c1 = static_cast<int>(take_byte(word(cw[R - 1], u), sel_i));
+            if (kCheck) c1 = clamp_code(c1, Nc, err);
+            e = hadd2x4(lds128(smem, gF[u] + (c0 << 7)), lds128(smem, gS[u] + (c1 << 7)));
+          } else {
+            e = lds128(smem, gF[u] + (c0 << 7));
           }
+          uint32_t h0, h2, n0, n2, h0b, h2b, n0b, n2b;
+          rotate_two(e.x, e.y, pc[2 * u], ps[2 * u], h0, h2, n0, n2);
+          rotate_two(e.z, e.w, pc[2 * u + 1], ps[2 * u + 1], h0b, h2b, n0b, n2b);
           const uint2 b0 = qf[(kv * 8 + 2 * u) * 32 + lane];
           const uint2 b1 = qf[(kv * 8 + 2 * u + 1) * 32 + lane];
-          mma16816(acc, A[0][0], A[0][1], A[0][2], A[0][3], b0.x, b0.y);
-          mma16816(acc, A[1][0], A[1][1], A[1][2], A[1][3], b1.x, b1.y);
+          mma16816(acc, h0, 0u, h2, 0u, b0.x, b0.y);
+          mma16816(accn, n0, 0u, n2, 0u, b0.x, b0.y);
+          mma16816(acc, h0b, 0u, h2b, 0u, b1.x, b1.y);
+          mma16816(accn, n0b, 0u, n2b, 0u, b1.x, b1.y);
         }
-        // Add the two halves' partial S. For even kv half 1 hands its partial to half 0, for
-        // odd kv the reverse, so the finishing work (stores, maxima) alternates between the
-        // two warps. The buffer alternates with kv, so the handing half can run one kv ahead.
-        const int finisher = kv & 1;
-        float4* xs = xch + (tile * 2 + (kv & 1)) * 32 + lane;
-        if (half != finisher) *xs = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        named_barrier_sync(1 + tile, 64);
-        if (half != finisher) continue;
-        {
-          const float4 o = *xs;
-          acc[0] += o.x;
-          acc[1] += o.y;
-          acc[2] += o.z;
-          acc[3] += o.w;
-        }
-        // acc: rows g (c0, c1) and g+8 (c2, c3); columns 2i, 2i+1 = query heads kv*G + col.
-        const int64_t tau = tt0 / kTileT;
+        acc[0] -= accn[0];
+        acc[1] -= accn[1];
+        // acc[0], acc[1]: row g, columns 2i, 2i+1 = query heads kv*G + col (rows 8..15 are zero)
         float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int col = 2 * i + c;
           if (col >= G) continue;
-          const float v0 = acc[c] * scale, v1 = acc[2 + c] * scale;
-          float* sp = a.scores + score_index(b, tau, kv, col, g >> 1, g & 1, n_tiles, KV, G);
-          if (valid0) sp[0] = v0;
-          if (valid1) sp[2] = v1;
-          const float mv = fmaxf(valid0 ? v0 : -INFINITY, valid1 ? v1 : -INFINITY);
-          if (c == 0) m0 = mv; else m1 = mv;
+          const float v = acc[c] * scale;
+          if (valid) a.scores[score_index(b, tau, kv, col, g >> 1, sc_k, n_tiles, KV, G)] = v;
+          if (c == 0) m0 = valid ? v : -INFINITY; else m1 = valid ? v : -INFINITY;
         }
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
@@ -452,23 +438,24 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
           m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
         }
         if (g == 0) {
-          float* rw = red + tile * KV * 8 + kv * 8 + 2 * i;
+          float* rw = red_w + kv * 8 + 2 * i;
           rw[0] = fmaxf(rw[0], m0);
           rw[1] = fmaxf(rw[1], m1);
         }
       }
     }
-    __syncthreads();
+    __syncwarp();   // the buffer just read is refilled by the next iteration's copies
   }
+  cp_async_wait<0>();
+  __syncthreads();
 
-  // split maxima: each tile's warp pair kept a row of maxima (entries of even kv heads written
-  // by half 0, odd by half 1); take the max over tiles
+  // split maxima: each warp kept a row of maxima; take the max over warps
   for (int e = tid; e < KV * 8; e += kMmaThreads) {
     const int kv = e >> 3, col = e & 7;
     if (col >= G) continue;
     float v = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kTiles; ++w) v = fmaxf(v, red[w * KV * 8 + e]);
+    for (int w = 0; w < kMmaWarps; ++w) v = fmaxf(v, red[w * KV * 8 + e]);
     part[static_cast<int64_t>(kv * G + col) * S].m = v;
   }
   if (kCheck) {
@@ -610,8 +597,10 @@ attend_values_kernel(AttendArgs a) {
         for (int k2 = 0; k2 < 2; ++k2) {
           const int k = 2 * pr + k2;
           const bool valid = tau[k] < rem;
-          // the code word of groups 2g, 2g+1; with two rounds, round vsel first
-          const uint32_t w0 = valid ? lds32(smem, sbt + cw_off[k][0]) : 0u;
+          // the code word of groups 2g, 2g+1; with two rounds, round vsel first. (With 256
+          // entries every byte is a valid code: positions past the end read stale codes and
+          // weigh them by p = 0; with fewer entries they read code 0.)
+          const uint32_t w0 = (kCheck && !valid) ? 0u : lds32(smem, sbt + cw_off[k][0]);
           int cA0 = static_cast<int>(take_byte(w0, selA)), cB0 = static_cast<int>(take_byte(w0, selB));
           if (kCheck) {
             cA0 = clamp_code(cA0, Nc, err);
@@ -620,7 +609,7 @@ attend_values_kernel(AttendArgs a) {
           uint4 SA = lds128(smem, gA[0] + (cA0 << 7));
           uint4 SB = lds128(smem, gB[0] + (cB0 << 7));
           if (R == 2) {
-            const uint32_t w1 = valid ? lds32(smem, sbt + cw_off[k][R - 1]) : 0u;
+            const uint32_t w1 = (kCheck && !valid) ? 0u : lds32(smem, sbt + cw_off[k][R - 1]);
             int cA1 = static_cast<int>(take_byte(w1, selA)), cB1 = static_cast<int>(take_byte(w1, selB));
             if (kCheck) {
               cA1 = clamp_code(cA1, Nc, err);
@@ -697,13 +686,6 @@ commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt,
   const size_t smem_s = mma_scores_smem_bytes(R, KV, a.n_codes);
   const size_t smem_v = mma_values_smem_bytes(R, KV, a.q_heads, a.n_codes);
   dim3 grid(S, a.B);
-  {
-    const int n = 2 * kGroups * a.n_codes;
-    int bx = max((n + kThreads - 1) / kThreads, (kPhaseRows * (kD / 2) + kThreads - 1) / kThreads);
-    bx = max(bx, (a.B * a.kv_heads * 256 + kThreads - 1) / kThreads);
-    bx = max(bx, (a.B * S * (kD / 2) + kThreads - 1) / kThreads);
-    prep_kernel<<<dim3(bx, 5), kThreads, 0, st>>>(a, R, q, static_cast<int>(qt), S);
-  }
   if (a.main_start &&
       cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a.main_start), st, cudaEventRecordExternal) != cudaSuccess)
     return COMMVQ_ERR_CUDA;
@@ -753,8 +735,8 @@ commvq_status launch_mma_kv(const AttendArgs& a, const void* q, commvq_dtype qt,
 }  // namespace
 
 size_t mma_scores_smem_bytes(int R, int KV, int n_codes) {
-  return static_cast<size_t>(512) * n_codes + static_cast<size_t>(KV) * 8 * 32 * 8 + 64 * sizeof(float2) +
-         static_cast<size_t>(kTiles) * KV * 8 * 4 + static_cast<size_t>(kTiles) * 2 * 32 * 16 +
+  return static_cast<size_t>(512) * n_codes + static_cast<size_t>(KV) * 8 * 32 * 8 + 2 * 32 * sizeof(float4) +
+         static_cast<size_t>(kMmaWarps) * KV * 8 * 4 + static_cast<size_t>(kMmaWarps) * 32 * sizeof(float4) +
          static_cast<size_t>(2) * kStageT * KV * R * kGroups;
 }
 
@@ -773,6 +755,14 @@ bool mma_supported(int R, int q_heads, int kv_heads, int n_codes) {
   if (kv_heads != 1 && kv_heads != 2 && kv_heads != 4 && kv_heads != 8) return false;
   if (q_heads % kv_heads || q_heads / kv_heads > 8) return false;
   return true;
+}
+
+commvq_status launch_attend_prep(const AttendArgs& a, cudaStream_t st) {
+  if (a.R != 1 && a.R != 2) return COMMVQ_ERR_UNSUPPORTED;
+  const int n = 2 * kGroups * a.n_codes;
+  const int bx = max((n + kThreads - 1) / kThreads, (kPhaseRows * (kD / 2) + kThreads - 1) / kThreads);
+  prep_kernel<<<dim3(bx, 3), kThreads, 0, st>>>(a, a.R);
+  return launch_status();
 }
 
 commvq_status launch_attend_mma(const AttendArgs& a, const void* q, commvq_dtype qt, int S, cudaStream_t st) {

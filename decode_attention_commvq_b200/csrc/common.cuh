@@ -120,4 +120,50 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
+// Two fp32 values in one 64-bit register pair, for the packed fp32x2 arithmetic of sm_100
+// (one instruction works on both lanes; each lane rounds as its scalar counterpart would).
+using f32x2 = unsigned long long;
+__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(f32x2 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// Complex product of packed phasors: (c, s) <- (c, s) * (cc, ss), two pairs at a time.
+__device__ __forceinline__ void cmul2(f32x2& c, f32x2& s, f32x2 cc, f32x2 ss) {
+  const f32x2 nc = sub2(mul2(c, cc), mul2(s, ss));
+  s = fma2(c, ss, mul2(s, cc));
+  c = nc;
+}
+// The phasors of RoPE pairs (p, p+1) from a packed row entry (cos p, cos p+1, sin p, sin p+1).
+__device__ __forceinline__ void load_phasor(float4 v, f32x2& c, f32x2& s) {
+  c = pack2(v.x, v.y);
+  s = pack2(v.z, v.w);
+}
+
+// Phasor e^{i phi} of RoPE pair p into a packed row: float4 p/2 holds (cos p, cos p+1, sin p,
+// sin p+1) for even p, the operand order of the packed rotation.
+__device__ __forceinline__ void put_phasor(float4* row, int p, double cs, double sn) {
+  float* f = reinterpret_cast<float*>(row + (p >> 1));
+  f[p & 1] = static_cast<float>(cs);
+  f[2 + (p & 1)] = static_cast<float>(sn);
+}
+
 }  // namespace commvq

@@ -77,12 +77,21 @@ typedef struct {
   int32_t code_bytes; /* 1 if n_codes <= 256 else 2 */
 } commvq_config;
 
+/* commvq_attend_options.flags */
+enum {
+  /* The workspace already holds this configuration's and these codebooks' prepared state,
+     written by commvq_attend_prepare (or by an earlier commvq_attend_decode without the
+     flag) with the same cfg, B, max_T, algo and splits; the call skips rewriting it. */
+  COMMVQ_ATTEND_PREPARED = 1
+};
+
 typedef struct {
   int32_t algo;        /* commvq_attn_algo */
   int32_t splits;      /* split-T partitions per sequence; 0 = chosen by the library */
   void* main_start;    /* nullable cudaEvent_t, recorded on `stream` right before the main
                           attention kernel (instrumentation; no effect on the result) */
   void* main_stop;     /* nullable cudaEvent_t, recorded right after it, before the merge */
+  int32_t flags;       /* COMMVQ_ATTEND_* bits; 0 = none */
 } commvq_attend_options;
 
 /* Residual nearest-codeword encoder (abstract: additive quantization; "What carries the
@@ -123,8 +132,11 @@ size_t commvq_attend_workspace_bytes(const commvq_config* cfg, int32_t B, int64_
  *   lse = -inf.
  * The rotation is applied per position to query x codebook products (key side) and the
  * softmax weights are accumulated per code before the value codebook multiply, as the
- * review describes. Precision: fp32 accumulation; the per-query table / decoded rows are
- * held in fp16 (relative error ~5e-4 per product).
+ * review describes. Precision: fp32 accumulation. Codebook entries are held in fp16 (relative
+ * error <= 2^-11 each). The table algorithm keeps its per-query table in fp16. The
+ * decode-and-rotate algorithm rotates keys in fp32 and feeds each rotated key to the tensor
+ * cores as two fp16 terms (value and rounding error), so only the entries' own rounding reaches
+ * the scores; softmax weights and value entries enter the second product in fp16.
  * q           [B, q_heads, d] in q_dtype (F32, F16 or BF16), 16-byte aligned.
  * k_codes, v_codes  [total_T, kv_heads, R, d/g] uint8 (attention supports Nc' <= 256),
  *             16-byte aligned; total_T = seq_offsets[B].
@@ -137,7 +149,9 @@ size_t commvq_attend_workspace_bytes(const commvq_config* cfg, int32_t B, int64_
  * workspace   device buffer of at least commvq_attend_workspace_bytes(...) bytes,
  *             256-byte aligned; its first 64 bytes hold the device error word, which this
  *             call clears. Calls that share a workspace must be ordered on one stream.
- * options     nullable (defaults: AUTO algorithm, library-chosen splits).
+ * options     nullable (defaults: AUTO algorithm, library-chosen splits, no flags). With
+ *             COMMVQ_ATTEND_PREPARED the workspace's prepared state (see commvq_attend_prepare)
+ *             is used as it stands; otherwise the call writes it first.
  * Supports d = 128, g = 8, Nc' <= 256 (code_bytes = 1), 1 <= R <= 4, q_heads % kv_heads == 0,
  * B >= 0 (B = 0 is a no-op). */
 commvq_status commvq_attend_decode(const commvq_config* cfg, const void* q, commvq_dtype q_dtype,
@@ -147,6 +161,19 @@ commvq_status commvq_attend_decode(const commvq_config* cfg, const void* q, comm
                                    float* out, float* lse, void* workspace,
                                    size_t workspace_bytes, const commvq_attend_options* options,
                                    void* stream);
+
+/* Write the state of commvq_attend_decode that depends only on cfg and the codebooks into
+ * the workspace: for the decode-and-rotate algorithm, the fp16 codebook images and the RoPE
+ * phasor tables; it also clears the device error word. Later commvq_attend_decode calls with
+ * the same cfg, B, max_T, algo, splits, codebooks and workspace pass COMMVQ_ATTEND_PREPARED in
+ * options->flags and skip this work (it is the same for every decode step of a layer). The
+ * prepared state stays valid until the workspace or the codebooks change. With the table
+ * algorithm there is no such state and the call only clears the error word.
+ * Arguments and errors as in commvq_attend_decode. */
+commvq_status commvq_attend_prepare(const commvq_config* cfg, int32_t B, int64_t max_T,
+                                    const float* k_codebook, const float* v_codebook,
+                                    void* workspace, size_t workspace_bytes,
+                                    const commvq_attend_options* options, void* stream);
 
 /* commvq_attend_decode for callers that cannot allocate device memory -- for example a
  * plugin inside a host framework that owns the device allocator, or a latency-critical loop
@@ -214,6 +241,62 @@ commvq_status commvq_em_step(const commvq_config* cfg, const float* rows, int64_
 commvq_status commvq_em_step_soft(const commvq_config* cfg, const float* rows, int64_t N,
                                   float* codebook_round, float tau, double* sse_out,
                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- Decompress-then-attend comparator ----------------------------------------------------
+ * The review compares CommVQ's decode latency with a "naive implementation of the same
+ * quantization" ("What carries the argument", Table 5: 6x-9.6x lower latency). These two calls
+ * are that implementation: commvq_decompress writes the whole cache out as dense 16-bit rows,
+ * keys already rotated, and commvq_dense_decode runs ordinary flash-decoding over them. Together
+ * they compute what commvq_attend_decode computes, with the cache decompressed in HBM.
+ */
+
+/* Bytes of device workspace commvq_decompress needs (its fp16 codebook images and phasor
+ * tables). 0 for invalid or unsupported input. */
+size_t commvq_decompress_workspace_bytes(const commvq_config* cfg, int64_t max_T);
+
+/* Decode every cached position and write it densely:
+ *   k_out[t, kvh, :] = RoPE_pos(sum_r kcb[r, j, kcode[t,kvh,r,j], :] per group j),
+ *   v_out[t, kvh, :] = sum_r vcb[r, j, vcode[t,kvh,r,j], :],
+ * where pos = t - seq_offsets[b] is the row's position in its sequence b (RoPE as in
+ * commvq_attend_decode: pair p = channels (2p, 2p+1), theta_p = rope_base^(-2p/d)).
+ * k_codes, v_codes  [total_T, kv_heads, R, d/g] uint8, total_T = seq_offsets[B].
+ * seq_offsets       [B+1] int64 device array as in commvq_attend_decode; rows past
+ *                   max_T positions of a sequence are not written.
+ * out_dtype         COMMVQ_BF16 or COMMVQ_F16.
+ * k_out, v_out      [total_T, kv_heads, d] of out_dtype, 16-byte aligned.
+ * workspace         >= commvq_decompress_workspace_bytes(cfg, max_T) bytes, 256-byte aligned;
+ *                   its first 4 bytes are the device error word (bit 0: a code >= Nc' was
+ *                   seen and clamped), cleared by this call.
+ * Precision: entries are held in fp16 and summed in fp16; keys are rotated in fp32 with
+ * phasors from fp64 angles; one final rounding to out_dtype.
+ * Supports d = 128, g = 8, R <= 2, Nc' <= 256. */
+commvq_status commvq_decompress(const commvq_config* cfg, const void* k_codes, const void* v_codes,
+                                const int64_t* seq_offsets, int32_t B, int64_t max_T,
+                                const float* k_codebook, const float* v_codebook,
+                                commvq_dtype out_dtype, void* k_out, void* v_out, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace commvq_dense_decode needs (per-split partials). 0 for invalid or
+ * unsupported input. options: only `splits` is read (0 = library choice, at most 512). */
+size_t commvq_dense_decode_workspace_bytes(const commvq_config* cfg, int32_t B, int64_t max_T,
+                                           const commvq_attend_options* options);
+
+/* Dense decode attention over rows that already carry their rotation:
+ *   s_t = q[b,h] . k[t, h / (q_heads / kv_heads)] / sqrt(d), out[b,h] = softmax(s) . v,
+ *   lse[b,h] = log sum_t exp(s_t) (natural log); an empty sequence gives 0 and -inf.
+ * q       [B, q_heads, d] in q_dtype (F32, F16 or BF16), converted to kv_dtype for the
+ *         tensor-core products.
+ * k, v    [total_T, kv_heads, d] in kv_dtype (F16 or BF16), 16-byte aligned.
+ * seq_offsets, B, max_T, out, lse: as in commvq_attend_decode.
+ * options nullable: splits (0 = library choice) and the main_start / main_stop events, recorded
+ *         around the attention kernel (before the split combine).
+ * Precision: fp32 accumulation; softmax weights are rounded to kv_dtype for the second product.
+ * Supports d = 128, kv_heads in {1, 2, 4, 8}, q_heads / kv_heads <= 16. */
+commvq_status commvq_dense_decode(const commvq_config* cfg, const void* q, commvq_dtype q_dtype,
+                                  const void* k, const void* v, commvq_dtype kv_dtype,
+                                  const int64_t* seq_offsets, int32_t B, int64_t max_T, float* out,
+                                  float* lse, void* workspace, size_t workspace_bytes,
+                                  const commvq_attend_options* options, void* stream);
 
 /* The device error word in an attention workspace: synchronises `stream`, copies the word
  * to the host and writes it to *device_error (0 = none; bit 0 = a code >= Nc' was seen

@@ -162,6 +162,23 @@ int oracle_scores_plain(const double* q, const double* keys, int64_t key_stride,
   return ORACLE_OK;
 }
 
+/* RoPE applied to whole rows: out[n] = R_{pos[n]} x[n], pair p rotated by angle pos[n]*theta_p
+ * in fp64 with R = [[cos, -sin], [sin, cos]] (the rotation of oracle_scores_plain, written out as
+ * rows: this is what a decompress-then-attend implementation stores as its key cache).
+ * x, out [n, d] fp64 (may alias); pos [n] int64, any sign (a negative position undoes one). */
+int oracle_rope(const double* x, const int64_t* pos, int64_t n, int d, double base, double* out) {
+  if (d <= 0 || (d % 2) || n < 0 || (n > 0 && (!x || !pos || !out))) return ORACLE_BAD_ARG;
+  for (int64_t r = 0; r < n; ++r)
+    for (int p = 0; p < d / 2; ++p) {
+      const double phi = rope_angle(pos[r], p, d, base);
+      const double c = cos(phi), sn = sin(phi);
+      const double a = x[r * d + 2 * p], b = x[r * d + 2 * p + 1];
+      out[r * d + 2 * p] = a * c - b * sn;
+      out[r * d + 2 * p + 1] = a * sn + b * c;
+    }
+  return ORACLE_OK;
+}
+
 /* Scores through the query x codebook table ("What carries the argument": the
  * query-dependent and codebook-dependent factors are formed once and reused for
  * every cached position; the rotation is applied afterwards by commutation).
@@ -251,6 +268,50 @@ int oracle_attend(const double* q, const double* khat, const double* vhat, const
         const double p = exp(s[t] - M) / Z;
         const double* v = vhat + ((t0 + t) * Hkv + kvh) * d;
         for (int i = 0; i < d; ++i) o[i] += p * v[i];
+      }
+      if (lse) lse[(int64_t)b * Hq + h] = M + log(Z);
+    }
+    free(s);
+  }
+  return ORACLE_OK;
+}
+
+/* Dense decode attention over keys that already carry their rotation (the second half of a
+ * decompress-then-attend implementation): s_t = q . k_t / sqrt(d), out = softmax(s) . v,
+ * lse = log sum e^{s_t}; shapes, GQA mapping, offsets and the empty case as oracle_attend. */
+int oracle_attend_dense(const double* q, const double* k, const double* v, const int64_t* offsets,
+                        int B, int Hq, int Hkv, int d, double* out, double* lse) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) || d <= 0 || !offsets || !out) return ORACLE_BAD_ARG;
+  const int group = Hq / Hkv;
+  const double inv_sqrt_d = 1.0 / sqrt((double)d);
+  for (int b = 0; b < B; ++b) {
+    const int64_t t0 = offsets[b], T = offsets[b + 1] - offsets[b];
+    if (T < 0) return ORACLE_BAD_ARG;
+    double* s = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    if (!s) return ORACLE_NO_MEM;
+    for (int h = 0; h < Hq; ++h) {
+      const int kvh = h / group;
+      const double* qh = q + ((int64_t)b * Hq + h) * d;
+      double* o = out + ((int64_t)b * Hq + h) * d;
+      for (int i = 0; i < d; ++i) o[i] = 0.0;
+      if (T == 0) {
+        if (lse) lse[(int64_t)b * Hq + h] = -INFINITY;
+        continue;
+      }
+      double M = -INFINITY;
+      for (int64_t t = 0; t < T; ++t) {
+        const double* kt = k + ((t0 + t) * Hkv + kvh) * d;
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i) acc += qh[i] * kt[i];
+        s[t] = acc * inv_sqrt_d;
+        M = s[t] > M ? s[t] : M;
+      }
+      double Z = 0.0;
+      for (int64_t t = 0; t < T; ++t) Z += exp(s[t] - M);
+      for (int64_t t = 0; t < T; ++t) {
+        const double p = exp(s[t] - M) / Z;
+        const double* vt = v + ((t0 + t) * Hkv + kvh) * d;
+        for (int i = 0; i < d; ++i) o[i] += p * vt[i];
       }
       if (lse) lse[(int64_t)b * Hq + h] = M + log(Z);
     }

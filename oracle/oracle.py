@@ -48,8 +48,11 @@ def lib():
         _lib.oracle_em_step.argtypes = [P, I64, I, I, I, P, P, P]
         _lib.oracle_values_hist.argtypes = [P, P, I64, I64, I, I, I, I, P, P, P]
         _lib.oracle_em_soft_step.argtypes = [P, I64, I, I, I, P, ctypes.c_double, P]
+        _lib.oracle_rope.argtypes = [P, P, I64, I, ctypes.c_double, P]
+        _lib.oracle_attend_dense.argtypes = [P, P, P, P, I, I, I, I, P, P]
         for f in ("oracle_encode", "oracle_decode", "oracle_scores_plain", "oracle_scores_table",
-                  "oracle_attend", "oracle_em_step", "oracle_values_hist", "oracle_em_soft_step"):
+                  "oracle_attend", "oracle_em_step", "oracle_values_hist", "oracle_em_soft_step",
+                  "oracle_rope", "oracle_attend_dense"):
             getattr(_lib, f).restype = ctypes.c_int
     return _lib
 
@@ -162,6 +165,37 @@ def attend(q: np.ndarray, khat: np.ndarray, vhat: np.ndarray, offsets: np.ndarra
     _check(lib().oracle_attend(_p(_c(q, np.float64)), _p(_c(khat, np.float64)),
                                _p(_c(vhat, np.float64)), _p(_c(offsets, np.int64)), B, Hq, Hkv, d,
                                float(base), _p(out), _p(lse)), "attend")
+    return out, lse
+
+
+def rope(x: np.ndarray, pos: np.ndarray, base: float) -> np.ndarray:
+    """Rows x [n, d] rotated to positions pos [n] (fp64): the key rows a decompress-then-attend
+    implementation stores."""
+    xd = _c(x, np.float64)
+    n, d = xd.shape
+    out = np.empty_like(xd)
+    _check(lib().oracle_rope(_p(xd), _p(_c(pos, np.int64)), n, d, float(base), _p(out)), "rope")
+    return out
+
+
+def rope_cache(khat: np.ndarray, offsets: np.ndarray, base: float) -> np.ndarray:
+    """A decoded key cache [sum T, Hkv, d] rotated row by row to its in-sequence positions."""
+    N, Hkv, d = khat.shape
+    pos = np.concatenate([np.arange(offsets[b + 1] - offsets[b]) for b in range(len(offsets) - 1)]
+                         + [np.zeros(0, np.int64)]).astype(np.int64)
+    return rope(khat.reshape(N * Hkv, d), np.repeat(pos, Hkv), base).reshape(N, Hkv, d)
+
+
+def attend_dense(q: np.ndarray, k: np.ndarray, v: np.ndarray, offsets: np.ndarray):
+    """Dense decode attention on keys that already carry their rotation. q [B, Hq, d];
+    k/v [sum T, Hkv, d]. Returns (out [B, Hq, d] fp64, lse [B, Hq] fp64)."""
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    out = np.empty((B, Hq, d), dtype=np.float64)
+    lse = np.empty((B, Hq), dtype=np.float64)
+    _check(lib().oracle_attend_dense(_p(_c(q, np.float64)), _p(_c(k, np.float64)), _p(_c(v, np.float64)),
+                                     _p(_c(offsets, np.int64)), B, Hq, Hkv, d, _p(out), _p(lse)),
+           "attend_dense")
     return out, lse
 
 

@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol(api):
 
 
 def test_status_strings_and_version(api):
-    assert api.abi_version() == 1
+    assert api.abi_version() == 2
     for s in range(6):
         assert api.status_string(s)
     assert "unknown" in api.status_string(99)
@@ -97,10 +97,7 @@ def test_workspace_sizes(api):
     part = 256 + 32 * 148 * 528
     img = 512 * 256
     phase = 64 * 8 + 128 * 64 * 8 + 64 * 8
-    qfrag = 1 * 8 * 256 * 8
-    base = 1 * 148 * 64 * 8
-    want = (-(-part // 256) * 256 + 2 * img + -(-phase // 256) * 256 + -(-qfrag // 256) * 256 +
-            -(-base // 256) * 256 + 32768 * 32 * 4)
+    want = -(-part // 256) * 256 + 2 * img + -(-phase // 256) * 256 + 32768 * 32 * 4
     assert mma == -(-want // 256) * 256
     assert api.attend_workspace_bytes(cfg, 1, 32768) == api.attend_workspace_bytes(
         cfg, 1, 32768, algo=api.ATTN_DECODE_MMA)
@@ -139,3 +136,73 @@ def test_soft_em_rejects_bad_temperature(api):
     f = api.LIB.commvq_em_step_soft
     for tau in (0.0, -1.0, float("nan"), float("inf")):
         assert f(ctypes.byref(cc), P(FAKE), 100, P(FAKE), tau, None, P(FAKE), 1 << 30, None) == 1
+
+
+def _decomp(api, cfg, B=1, max_T=100, kc=FAKE, vc=FAKE, offs=FAKE, kcb=FAKE, vcb=FAKE, odt=2,
+            ko=FAKE, vo=FAKE, ws=FAKE, ws_bytes=1 << 24):
+    cc = cfg.c()
+    P = ctypes.c_void_p
+    return api.LIB.commvq_decompress(ctypes.byref(cc), P(kc), P(vc), P(offs), B, max_T, P(kcb), P(vcb),
+                                     odt, P(ko), P(vo), P(ws), ws_bytes, None)
+
+
+def _dense(api, cfg, B=1, max_T=100, q=FAKE, k=FAKE, v=FAKE, kvdt=2, offs=FAKE, out=FAKE, ws=FAKE,
+           ws_bytes=1 << 24, opts=None):
+    cc = cfg.c()
+    P = ctypes.c_void_p
+    return api.LIB.commvq_dense_decode(ctypes.byref(cc), P(q), 2, P(k), P(v), kvdt, P(offs), B, max_T,
+                                       P(out), None, P(ws), ws_bytes, ctypes.byref(opts) if opts else None,
+                                       None)
+
+
+def test_decompress_and_dense_reject_bad_arguments(api):
+    INVALID, UNSUP, WS = 1, 2, 4
+    cfg = _cfg(api)
+    assert _decomp(api, cfg, B=0) == 0
+    assert _decomp(api, cfg, odt=0) == INVALID                       # fp32 output
+    assert _decomp(api, cfg, kc=0) == INVALID
+    assert _decomp(api, cfg, ko=FAKE + 8) == INVALID                 # misaligned output
+    assert _decomp(api, cfg, ws_bytes=1024) == WS
+    assert _decomp(api, _cfg(api, R=3)) == UNSUP
+    assert _decomp(api, _cfg(api, n_codes=512)) == UNSUP
+    assert _decomp(api, _cfg(api, q_heads=12, kv_heads=3)) == UNSUP   # KV heads not in {1,2,4,8}
+    assert _decomp(api, cfg, max_T=-1) == INVALID
+    assert _dense(api, cfg, B=0) == 0
+    assert _dense(api, cfg, kvdt=0) == INVALID                       # fp32 rows
+    assert _dense(api, cfg, q=0) == INVALID
+    assert _dense(api, cfg, k=FAKE + 4) == INVALID
+    assert _dense(api, cfg, ws_bytes=512) == WS
+    assert _dense(api, _cfg(api, q_heads=12, kv_heads=3)) == UNSUP   # KV heads not in {1,2,4,8}
+    assert _dense(api, _cfg(api, q_heads=32, kv_heads=1)) == UNSUP   # 32 heads per group
+    assert _dense(api, cfg, opts=api.CAttendOptions(0, 513)) == INVALID
+
+
+def test_decompress_and_dense_workspace_sizes(api):
+    cfg = _cfg(api)
+    img = 2 * 16 * 256 * 16
+    want = 256 + 2 * img + 128 * 32 * 16 + 256 * 32 * 16            # header, images, tables
+    assert api.decompress_workspace_bytes(cfg, 32768) == want
+    assert api.decompress_workspace_bytes(_cfg(api, R=3), 10) == 0
+    assert api.dense_decode_workspace_bytes(cfg, 1, 32768, splits=8) == 256 + 32 * 8 * 528
+    # 2 KV heads: 4 warps per head write their own partials
+    c2 = _cfg(api, q_heads=8, kv_heads=2)
+    assert api.dense_decode_workspace_bytes(c2, 2, 1000, splits=3) == 256 + 2 * 8 * 3 * 4 * 528
+    assert api.dense_decode_workspace_bytes(_cfg(api, q_heads=12, kv_heads=3), 1, 10) == 0
+
+
+def test_prepare_rejects_bad_arguments(api):
+    INVALID, UNSUP, WS = 1, 2, 4
+    P = ctypes.c_void_p
+    f = api.LIB.commvq_attend_prepare
+    cc = _cfg(api).c()
+    assert f(ctypes.byref(cc), 0, 100, P(FAKE), P(FAKE), P(FAKE), 1 << 24, None, None) == 0   # B = 0
+    assert f(ctypes.byref(cc), 1, 100, None, P(FAKE), P(FAKE), 1 << 24, None, None) == INVALID
+    assert f(ctypes.byref(cc), 1, 100, P(FAKE + 4), P(FAKE), P(FAKE), 1 << 24, None, None) == INVALID
+    assert f(ctypes.byref(cc), 1, 100, P(FAKE), P(FAKE), P(FAKE + 16), 1 << 24, None, None) == INVALID
+    assert f(ctypes.byref(cc), 1, 100, P(FAKE), P(FAKE), P(FAKE), 64, None, None) == WS
+    assert f(ctypes.byref(cc), -1, 100, P(FAKE), P(FAKE), P(FAKE), 1 << 24, None, None) == INVALID
+    c5 = _cfg(api, R=5).c()
+    assert f(ctypes.byref(c5), 1, 100, P(FAKE), P(FAKE), P(FAKE), 1 << 24, None, None) == UNSUP
+    o = api.CAttendOptions(api.ATTN_DECODE_MMA, 0, None, None, 0)
+    c3 = _cfg(api, R=3, n_codes=64).c()
+    assert f(ctypes.byref(c3), 1, 100, P(FAKE), P(FAKE), P(FAKE), 1 << 24, ctypes.byref(o), None) == UNSUP

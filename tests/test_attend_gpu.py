@@ -260,3 +260,51 @@ def test_shapes_and_query_types(api, gpu, algo, shape):
     ref, ref_lse = O.attend_codes(q_as_f64(w, q), kc, vc, offs, kcb, vcb, w.rope_base)
     assert rel_err(out, ref) <= tol_for(w)
     assert np.allclose(lse, ref_lse, rtol=1e-3, atol=5e-3)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_prepared_workspace_is_identical(api, gpu, algo):
+    """commvq_attend_prepare once, then decode steps with COMMVQ_ATTEND_PREPARED: the same
+    results as unprepared calls, for two different queries on one prepared workspace (the
+    same bits on the decode-and-rotate path; the table path adds histogram weights with
+    shared-memory atomics, whose order varies, so there within 1e-6)."""
+    w, kc, vc, kcb, vcb = _encoded_inputs(synth.WORKLOADS[1], T=3000)
+    cfg = _cfg(api, w)
+    offs = w.offsets()
+    max_T = int(np.diff(offs).max())
+    offsets = torch.from_numpy(offs.astype(np.int64)).to(gpu)
+    kcg, vcg = _codes_np_to_gpu(kc, gpu), _codes_np_to_gpu(vc, gpu)
+    kcbt, vcbt = torch.from_numpy(kcb).to(gpu), torch.from_numpy(vcb).to(gpu)
+    ws = api.attend_workspace(cfg, 1, max_T, gpu, algo)
+    api.attend_prepare(cfg, 1, max_T, kcbt, vcbt, ws, algo=algo)
+    q0 = synth.queries(w)
+    q1 = synth.queries(w.with_(seed=w.seed + 7))
+    for q_np in (q0, q1):
+        q = to_torch_q(q_np, w.q_dtype, gpu)
+        out_p, lse_p = api.attend_decode(cfg, q, kcg, vcg, offsets, max_T, kcbt, vcbt, workspace=ws,
+                                         algo=algo, prepared=True)
+        out_u, lse_u = api.attend_decode(cfg, q, kcg, vcg, offsets, max_T, kcbt, vcbt, algo=algo)
+        torch.cuda.synchronize()
+        if algo == 2:
+            assert torch.equal(out_p, out_u) and torch.equal(lse_p, lse_u)
+        else:
+            assert rel_err(out_p.cpu().numpy(), out_u.cpu().numpy()) <= 1e-6
+            assert torch.allclose(lse_p, lse_u, rtol=1e-6, atol=1e-6)
+        ref, _ = O.attend_codes(q_as_f64(w, q_np), kc, vc, offs, kcb, vcb, w.rope_base)
+        assert rel_err(out_p.cpu().numpy(), ref) <= tol_for(w)
+    assert api.workspace_error(ws) == 0
+
+
+def test_many_queries_within_bound(api, gpu):
+    """The bf16 bound on 6 seeded queries x 32 heads (192 heads) over 3000 encoded positions of
+    the 2-bit layer, decode-and-rotate path: the tail of the error distribution, not one
+    query's."""
+    w, kc, vc, kcb, vcb = _encoded_inputs(synth.WORKLOADS[1], T=3000)
+    offs = w.offsets()
+    worst = 0.0
+    for seed in range(11, 17):
+        q = synth.queries(w.with_(seed=seed))
+        out, _ = _run(api, w, q, kc, vc, offs, kcb, vcb, gpu, algo=2)
+        ref, _ = O.attend_codes(q_as_f64(w, q), kc, vc, offs, kcb, vcb, w.rope_base)
+        worst = max(worst, rel_err(out, ref))
+    assert worst <= tol_for(w), worst

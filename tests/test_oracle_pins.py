@@ -495,3 +495,57 @@ def test_soft_em_brute_force():
         want[j] = num / den[:, None]
     assert np.allclose(soft, want.astype(np.float32), rtol=1e-6, atol=1e-7)
     assert sse == pytest.approx(want_sse, rel=1e-12)
+
+
+# ----------------------------------------------------------------------------------------
+# decompress-then-attend comparator: RoPE on whole rows, dense attention on rotated rows
+
+def test_rope_rows_equal_complex_rotation():
+    """Row rotation against numpy's complex exponential (an independent routine), at
+    positions up to 131071, plus its inverse and the group law in the position."""
+    rng = np.random.default_rng(61)
+    d, base = 128, 500000.0
+    k = rng.standard_normal((40, d))
+    pos = rng.integers(0, 131072, size=40)
+    got = O.rope(k, pos, base)
+    z = k[:, 0::2] + 1j * k[:, 1::2]
+    z = z * np.exp(1j * pos[:, None] * base ** (-np.arange(0, d, 2) / d)[None, :])
+    want = np.empty_like(k)
+    want[:, 0::2], want[:, 1::2] = z.real, z.imag
+    assert np.abs(got - want).max() <= 1e-9 * np.abs(want).max()
+    assert np.abs(O.rope(got, -pos, base) - k).max() <= 1e-9
+    a = rng.integers(0, 5000, size=40)
+    assert np.abs(O.rope(O.rope(k, a, base), pos, base) - O.rope(k, a + pos, base)).max() <= 1e-9
+
+
+def test_rope_cache_positions_restart_per_sequence():
+    rng = np.random.default_rng(62)
+    kh = rng.standard_normal((7, 2, 16))
+    offs = np.array([0, 3, 3, 7])
+    got = O.rope_cache(kh, offs, 1e4)
+    assert np.array_equal(got[0], kh[0]) and np.array_equal(got[3], kh[3])   # position 0
+    want = _rope_complex(kh[3:7, 1], 1e4)
+    assert np.abs(got[3:7, 1] - want).max() <= 1e-12
+
+
+def test_attend_dense_equals_rotating_attend_and_sdpa():
+    """Dense attention on pre-rotated rows equals the rotating oracle on the unrotated rows,
+    and torch's scaled_dot_product_attention."""
+    rng = np.random.default_rng(63)
+    Hq, Hkv, d, base = 8, 2, 128, 500000.0
+    offs = np.array([0, 45, 45, 200])
+    N = offs[-1]
+    q = rng.standard_normal((3, Hq, d))
+    kh = rng.standard_normal((N, Hkv, d)) * 2
+    vh = rng.standard_normal((N, Hkv, d))
+    out, lse = O.attend_dense(q, O.rope_cache(kh, offs, base), vh, offs)
+    ref, ref_lse = O.attend(q, kh, vh, offs, base)
+    assert np.abs(out - ref).max() <= 1e-12 * np.abs(ref).max()
+    assert np.allclose(lse[[0, 2]], ref_lse[[0, 2]], rtol=0, atol=1e-12)
+    assert np.all(out[1] == 0) and np.all(lse[1] == -np.inf)
+    kr = O.rope_cache(kh, offs, base)[45:200].transpose(1, 0, 2)              # [Hkv, T, d]
+    K = torch.from_numpy(np.repeat(kr, Hq // Hkv, axis=0))[None]
+    V = torch.from_numpy(np.repeat(vh[45:200].transpose(1, 0, 2), Hq // Hkv, axis=0))[None]
+    Q = torch.from_numpy(q[2])[None, :, None, :]
+    sd = torch.nn.functional.scaled_dot_product_attention(Q, K, V)[0, :, 0].numpy()
+    assert np.abs(out[2] - sd).max() <= 1e-12 * np.abs(sd).max()

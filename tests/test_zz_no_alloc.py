@@ -74,3 +74,23 @@ def test_noalloc_rejects_requests_beyond_its_scratch(api, gpu):
         api.attend_decode_noalloc(cfg, q, codes, codes, offs, 1 << 20, cb, cb, out)
     assert e.value.status == 4
     assert torch.count_nonzero(out).item() == 0
+
+
+@pytest.mark.parametrize("algo", [1, 2])
+def test_noalloc_reuses_its_prepared_state(api, gpu, algo):
+    """A call without the flag prepares the internal scratch; the next call on the same layer
+    passes COMMVQ_ATTEND_PREPARED and gives the same result."""
+    w = synth.WORKLOADS[1]
+    cfg, q, kc, vc, offs, max_T, kcb, vcb = _inputs(api, w, gpu)
+    outs = []
+    for prepared in (False, True):
+        out = torch.full((w.batch, w.q_heads, w.d), float("nan"), dtype=torch.float32, device=gpu)
+        lse = torch.full((w.batch, w.q_heads), float("nan"), dtype=torch.float32, device=gpu)
+        api.attend_decode_noalloc(cfg, q, kc, vc, offs, max_T, kcb, vcb, out, lse, algo=algo,
+                                  prepared=prepared)
+        torch.cuda.synchronize()
+        outs.append((out, lse))
+    if algo == 2:   # no atomics on this path: the same bits
+        assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    else:           # histogram weights added with shared-memory atomics
+        assert rel_err(outs[1][0].cpu().numpy(), outs[0][0].cpu().numpy()) <= 1e-6
