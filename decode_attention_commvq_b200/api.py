@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libcommvq_b200.so")
 
 F32, F16, BF16 = 0, 1, 2
-ATTN_AUTO, ATTN_TABLE, ATTN_DECODE_MMA = 0, 1, 2
+ATTN_AUTO, ATTN_TABLE, ATTN_DECODE_MMA, ATTN_GENERIC = 0, 1, 2, 3
 ATTEND_PREPARED = 1
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "WORKSPACE", 5: "DEVICE_CHECK"}

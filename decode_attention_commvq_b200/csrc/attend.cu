@@ -122,12 +122,25 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(AttendArgs a, 
   }
 }
 
-// Algorithm actually run for a request (AUTO -> decode-and-rotate when it supports the shape).
+// Whether an algorithm takes the shape (the table's shared-memory fit is checked at the call).
+bool algo_supported(const commvq_config* cfg, int algo) {
+  const bool g8 = cfg->g == kG && cfg->n_codes <= 256;
+  switch (algo) {
+    case COMMVQ_ATTN_DECODE_MMA: return g8 && mma_supported(cfg->R, cfg->q_heads, cfg->kv_heads, cfg->n_codes);
+    case COMMVQ_ATTN_TABLE: return g8 && cfg->R <= 4;
+    case COMMVQ_ATTN_GENERIC: return generic_supported(cfg);
+    default: return false;
+  }
+}
+
+// Algorithm actually run for a request: AUTO takes decode-and-rotate, else the table form,
+// else the generic form, whichever first supports the shape (-1: none).
 int resolve_algo(const commvq_config* cfg, const commvq_attend_options* opt) {
   const int algo = opt ? opt->algo : COMMVQ_ATTN_AUTO;
   if (algo != COMMVQ_ATTN_AUTO) return algo;
-  return mma_supported(cfg->R, cfg->q_heads, cfg->kv_heads, cfg->n_codes) ? COMMVQ_ATTN_DECODE_MMA
-                                                                          : COMMVQ_ATTN_TABLE;
+  for (int a : {COMMVQ_ATTN_DECODE_MMA, COMMVQ_ATTN_TABLE, COMMVQ_ATTN_GENERIC})
+    if (algo_supported(cfg, a)) return a;
+  return -1;
 }
 
 // Split-T partitions per sequence. Table form: one CTA per (sequence, query head, split);
@@ -142,6 +155,10 @@ int choose_splits(int algo, int B, int q_heads, int64_t max_T, const commvq_atte
     S = B >= sms ? 1 : sms / B;
     const int64_t by_len = (max_T + 15) / 16;
     if (S > by_len) S = by_len;
+  } else if (algo == COMMVQ_ATTN_GENERIC) {   // latency bound: several CTAs per SM
+    S = 4 * sms / B;
+    const int64_t by_len = (max_T + 63) / 64;
+    if (S > by_len) S = by_len;
   } else {
     const int64_t units = static_cast<int64_t>(B) * q_heads;
     S = units >= sms ? 1 : sms / units;
@@ -153,15 +170,24 @@ int choose_splits(int algo, int B, int q_heads, int64_t max_T, const commvq_atte
   return static_cast<int>(S);
 }
 
+// Partial slots per (sequence, head): the generic form writes one per warp of a KV head.
+int partial_slots(const commvq_config* cfg, int algo, int S) {
+  return algo == COMMVQ_ATTN_GENERIC ? S * generic_warps_per_kv(cfg->kv_heads) : S;
+}
+
 struct WorkspaceLayout {
-  size_t partials_off, kimg_off, vimg_off, phase_off, scores_off, total;
+  size_t partials_off, kimg_off, vimg_off, phase_off, scores_off, tables_off, total;
 };
 constexpr size_t kPhaseBytes = 64 * sizeof(double) + 128 * 64 * 8 + 64 * 8;   // theta, rows, advance
 
 WorkspaceLayout workspace_layout(const commvq_config* cfg, int algo, int B, int64_t max_T, int S) {
   WorkspaceLayout L{};
   L.partials_off = kHeaderBytes;
-  size_t end = L.partials_off + static_cast<size_t>(B) * cfg->q_heads * S * sizeof(Partial);
+  size_t end = L.partials_off + static_cast<size_t>(B) * cfg->q_heads * partial_slots(cfg, algo, S) * sizeof(Partial);
+  if (algo == COMMVQ_ATTN_GENERIC) {
+    L.tables_off = round_up(end, 256);
+    end = L.tables_off + generic_tables_bytes(max_T);
+  }
   if (algo == COMMVQ_ATTN_DECODE_MMA) {
     const size_t img = static_cast<size_t>(512) * cfg->n_codes;
     L.kimg_off = round_up(end, 256);
@@ -183,7 +209,7 @@ commvq_status check_config(const commvq_config* cfg) {
       !isfinite(cfg->rope_base))
     return COMMVQ_ERR_INVALID_ARG;
   if (cfg->code_bytes != (Nc <= 256 ? 1 : 2)) return COMMVQ_ERR_INVALID_ARG;
-  if (d != kD || g != kG || Nc > 256 || R > 4) return COMMVQ_ERR_UNSUPPORTED;
+  if (d != kD || (g != 8 && g != 16 && g != 32 && g != 64) || R > 32) return COMMVQ_ERR_UNSUPPORTED;
   if (cfg->q_heads > 65535) return COMMVQ_ERR_UNSUPPORTED;
   return COMMVQ_OK;
 }
@@ -196,11 +222,10 @@ using namespace commvq;
 extern "C" size_t commvq_attend_workspace_bytes(const commvq_config* cfg, int32_t B, int64_t max_T,
                                                 const commvq_attend_options* options) {
   if (check_config(cfg) != COMMVQ_OK || B < 0 || max_T < 0) return 0;
-  if (options && (options->splits < 0 || options->splits > kMaxSplits || options->algo < 0 || options->algo > 2))
+  if (options && (options->splits < 0 || options->splits > kMaxSplits || options->algo < 0 || options->algo > 3))
     return 0;
   const int algo = resolve_algo(cfg, options);
-  if (algo == COMMVQ_ATTN_DECODE_MMA && !mma_supported(cfg->R, cfg->q_heads, cfg->kv_heads, cfg->n_codes))
-    return 0;
+  if (!algo_supported(cfg, algo)) return 0;
   const int S = choose_splits(algo, B > 0 ? B : 1, cfg->q_heads, max_T, options);
   return workspace_layout(cfg, algo, B, max_T, S).total;
 }
@@ -219,8 +244,7 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
     return COMMVQ_ERR_INVALID_ARG;
   const int algo = options ? options->algo : COMMVQ_ATTN_AUTO;
   if (options && (options->splits < 0 || options->splits > kMaxSplits)) return COMMVQ_ERR_INVALID_ARG;
-  if (algo != COMMVQ_ATTN_AUTO && algo != COMMVQ_ATTN_TABLE && algo != COMMVQ_ATTN_DECODE_MMA)
-    return COMMVQ_ERR_INVALID_ARG;
+  if (algo < COMMVQ_ATTN_AUTO || algo > COMMVQ_ATTN_GENERIC) return COMMVQ_ERR_INVALID_ARG;
   if (B == 0) return COMMVQ_OK;
   if (B > 65535) return COMMVQ_ERR_UNSUPPORTED;
   if (!q || !k_codes || !v_codes || !seq_offsets || !k_codebook || !v_codebook || !out || !workspace)
@@ -229,20 +253,18 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
       !aligned(v_codebook, 16) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(seq_offsets, 8) ||
       !aligned(workspace, 256))
     return COMMVQ_ERR_INVALID_ARG;
-  if (algo == COMMVQ_ATTN_DECODE_MMA && !mma_supported(cfg->R, cfg->q_heads, cfg->kv_heads, cfg->n_codes))
-    return COMMVQ_ERR_UNSUPPORTED;
+  const int run = resolve_algo(cfg, options);
+  if (!algo_supported(cfg, run)) return COMMVQ_ERR_UNSUPPORTED;
   const size_t need = commvq_attend_workspace_bytes(cfg, B, max_T, options);
   if (need == 0 || workspace_bytes < need) return COMMVQ_ERR_WORKSPACE;
 
   const DeviceInfo di = current_device_info();
   if (di.device < 0) return COMMVQ_ERR_CUDA;
-  const int run = resolve_algo(cfg, options);
   if (run == COMMVQ_ATTN_DECODE_MMA) {
-    if (!mma_supported(cfg->R, cfg->q_heads, cfg->kv_heads, cfg->n_codes)) return COMMVQ_ERR_UNSUPPORTED;
     if (mma_scores_smem_bytes(cfg->R, cfg->kv_heads, cfg->n_codes) > di.smem_optin ||
         mma_values_smem_bytes(cfg->R, cfg->kv_heads, cfg->q_heads, cfg->n_codes) > di.smem_optin)
       return COMMVQ_ERR_UNSUPPORTED;
-  } else if (table_smem_bytes(cfg->R, cfg->n_codes) > di.smem_optin) {
+  } else if (run == COMMVQ_ATTN_TABLE && table_smem_bytes(cfg->R, cfg->n_codes) > di.smem_optin) {
     return COMMVQ_ERR_UNSUPPORTED;
   }
 
@@ -289,20 +311,21 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
       return COMMVQ_ERR_CUDA;
     }
     rc = launch_attend_mma(a, q, q_dtype, S, st);
+  } else if (run == COMMVQ_ATTN_GENERIC) {
+    rc = launch_attend_generic(a, cfg, q, q_dtype, S, ws + L.tables_off, st);   // clears the error word
   } else {
     if (cudaMemsetAsync(a.error_word, 0, sizeof(int), st) != cudaSuccess) return COMMVQ_ERR_CUDA;
-    // External records so the events keep their timestamps inside a captured CUDA graph too.
-    if (a.main_start && cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a.main_start), st,
-                                                 cudaEventRecordExternal) != cudaSuccess)
+    // Timing events around the main kernel (external event nodes when the stream is captured).
+    if (a.main_start && record_event(a.main_start, st) != cudaSuccess)
       return COMMVQ_ERR_CUDA;
     rc = launch_attend_table(a, q, q_dtype, S, st);
     if (rc == COMMVQ_OK && a.main_stop &&
-        cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a.main_stop), st, cudaEventRecordExternal) !=
+        record_event(a.main_stop, st) !=
             cudaSuccess)
       return COMMVQ_ERR_CUDA;
   }
   if (rc != COMMVQ_OK) return rc;
-  return launch_combine(a, S, st);
+  return launch_combine(a, partial_slots(cfg, run, S), st);
 }
 
 extern "C" commvq_status commvq_attend_prepare(const commvq_config* cfg, int32_t B, int64_t max_T,
@@ -314,21 +337,19 @@ extern "C" commvq_status commvq_attend_prepare(const commvq_config* cfg, int32_t
   if (B < 0 || max_T < 0) return COMMVQ_ERR_INVALID_ARG;
   const int algo = options ? options->algo : COMMVQ_ATTN_AUTO;
   if (options && (options->splits < 0 || options->splits > kMaxSplits)) return COMMVQ_ERR_INVALID_ARG;
-  if (algo != COMMVQ_ATTN_AUTO && algo != COMMVQ_ATTN_TABLE && algo != COMMVQ_ATTN_DECODE_MMA)
-    return COMMVQ_ERR_INVALID_ARG;
+  if (algo < COMMVQ_ATTN_AUTO || algo > COMMVQ_ATTN_GENERIC) return COMMVQ_ERR_INVALID_ARG;
   if (B == 0) return COMMVQ_OK;
   if (B > 65535) return COMMVQ_ERR_UNSUPPORTED;
   if (!k_codebook || !v_codebook || !workspace) return COMMVQ_ERR_INVALID_ARG;
   if (!aligned(k_codebook, 16) || !aligned(v_codebook, 16) || !aligned(workspace, 256))
     return COMMVQ_ERR_INVALID_ARG;
-  if (algo == COMMVQ_ATTN_DECODE_MMA && !mma_supported(cfg->R, cfg->q_heads, cfg->kv_heads, cfg->n_codes))
-    return COMMVQ_ERR_UNSUPPORTED;
+  const int run = resolve_algo(cfg, options);
+  if (!algo_supported(cfg, run)) return COMMVQ_ERR_UNSUPPORTED;
   const size_t need = commvq_attend_workspace_bytes(cfg, B, max_T, options);
   if (need == 0 || workspace_bytes < need) return COMMVQ_ERR_WORKSPACE;
   const DeviceInfo di = current_device_info();
   if (di.device < 0) return COMMVQ_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int run = resolve_algo(cfg, options);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   if (run != COMMVQ_ATTN_DECODE_MMA)
     return cudaMemsetAsync(workspace, 0, sizeof(int), st) == cudaSuccess ? COMMVQ_OK : COMMVQ_ERR_CUDA;

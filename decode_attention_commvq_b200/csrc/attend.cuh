@@ -54,5 +54,10 @@ commvq_status launch_attend_mma(const AttendArgs& a, const void* q, commvq_dtype
 commvq_status launch_attend_table(const AttendArgs& a, const void* q, commvq_dtype qt, int splits,
                                   cudaStream_t st);
 commvq_status launch_combine(const AttendArgs& a, int splits, cudaStream_t st);
+bool generic_supported(const commvq_config* cfg);
+int generic_warps_per_kv(int kv_heads);
+size_t generic_tables_bytes(int64_t max_T);
+commvq_status launch_attend_generic(const AttendArgs& a, const commvq_config* cfg, const void* q,
+                                    commvq_dtype qt, int S, void* tables, cudaStream_t st);
 
 }  // namespace commvq

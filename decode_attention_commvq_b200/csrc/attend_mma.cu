@@ -254,7 +254,10 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
   float4* base_all = reinterpret_cast<float4*>(red + kMmaWarps * KV * 8);   // [16 warps][32] refreshes
   uint8_t* stage_all = reinterpret_cast<uint8_t*>(base_all + kMmaWarps * 32);   // [16 warps][2][8 rows][KV R][16]
   using SL = StageLayout<R, KV>;
-  constexpr int kWarpStage = kRows * SL::kPieces * 16;                // one warp's rows of one stage
+  // One warp's rows of one stage, each padded to at least 8 pieces of 16 bytes so that a
+  // 3-bit XOR swizzle has room (see kRowSwz).
+  constexpr int kRowPieces = SL::kPieces > 8 ? SL::kPieces : 8;
+  constexpr int kWarpStage = kRows * kRowPieces * 16;
 
   const int s = blockIdx.x, b = blockIdx.y, S = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -270,6 +273,11 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
 
   // Each warp streams its own rows: the 8 rows 8w..8w+7 of every 128-position stage, into a
   // private double buffer (XOR-swizzled pieces, as StageLayout), with no CTA barrier in the loop.
+  // Piece p of warp row r sits at slot p ^ (r & kRowSwz). With two rounds a row reads piece
+  // kv R + (r' ^ parity), the round order already flipped by the row's parity, so only bits 1-2
+  // of the row enter the XOR; with one round all three do. Either way the 8 rows of a load fall
+  // in 8 different 16-byte bank groups.
+  constexpr int kRowSwz = R == 2 ? 6 : 7;
   uint8_t* wstage = stage_all + warp * 2 * kWarpStage;
   auto issue_rows = [&](int buf, int64_t t0) {
     const int64_t r0 = t0 + warp * kRows;
@@ -277,7 +285,7 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
     const uint8_t* src = a.k_codes + (row0 + r0) * (SL::kPieces * 16);
     for (int p = lane; p < n * SL::kPieces; p += 32) {
       const int row = p / SL::kPieces, piece = p - row * SL::kPieces;
-      cp_async16(wstage + buf * kWarpStage + SL::offset(row, piece), src + p * 16);
+      cp_async16(wstage + buf * kWarpStage + (row * kRowPieces + (piece ^ (row & kRowSwz))) * 16, src + p * 16);
     }
   };
   // Set-up: asynchronous copies of the prepared codebook image and advance phasors, then the
@@ -334,9 +342,9 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
     gF[u] = static_cast<uint32_t>(slot(par, 4 * u + i, 0, Nc)) * 16;
     gS[u] = static_cast<uint32_t>(slot(par ^ 1, 4 * u + i, 0, Nc)) * 16;
   }
-  // The row's record: piece kv R + r sits at 16 ((kv R + r) ^ swz), swz = the row's low bits.
-  const int swz = g & SL::kSwz;
-  const uint32_t cw_lane = static_cast<uint32_t>(g * SL::kPieces * 16);
+  // The row's record: piece kv R + r sits at 16 ((kv R + r) ^ swz), swz = g & kRowSwz.
+  const int swz = g & kRowSwz;
+  const uint32_t cw_lane = static_cast<uint32_t>(g * kRowPieces * 16);
   // score buffer slot of this row: 16-position tile, values-kernel quad g/2, k = (g&1) + 2 (w&1)
   const int sc_k = (g & 1) + 2 * (warp & 1);
   float* red_w = red + warp * KV * 8;
@@ -687,7 +695,7 @@ commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt,
   const size_t smem_v = mma_values_smem_bytes(R, KV, a.q_heads, a.n_codes);
   dim3 grid(S, a.B);
   if (a.main_start &&
-      cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a.main_start), st, cudaEventRecordExternal) != cudaSuccess)
+      record_event(a.main_start, st) != cudaSuccess)
     return COMMVQ_ERR_CUDA;
 #define COMMVQ_LAUNCH_SCORES(T)                                                                      \
   {                                                                                                \
@@ -710,7 +718,7 @@ commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt,
     k<<<grid, kMmaThreads, smem_v, st>>>(a);
   }
   if (a.main_stop &&
-      cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a.main_stop), st, cudaEventRecordExternal) != cudaSuccess)
+      record_event(a.main_stop, st) != cudaSuccess)
     return COMMVQ_ERR_CUDA;
   return launch_status();
 }
@@ -735,9 +743,10 @@ commvq_status launch_mma_kv(const AttendArgs& a, const void* q, commvq_dtype qt,
 }  // namespace
 
 size_t mma_scores_smem_bytes(int R, int KV, int n_codes) {
+  const size_t row_pieces = KV * R > 8 ? static_cast<size_t>(KV * R) : 8;
   return static_cast<size_t>(512) * n_codes + static_cast<size_t>(KV) * 8 * 32 * 8 + 2 * 32 * sizeof(float4) +
          static_cast<size_t>(kMmaWarps) * KV * 8 * 4 + static_cast<size_t>(kMmaWarps) * 32 * sizeof(float4) +
-         static_cast<size_t>(2) * kStageT * KV * R * kGroups;
+         static_cast<size_t>(2) * kStageT * row_pieces * 16;
 }
 
 size_t mma_values_smem_bytes(int R, int KV, int q_heads, int n_codes) {

@@ -36,6 +36,18 @@ DeviceInfo current_device_info();
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Record a caller's timing event on `st`. Inside a stream capture the record becomes an
+// external event node, so the event keeps real timestamps when the graph is replayed; outside
+// a capture it is an ordinary record.
+inline cudaError_t record_event(void* ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  const cudaError_t e = cudaStreamIsCapturing(st, &cs);
+  if (e != cudaSuccess) return e;
+  return cs == cudaStreamCaptureStatusActive
+             ? cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev), st, cudaEventRecordExternal)
+             : cudaEventRecord(static_cast<cudaEvent_t>(ev), st);
+}
+
 // ---------------------------------------------------------------------------------------
 // Nearest entry of a sub-codebook, the encoder's distance rule. Exactly the fp32 operations
 // the definition names, so codes are reproducible bit for bit:
@@ -66,6 +78,29 @@ __device__ __forceinline__ void nearest_step(Nearest& n, const float (&res)[kG],
   e = __fsub_rn(res[5], hi.y); dist = __fmaf_rn(e, e, dist);
   e = __fsub_rn(res[6], hi.z); dist = __fmaf_rn(e, e, dist);
   e = __fsub_rn(res[7], hi.w); dist = __fmaf_rn(e, e, dist);
+  if (dist < n.best) {
+    if (kTrack) n.second = n.best;
+    n.best = dist;
+    n.idx = c;
+  } else if (kTrack && dist < n.second) {
+    n.second = dist;
+  }
+}
+
+// Nearest entry for GG-scalar groups: the same fp32 rule as nearest_step (subtract, then a fused
+// multiply-add, k = 0..GG-1 in order; strictly smaller wins), entry read from shared memory.
+template <int GG, bool kTrack>
+__device__ __forceinline__ void nearest_step_g(Nearest& n, const float (&res)[GG], const float4* e, int c) {
+  float dist = 0.0f;
+#pragma unroll
+  for (int q = 0; q < GG / 4; ++q) {
+    const float4 v = e[q];
+    float t;
+    t = __fsub_rn(res[4 * q + 0], v.x); dist = __fmaf_rn(t, t, dist);
+    t = __fsub_rn(res[4 * q + 1], v.y); dist = __fmaf_rn(t, t, dist);
+    t = __fsub_rn(res[4 * q + 2], v.z); dist = __fmaf_rn(t, t, dist);
+    t = __fsub_rn(res[4 * q + 3], v.w); dist = __fmaf_rn(t, t, dist);
+  }
   if (dist < n.best) {
     if (kTrack) n.second = n.best;
     n.best = dist;

@@ -709,12 +709,12 @@ extern "C" commvq_status commvq_dense_decode(const commvq_config* cfg, const voi
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   void* start = options ? options->main_start : nullptr;
   void* stop = options ? options->main_stop : nullptr;
-  if (start && cudaEventRecordWithFlags(static_cast<cudaEvent_t>(start), st, cudaEventRecordExternal) != cudaSuccess)
+  if (start && record_event(start, st) != cudaSuccess)
     return COMMVQ_ERR_CUDA;
   const commvq_status rc = kv_dtype == COMMVQ_F16 ? launch_dense_kv<__half>(d, q, q_dtype, S, st)
                                                   : launch_dense_kv<__nv_bfloat16>(d, q, q_dtype, S, st);
   if (rc != COMMVQ_OK) return rc;
-  if (stop && cudaEventRecordWithFlags(static_cast<cudaEvent_t>(stop), st, cudaEventRecordExternal) != cudaSuccess)
+  if (stop && record_event(stop, st) != cudaSuccess)
     return COMMVQ_ERR_CUDA;
   AttendArgs c{};
   c.out = out;

@@ -98,8 +98,8 @@ class Workload:
         return replace(self, **kw)
 
 
-# The five workloads, in order: tiny fp32 case, 2-bit 32K layer, 1-bit 128K layer,
-# ragged batch of 16, and the encode + codebook-fit workload.
+# The workloads, in order: tiny fp32 case, 2-bit 32K layer, 1-bit 128K layer, ragged batch of
+# 16, the encode + codebook-fit workload, and the pages' own g = 64 setting at 2 and 1 bits.
 WORKLOADS = [
     Workload(name="tiny_fp32_T256_R1_N16", seed=0, R=1, n_codes=16, q_heads=1, kv_heads=1,
              rope_base=10000.0, seq_len=256, kv_dtype="f32", q_dtype="f32", n_outliers=0,
@@ -110,6 +110,10 @@ WORKLOADS = [
              ragged=(4096, 8192)),
     Workload(name="encode_fit_131072x8", seed=4, R=2, encode_tokens=131072, em_rows=65536,
              em_iters=10),
+    # the pages' own hyper-parameters: 64 scalars per index, 64 entries, 21 (2-bit) or 11
+    # (1-bit) residual rounds: R * log2(64) / 64 = 1.97 and 1.03 bits per scalar
+    Workload(name="pages_g64_2bit_T32768", seed=5, g=64, R=21, n_codes=64, seq_len=32768),
+    Workload(name="pages_g64_1bit_T32768", seed=6, fit_seed=5, g=64, R=11, n_codes=64, seq_len=32768),
 ]
 # The 1-bit layer and the ragged batch take their codebooks (and outlier channels) from
 # the 2-bit layer's fit seed: under sequential residual fitting the R=1 codebook is

@@ -14,8 +14,9 @@
  * multiply).
  *
  * Conventions shared by every call
- *  - d = 128, g = 8 (4 RoPE pairs per index), d/g = 16 groups for attention; the
- *    encoder and the EM step accept any d that is a multiple of 8 with g = 8.
+ *  - g = 8 (4 RoPE pairs per index, d/g = 16 groups) is the layout of the fast attention
+ *    kernels; g = 16, 32 and 64 (the pages' own g) are taken by the encoder, the hard EM
+ *    step and the GENERIC attention algorithm. Attention needs d = 128.
  *  - RoPE pair p is channels (2p, 2p+1), theta_p = rope_base^(-2p/d); the key of row t of
  *    a sequence sits at position t; queries arrive already rotated; scores are scaled
  *    by 1/sqrt(d); there is no mask.
@@ -63,7 +64,9 @@ typedef enum { COMMVQ_F32 = 0, COMMVQ_F16 = 1, COMMVQ_BF16 = 2 } commvq_dtype;
 typedef enum {
   COMMVQ_ATTN_AUTO = 0,       /* the library's fastest for the shape */
   COMMVQ_ATTN_TABLE = 1,      /* per-query table + value histograms, one CTA per (b, q head, split) */
-  COMMVQ_ATTN_DECODE_MMA = 2  /* decode each (token, KV head) once, rotate, tensor-core QK and PV */
+  COMMVQ_ATTN_DECODE_MMA = 2, /* decode each (token, KV head) once, rotate, tensor-core QK and PV */
+  COMMVQ_ATTN_GENERIC = 3     /* any g in {8, 16, 32, 64}, R <= 32, Nc' <= 65536: fp32 decode from
+                                 the fp32 codebooks, one warp per (token, KV head) */
 } commvq_attn_algo;
 
 typedef struct {
@@ -112,7 +115,8 @@ typedef struct {
  * residual_out nullable [n_tokens, kv_heads, d] float32, 16-byte aligned: the residual
  *          after the last round (what a further round, or the next round of a codebook
  *          fit, would encode).
- * Supports g = 8, d % 8 == 0, 1 <= Nc' <= 65536, 1 <= R <= 16. n_tokens = 0 is a no-op. */
+ * Supports g in {8, 16, 32, 64}, d % g == 0, 1 <= Nc' <= 65536, 1 <= R <= 32. n_tokens = 0 is
+ * a no-op. */
 commvq_status commvq_encode(const commvq_config* cfg, const void* x, commvq_dtype x_dtype,
                             int64_t n_tokens, const float* codebook, void* codes,
                             unsigned long long* near_ties, float* residual_out, void* stream);
@@ -138,8 +142,8 @@ size_t commvq_attend_workspace_bytes(const commvq_config* cfg, int32_t B, int64_
  * cores as two fp16 terms (value and rounding error), so only the entries' own rounding reaches
  * the scores; softmax weights and value entries enter the second product in fp16.
  * q           [B, q_heads, d] in q_dtype (F32, F16 or BF16), 16-byte aligned.
- * k_codes, v_codes  [total_T, kv_heads, R, d/g] uint8 (attention supports Nc' <= 256),
- *             16-byte aligned; total_T = seq_offsets[B].
+ * k_codes, v_codes  [total_T, kv_heads, R, d/g], code_bytes per element (uint16 above 256
+ *             entries, GENERIC only), 16-byte aligned; total_T = seq_offsets[B].
  * seq_offsets [B+1] int64 device array, non-decreasing, seq_offsets[0] = 0, every
  *             T_b <= max_T (a longer sequence is truncated to max_T rows: the caller
  *             must pass the true maximum).
@@ -152,8 +156,13 @@ size_t commvq_attend_workspace_bytes(const commvq_config* cfg, int32_t B, int64_
  * options     nullable (defaults: AUTO algorithm, library-chosen splits, no flags). With
  *             COMMVQ_ATTEND_PREPARED the workspace's prepared state (see commvq_attend_prepare)
  *             is used as it stands; otherwise the call writes it first.
- * Supports d = 128, g = 8, Nc' <= 256 (code_bytes = 1), 1 <= R <= 4, q_heads % kv_heads == 0,
- * B >= 0 (B = 0 is a no-op). */
+ * Shapes: d = 128, q_heads % kv_heads == 0, B >= 0 (B = 0 is a no-op), and per algorithm
+ *   DECODE_MMA  g = 8, R <= 2, Nc' <= 256, kv_heads in {1, 2, 4, 8}, q_heads / kv_heads <= 8;
+ *   TABLE       g = 8, R <= 4, Nc' <= 256;
+ *   GENERIC     g in {8, 16, 32, 64}, R <= 32, Nc' <= 65536, kv_heads in {1, 2, 4, 8},
+ *               q_heads / kv_heads <= 16 (the pages' g = 64, Nc' = 64, R = 21 / 11 setting).
+ * AUTO takes the first of DECODE_MMA, TABLE, GENERIC that accepts the shape; an explicit algo
+ * that does not accept it returns COMMVQ_ERR_UNSUPPORTED. */
 commvq_status commvq_attend_decode(const commvq_config* cfg, const void* q, commvq_dtype q_dtype,
                                    const void* k_codes, const void* v_codes,
                                    const int64_t* seq_offsets, int32_t B, int64_t max_T,
@@ -222,7 +231,7 @@ size_t commvq_em_workspace_bytes(const commvq_config* cfg, int64_t N);
  *                accumulated in fp64.
  * workspace      >= commvq_em_workspace_bytes(cfg, N) bytes, 256-byte aligned.
  * The result does not depend on launch order (fixed-order fp64 reductions). Supports
- * g = 8, d % 8 == 0, 1 <= Nc' <= 4096, N >= 1. cfg->R is ignored. */
+ * g in {8, 16, 32, 64}, d % g == 0, 1 <= Nc' <= 4096, N >= 1. cfg->R is ignored. */
 commvq_status commvq_em_step(const commvq_config* cfg, const float* rows, int64_t N,
                              float* codebook_round, void* codes_out, double* sse_out,
                              void* workspace, size_t workspace_bytes, void* stream);
@@ -237,7 +246,8 @@ commvq_status commvq_em_step(const commvq_config* cfg, const float* rows, int64_
  * sse_out: sum over (row, group) of d_min (the hard distortion against the input codebook).
  * tau must be finite and > 0 (COMMVQ_ERR_INVALID_ARG otherwise); as tau -> 0 the step tends
  * to commvq_em_step. Arguments, workspace (commvq_em_workspace_bytes covers both steps) and
- * limits are those of commvq_em_step. Deterministic run to run. */
+ * limits are those of commvq_em_step, except that this step takes g = 8 only. Deterministic
+ * run to run. */
 commvq_status commvq_em_step_soft(const commvq_config* cfg, const float* rows, int64_t N,
                                   float* codebook_round, float tau, double* sse_out,
                                   void* workspace, size_t workspace_bytes, void* stream);

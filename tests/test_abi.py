@@ -72,8 +72,10 @@ def test_attend_rejects_bad_arguments(api):
     assert _attend(api, _cfg(api, n_codes=0)) == INVALID
     assert _attend(api, _cfg(api, rope_base=-1.0)) == INVALID
     assert _attend(api, _cfg(api, d=64)) == UNSUP
-    assert _attend(api, _cfg(api, n_codes=512)) == UNSUP            # uint16 codes
-    assert _attend(api, _cfg(api, R=5)) == UNSUP
+    assert _attend(api, _cfg(api, g=128)) == UNSUP                  # group width
+    assert _attend(api, _cfg(api, R=40)) == UNSUP
+    assert _attend(api, _cfg(api, n_codes=512), opts=api.CAttendOptions(2, 0)) == UNSUP   # MMA: uint16 codes
+    assert _attend(api, _cfg(api, g=64, n_codes=64), opts=api.CAttendOptions(1, 0)) == UNSUP   # table: g = 8 only
     assert _attend(api, cfg, q=0) == INVALID
     assert _attend(api, cfg, q=FAKE + 8) == INVALID                 # misaligned
     assert _attend(api, cfg, ws=FAKE + 16) == INVALID               # workspace alignment
@@ -81,7 +83,7 @@ def test_attend_rejects_bad_arguments(api):
     assert _attend(api, cfg, B=-1) == INVALID
     assert _attend(api, cfg, ws_bytes=16) == WS
     assert _attend(api, cfg, B=0) == 0                               # no-op
-    bad = api.CAttendOptions(9, 0)
+    bad = api.CAttendOptions(4, 0)
     assert _attend(api, cfg, opts=bad) == INVALID
     bad = api.CAttendOptions(0, -2)
     assert _attend(api, cfg, opts=bad) == INVALID
@@ -201,8 +203,22 @@ def test_prepare_rejects_bad_arguments(api):
     assert f(ctypes.byref(cc), 1, 100, P(FAKE), P(FAKE), P(FAKE + 16), 1 << 24, None, None) == INVALID
     assert f(ctypes.byref(cc), 1, 100, P(FAKE), P(FAKE), P(FAKE), 64, None, None) == WS
     assert f(ctypes.byref(cc), -1, 100, P(FAKE), P(FAKE), P(FAKE), 1 << 24, None, None) == INVALID
-    c5 = _cfg(api, R=5).c()
+    c5 = _cfg(api, R=40).c()
     assert f(ctypes.byref(c5), 1, 100, P(FAKE), P(FAKE), P(FAKE), 1 << 24, None, None) == UNSUP
     o = api.CAttendOptions(api.ATTN_DECODE_MMA, 0, None, None, 0)
     c3 = _cfg(api, R=3, n_codes=64).c()
     assert f(ctypes.byref(c3), 1, 100, P(FAKE), P(FAKE), P(FAKE), 1 << 24, ctypes.byref(o), None) == UNSUP
+
+
+def test_generic_algo_workspace(api):
+    """The pages' setting (g = 64, Nc' = 64, R = 21) resolves to the generic algorithm: partials
+    for every warp of a KV head (8 / KV) plus the phasor tables (128 offsets + one chunk per
+    128 positions, 512 B each)."""
+    cfg = _cfg(api, g=64, n_codes=64, R=21)
+    n = api.attend_workspace_bytes(cfg, 1, 32768, splits=4)
+    part = 256 + 32 * 4 * 1 * 528
+    want = -(-part // 256) * 256 + (128 + 256) * 512
+    assert n == -(-want // 256) * 256
+    assert api.attend_workspace_bytes(cfg, 1, 32768, splits=4, algo=api.ATTN_GENERIC) == n
+    assert api.attend_workspace_bytes(cfg, 1, 32768, algo=api.ATTN_DECODE_MMA) == 0
+    assert api.attend_workspace_bytes(_cfg(api, g=64, n_codes=64, R=21, q_heads=64, kv_heads=2), 1, 10) == 0

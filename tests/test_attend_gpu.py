@@ -308,3 +308,38 @@ def test_many_queries_within_bound(api, gpu):
         ref, _ = O.attend_codes(q_as_f64(w, q), kc, vc, offs, kcb, vcb, w.rope_base)
         worst = max(worst, rel_err(out, ref))
     assert worst <= tol_for(w), worst
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_timing_events_outside_and_inside_a_capture(api, gpu, algo):
+    """The caller's main-kernel events are recorded on direct launches and inside a CUDA
+    graph capture alike, and do not change the result."""
+    w, kc, vc, kcb, vcb = _encoded_inputs(synth.WORKLOADS[1], T=1000)
+    cfg = _cfg(api, w)
+    offs = w.offsets()
+    offsets = torch.from_numpy(offs.astype(np.int64)).to(gpu)
+    kcg, vcg = _codes_np_to_gpu(kc, gpu), _codes_np_to_gpu(vc, gpu)
+    kcbt, vcbt = torch.from_numpy(kcb).to(gpu), torch.from_numpy(vcb).to(gpu)
+    q = to_torch_q(synth.queries(w), w.q_dtype, gpu)
+    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    ev[0].record()   # torch times only events it has recorded once itself
+    ev[1].record()
+    ws = api.attend_workspace(cfg, 1, 1000, gpu, algo)
+    out_e, _ = api.attend_decode(cfg, q, kcg, vcg, offsets, 1000, kcbt, vcbt, workspace=ws, algo=algo,
+                                 main_events=ev)
+    torch.cuda.synchronize()
+    assert ev[0].elapsed_time(ev[1]) > 0
+    out_p, _ = api.attend_decode(cfg, q, kcg, vcg, offsets, 1000, kcbt, vcbt, workspace=ws, algo=algo)
+    torch.cuda.synchronize()
+    assert rel_err(out_e.cpu().numpy(), out_p.cpu().numpy()) <= 1e-6
+    stream = torch.cuda.Stream()
+    out_g = torch.empty_like(out_p)
+    with torch.cuda.stream(stream):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            api.attend_decode(cfg, q, kcg, vcg, offsets, 1000, kcbt, vcbt, out=out_g, workspace=ws,
+                              algo=algo, stream=stream, main_events=ev)
+        g.replay()
+    torch.cuda.synchronize()
+    assert ev[0].elapsed_time(ev[1]) > 0
+    assert rel_err(out_g.cpu().numpy(), out_p.cpu().numpy()) <= 1e-6
