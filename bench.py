@@ -205,7 +205,7 @@ def setup_inputs(w, dev, torch, api, fit):
         else:
             rows = torch.from_numpy(synth.fit_rows(w, key)).to(dev)
             cbs.append(fit.fit_codebook(rows, w.R, w.n_codes, w.em_iters,
-                                        lambda r, N, key=key: synth.forgy_indices(w, key, r, N)))
+                                        lambda r, N, key=key: synth.forgy_indices(w, key, r, N), g=w.g))
     kcb, vcb = cbs
     codes = []
     for key, cb in ((True, kcb), (False, vcb)):
@@ -484,7 +484,7 @@ def run_encode_fit(args, w, rank, world, dev):
     fit_ms = {}
     cbs = []
     warm = torch.from_numpy(synth.fit_rows(w.with_(em_rows=1024), True)).to(dev)
-    fit.fit_codebook(warm, w.R, w.n_codes, 1, lambda r, N: synth.forgy_indices(w, True, r, N))
+    fit.fit_codebook(warm, w.R, w.n_codes, 1, lambda r, N: synth.forgy_indices(w, True, r, N), g=w.g)
     for key in (True, False):
         rows = torch.from_numpy(synth.fit_rows(w, key)).to(dev)
         torch.cuda.synchronize(dev)
@@ -492,7 +492,7 @@ def run_encode_fit(args, w, rank, world, dev):
         with torch.cuda.stream(stream):
             e0.record(stream)
             cb = fit.fit_codebook(rows, w.R, w.n_codes, w.em_iters,
-                                  lambda r, N, key=key: synth.forgy_indices(w, key, r, N))
+                                  lambda r, N, key=key: synth.forgy_indices(w, key, r, N), g=w.g)
             e1.record(stream)
         torch.cuda.synchronize(dev)
         fit_ms["K" if key else "V"] = e0.elapsed_time(e1)

@@ -46,6 +46,7 @@ constexpr int kMaxSplits = 4096;
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(AttendArgs a, int S) {
   __shared__ float4 acc_s[kCombineGroups][8];
   __shared__ float ml_s[kCombineGroups][2];
+  pdl_wait();   // launched as a dependent of the kernel that writes the partials
   const int bh = blockIdx.x, quarter = blockIdx.y;
   const int tid = threadIdx.x, grp = tid >> 3, gl = tid & 7;
   const Partial* p = a.partials + static_cast<int64_t>(bh) * S;
@@ -376,7 +377,9 @@ extern "C" commvq_status commvq_attend_prepare(const commvq_config* cfg, int32_t
 
 namespace commvq {
 commvq_status launch_combine(const AttendArgs& a, int S, cudaStream_t st) {
-  combine_kernel<<<dim3(a.B * a.q_heads, kCombineQuarters), kCombineThreads, 0, st>>>(a, S);
+  if (launch_dependent(combine_kernel, dim3(a.B * a.q_heads, kCombineQuarters), dim3(kCombineThreads), 0, st, a,
+                       S) != cudaSuccess)
+    return COMMVQ_ERR_CUDA;
   return launch_status();
 }
 }  // namespace commvq

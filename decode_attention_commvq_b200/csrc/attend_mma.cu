@@ -271,6 +271,7 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
     return;
   }
 
+  pdl_trigger();   // the values kernel may take SMs as this grid's CTAs finish
   // Each warp streams its own rows: the 8 rows 8w..8w+7 of every 128-position stage, into a
   // private double buffer (XOR-swizzled pieces, as StageLayout), with no CTA barrier in the loop.
   // Piece p of warp row r sits at slot p ^ (r & kRowSwz). With two rounds a row reads piece
@@ -525,9 +526,12 @@ attend_values_kernel(AttendArgs a) {
         a.scores + score_index(b, tau0, 0, 0, 0, 0, n_tiles, KV, G));
     for (int p = tid; p < pieces; p += kMmaThreads) cp_async16(dst + p * 16, src + p * 16);
   };
+  pdl_trigger();   // the combine may be scheduled as SMs free up; it waits for this grid
+  // The prologue reads only prepared state and codes; the scores kernel may still be running.
   for (int p = tid; p < 32 * Nc; p += kMmaThreads) cp_async16(cbv + p, a.v_img + p);
   cp_async_commit();
   issue_stage<R, KV>(stage_buf, a.v_codes, row0, t_begin, t_end);
+  pdl_wait();      // the scores kernel's maxima and score buffer are complete from here on
   issue_scores(score_buf, t_begin);
   cp_async_commit();
 
@@ -715,7 +719,7 @@ commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt,
     auto k = attend_values_kernel<R, KV, NC>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_v) != cudaSuccess)
       return COMMVQ_ERR_CUDA;
-    k<<<grid, kMmaThreads, smem_v, st>>>(a);
+    if (launch_dependent(k, grid, dim3(kMmaThreads), smem_v, st, a) != cudaSuccess) return COMMVQ_ERR_CUDA;
   }
   if (a.main_stop &&
       record_event(a.main_stop, st) != cudaSuccess)

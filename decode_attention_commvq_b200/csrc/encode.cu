@@ -106,10 +106,89 @@ encode_kernel(const XT* __restrict__ x, int64_t n_rows, int d, int R, int n_code
   }
 }
 
+// Few rows (a decode step's new position): one warp per (row, group). Lane l scans entries
+// l, l+32, ... with the same fp32 distance rule (entries read through L1/L2); the warp then
+// merges (best, index, second best) by shuffles: the smallest distance wins, ties go to the
+// lowest entry, and the second best is the second smallest distance overall -- exactly what the
+// in-order scan of encode_kernel produces, so codes and near-tie counts are the same.
+constexpr int kWarpUnitsPerBlock = 8;
+
+template <typename XT, bool kTrack, int GG>
+__global__ void __launch_bounds__(32 * kWarpUnitsPerBlock)
+encode_warp_kernel(const XT* __restrict__ x, int64_t n_rows, int d, int R, int n_codes,
+                   const float* __restrict__ cb, void* __restrict__ codes, int code_bytes,
+                   unsigned long long* __restrict__ near_ties, float* __restrict__ residual_out) {
+  const int G = d / GG;
+  const int lane = threadIdx.x & 31;
+  const int64_t unit = static_cast<int64_t>(blockIdx.x) * kWarpUnitsPerBlock + (threadIdx.x >> 5);
+  if (unit >= n_rows * G) return;   // the whole warp leaves together
+  const int64_t n = unit / G;
+  const int j = static_cast<int>(unit - n * G);
+  float res[GG];
+#pragma unroll
+  for (int q = 0; q < GG / kG; ++q) {
+    float v[kG];
+    load_row8(x + n * d + j * GG + q * kG, v);
+#pragma unroll
+    for (int k = 0; k < kG; ++k) res[q * kG + k] = v[k];
+  }
+  unsigned ties = 0;
+  for (int r = 0; r < R; ++r) {
+    const float* sub = cb + (static_cast<int64_t>(r) * G + j) * n_codes * GG;
+    Nearest best;
+    nearest_init(best);
+    for (int c = lane; c < n_codes; c += 32)
+      nearest_step_g<GG, kTrack>(best, res, reinterpret_cast<const float4*>(sub + static_cast<int64_t>(c) * GG), c);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best.best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, best.idx, o);
+      const float os = __shfl_xor_sync(0xffffffffu, best.second, o);
+      const float hi = fmaxf(best.best, ob);
+      if (ob < best.best || (ob == best.best && oi < best.idx)) {
+        best.best = ob;
+        best.idx = oi;
+      }
+      best.second = fminf(hi, fminf(best.second, os));
+    }
+    if (lane == 0) {
+      if (kTrack) ties += near_tie(best, n_codes) ? 1u : 0u;
+      store_code(codes, (n * R + r) * G + j, best.idx, code_bytes);
+    }
+#pragma unroll
+    for (int q = 0; q < GG / kG; ++q) {
+      float w[kG];
+      load_row8(sub + static_cast<int64_t>(best.idx) * GG + q * kG, w);
+#pragma unroll
+      for (int k = 0; k < kG; ++k) res[q * kG + k] = __fsub_rn(res[q * kG + k], w[k]);
+    }
+  }
+  if (residual_out && lane == 0) {
+    float4* dst = reinterpret_cast<float4*>(residual_out + n * d + j * GG);
+#pragma unroll
+    for (int q = 0; q < GG / 4; ++q) dst[q] = make_float4(res[4 * q], res[4 * q + 1], res[4 * q + 2], res[4 * q + 3]);
+  }
+  if (kTrack && lane == 0 && ties) atomicAdd(near_ties, static_cast<unsigned long long>(ties));
+}
+
+// Row counts up to this many (row, group) units take the warp-per-unit kernel.
+constexpr int64_t kWarpEncodeMaxUnits = 4096;
+
 template <typename XT, int GG>
 void launch_encode_g(const XT* x, int64_t n_rows, int d, int R, int n_codes, const float* cb,
                      void* codes, int code_bytes, unsigned long long* near_ties, float* residual_out,
                      cudaStream_t s) {
+  const int64_t units = n_rows * (d / GG);
+  if (units <= kWarpEncodeMaxUnits) {
+    const unsigned blocks = static_cast<unsigned>((units + kWarpUnitsPerBlock - 1) / kWarpUnitsPerBlock);
+    if (near_ties)
+      encode_warp_kernel<XT, true, GG><<<blocks, 32 * kWarpUnitsPerBlock, 0, s>>>(
+          x, n_rows, d, R, n_codes, cb, codes, code_bytes, near_ties, residual_out);
+    else
+      encode_warp_kernel<XT, false, GG><<<blocks, 32 * kWarpUnitsPerBlock, 0, s>>>(
+          x, n_rows, d, R, n_codes, cb, codes, code_bytes, nullptr, residual_out);
+    return;
+  }
   const int64_t per_block = kThreads * (GG == 8 ? 2 : 1);
   dim3 grid(static_cast<unsigned>((n_rows + per_block - 1) / per_block), d / GG);
   if (near_ties)

@@ -117,3 +117,43 @@ def test_encode_empty(api, gpu):
     cb = torch.zeros((2, 16, 256, 8), dtype=torch.float32, device=gpu)
     codes = api.encode(cfg, x, cb)
     assert codes.shape == (0, 8, 2, 16)
+
+
+@pytest.mark.parametrize("wi", [1, 5])
+@pytest.mark.parametrize("tokens", [1, 3, 40])
+def test_few_rows_take_the_warp_encoder(gpu, wi, tokens):
+    """A decode step encodes one new position: up to 4096 (row, group) units go through the
+    warp-per-unit kernel. Codes, near-tie counts and residuals equal the oracle's, at the
+    library's g = 8 (R = 2, 256 entries) and the pages' g = 64 (R = 21, 64 entries)."""
+    from decode_attention_commvq_b200 import api
+    w = synth.WORKLOADS[wi]
+    cfg = api.Config(d=w.d, g=w.g, R=w.R, n_codes=w.n_codes, q_heads=w.q_heads, kv_heads=w.kv_heads)
+    kcb, _ = oracle_codebooks(w)
+    x = synth.kv_rows(w, True, tokens, sub=777, dtype="f16")
+    ref, ties, res_ref = O.encode(x, kcb, want_residual=True)
+    nt = torch.zeros(1, dtype=torch.int64, device=gpu)
+    res = torch.empty(x.shape, dtype=torch.float32, device=gpu)
+    codes = api.encode(cfg, torch.from_numpy(x).to(gpu), torch.from_numpy(kcb).to(gpu), near_ties=nt,
+                       residual_out=res)
+    torch.cuda.synchronize()
+    assert np.array_equal(codes.cpu().numpy().astype(np.int64), ref.astype(np.int64))
+    assert int(nt.item()) == ties
+    assert np.array_equal(res.cpu().numpy(), res_ref)
+
+
+def test_warp_encoder_ties_and_tiny_codebooks(gpu):
+    """Exact ties (duplicated entries) go to the lowest index and count as near ties; fewer
+    entries (5) than lanes."""
+    from decode_attention_commvq_b200 import api
+    rng = np.random.default_rng(97)
+    cb = rng.standard_normal((2, 16, 5, 8)).astype(np.float32)
+    cb[:, :, 3] = cb[:, :, 1]                       # entries 1 and 3 identical
+    x = cb[0, :, 1].reshape(1, 1, 128).astype(np.float32) + 0.0   # row = entry 1 exactly
+    cfg = api.Config(d=128, g=8, R=2, n_codes=5, q_heads=1, kv_heads=1)
+    nt = torch.zeros(1, dtype=torch.int64, device=gpu)
+    codes = api.encode(cfg, torch.from_numpy(x).to(gpu), torch.from_numpy(cb).to(gpu), near_ties=nt)
+    torch.cuda.synchronize()
+    ref, ties = O.encode(x, cb)
+    assert np.array_equal(codes.cpu().numpy().astype(np.int64), ref.astype(np.int64))
+    assert int(nt.item()) == ties and ties >= 16
+    assert (codes.cpu().numpy()[0, 0, 0] == 1).all()
