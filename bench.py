@@ -200,7 +200,9 @@ def setup_inputs(w, dev, torch, api, fit):
                      kv_heads=w.kv_heads, rope_base=w.rope_base)
     cbs = []
     for key in (True, False):
-        if w.codebook == "normal":
+        if w.v_bits and not key:    # binary value code: C [n_bits, kv_heads * d]
+            cbs.append(torch.from_numpy(synth.binary_value_codebook(w)).to(dev))
+        elif w.codebook == "normal":
             cbs.append(torch.from_numpy(synth.normal_codebook(w, key)).to(dev))
         else:
             rows = torch.from_numpy(synth.fit_rows(w, key)).to(dev)
@@ -209,6 +211,9 @@ def setup_inputs(w, dev, torch, api, fit):
     kcb, vcb = cbs
     codes = []
     for key, cb in ((True, kcb), (False, vcb)):
+        if w.v_bits and not key:    # seeded uniform bits (the value encoder is a learned network)
+            codes.append(torch.from_numpy(synth.value_bits(w, int(w.lengths().sum()))).to(dev))
+            continue
         parts = []
         L = w.lengths()
         for b in range(w.batch):
@@ -241,12 +246,24 @@ def run_ours(args, w, rank, world, dev):
     n_copies = max(1, math.ceil(3 * l2 / code_bytes))
     kcs = [kc] + [kc.clone() for _ in range(n_copies - 1)]
     vcs = [vc] + [vc.clone() for _ in range(n_copies - 1)]
+    # the binary code's C rotates with the codes, so that it is read from HBM like a layer's
+    # parameters in a many-layer model
+    cs = [vcb] + [vcb.clone() for _ in range(n_copies - 1)] if w.v_bits else None
     out = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32, device=dev)
     lse = torch.empty((w.batch, w.q_heads), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
     K, W = args.steps, args.warmup
     naive = args.path == "naive"
-    if naive:
+    binv = w.v_bits > 0
+    if binv and (naive or args.algo not in (0, api.ATTN_DECODE_MMA)):
+        raise SystemExit("the binary value code runs with the decode-and-rotate keys only")
+    if binv:
+        ws = torch.empty(api.attend_binv_workspace_bytes(cfg, w.v_bits, w.batch, max_T), dtype=torch.uint8,
+                         device=dev)
+        # the layer's key-side state (fp16 images, RoPE tables), once per layer
+        api.attend_decode_binv(cfg, q, kc, vc, offs, max_T, kcb, vcb, out=out, lse=lse, workspace=ws,
+                               stream=stream)
+    elif naive:
         ndt = torch.bfloat16 if args.naive_dtype == "bf16" else torch.float16
         k_rows = torch.empty((total_T, w.kv_heads, w.d), dtype=ndt, device=dev)
         v_rows = torch.empty_like(k_rows)
@@ -259,8 +276,16 @@ def run_ours(args, w, rank, world, dev):
         api.attend_prepare(cfg, w.batch, max_T, kcb, vcb, ws, args.algo, args.splits, stream)
     prepared = not naive and not args.unprepared
 
-    def attend(kc_i, vc_i, q_i, out_i, lse_i, events=None, prep=None):
-        if naive:
+    def attend(kc_i, vc_i, q_i, out_i, lse_i, events=None, prep=None, i=0):
+        if binv:
+            if events is not None:
+                events[0].record(stream)
+            api.attend_decode_binv(cfg, q_i, kc_i, vc_i, offs, max_T, kcb, cs[i % n_copies], out=out_i, lse=lse_i,
+                                   workspace=ws, want_lse=lse_i is not None,
+                                   prepared=prepared if prep is None else prep, stream=stream)
+            if events is not None:
+                events[1].record(stream)
+        elif naive:
             api.decompress(cfg, kc_i, vc_i, offs, max_T, kcb, vcb, k_out=k_rows, v_out=v_rows,
                            workspace=ws, stream=stream)
             api.dense_decode(cfg, q_i, k_rows, v_rows, offs, max_T, out=out_i, lse=lse_i,
@@ -273,7 +298,7 @@ def run_ours(args, w, rank, world, dev):
                               prepared=prepared if prep is None else prep)
 
     def step(i, events=None):
-        attend(kcs[i % n_copies], vcs[i % n_copies], q, out, lse, events)
+        attend(kcs[i % n_copies], vcs[i % n_copies], q, out, lse, events, i=i)
 
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(K)]
@@ -332,7 +357,7 @@ def run_ours(args, w, rank, world, dev):
         g2 = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g2, stream=stream):
             for i in range(K):
-                attend(kcs[i % n_copies], vcs[i % n_copies], q, out, lse, prep=False)
+                attend(kcs[i % n_copies], vcs[i % n_copies], q, out, lse, prep=False, i=i)
         with torch.cuda.stream(stream):
             g2.replay()
             torch.cuda.synchronize(dev)
@@ -376,10 +401,13 @@ def run_ours(args, w, rank, world, dev):
         kname, launches_per_step = "dense_decode_kernel", 4   # decompress prep, decompress, dense, merge
         alg_bytes = 2 * k_rows.numel() * k_rows.element_size()
     else:
-        kname, launches_per_step = main_kernel(api, cfg, args.algo)
+        if binv:   # scores, bit accumulation, split merge, contraction with C
+            kname, launches_per_step = "attend_scores_kernel+binv_*", 4
+        else:
+            kname, launches_per_step = main_kernel(api, cfg, args.algo)
         if not prepared and kname.startswith("attend_scores"):
             launches_per_step += 1   # the prep kernel
-        alg_bytes = code_bytes
+        alg_bytes = code_bytes + (vcb.numel() * vcb.element_size() if binv else 0)
     achieved = alg_bytes / (kern_ms / 1e3) / 1e9
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
@@ -388,12 +416,15 @@ def run_ours(args, w, rank, world, dev):
         "config": {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
                    "d": w.d, "T": total_T, "R": w.R, "g": w.g, "n_codes": w.n_codes,
                    "q_dtype": w.q_dtype, "parallelism": f"replicas{world}",
+                   **({"values": f"binary code, {w.v_bits} bits per position over the KV row, "
+                                 f"C [{w.v_bits}, {w.kv_heads * w.d}] fp32"} if binv else {}),
                    "path": args.path, "algo": args.algo, "splits": args.splits,
-                   "l2_defence": f"rotating {n_copies} cache copies ({n_copies * code_bytes / 2**20:.0f} MiB "
+                   "l2_defence": f"rotating {n_copies} cache copies{' and C' if binv else ''} "
+                                 f"({n_copies * code_bytes / 2**20:.0f} MiB of codes "
                                  f">= 3x L2 {l2 / 2**20:.0f} MiB)",
                    "timing": "K steps in one CUDA graph, CUDA events on the launch stream; main-kernel "
                              "times from the same K steps launched directly, events recorded by the "
-                             "library around its main kernels",
+                             "library around its main kernels" + (" (here: around the whole call)" if binv else ""),
                    "codebook_state": ("fp16 codebook images and RoPE tables prepared once per layer "
                                       "(commvq_attend_prepare), reused by every step") if prepared
                    else "rebuilt inside every step"},
@@ -423,6 +454,9 @@ def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, attend, stre
     kv_new = np.stack([synth.kv_rows(w, True, 1, sub=1000, dtype="f16"),
                        synth.kv_rows(w, False, 1, sub=1000, dtype="f16")])   # [2, 1, Hkv, d]
     kv_h = torch.from_numpy(kv_new).pin_memory()
+    binv = w.v_bits > 0
+    bits_h = torch.from_numpy(synth.value_bits(w, 1)).pin_memory() if binv else None
+    bits_d = torch.empty(bits_h.shape, dtype=torch.uint8, device=dev) if binv else None
     out_h = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32).pin_memory()
     q_d = torch.empty(q_h.shape, dtype=q_h.dtype, device=dev)
     kv_d = torch.empty(kv_h.shape, dtype=kv_h.dtype, device=dev)
@@ -435,8 +469,12 @@ def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, attend, stre
         q_d.copy_(q_h, non_blocking=True)
         kv_d.copy_(kv_h, non_blocking=True)
         api.encode(cfg, kv_d[0], kcb, codes=kc[last:last + 1], stream=stream)
-        api.encode(cfg, kv_d[1], vcb, codes=vc[last:last + 1], stream=stream)
-        attend(kc, vc, qv, out_d, None)
+        if binv:   # the value encoder is a learned network: its bits arrive from the host
+            bits_d.copy_(bits_h, non_blocking=True)
+            vc[last:last + 1].copy_(bits_d, non_blocking=True)
+        else:
+            api.encode(cfg, kv_d[1], vcb, codes=vc[last:last + 1], stream=stream)
+        attend(kc, vc, qv, out_d, None, i=i)
         out_h.copy_(out_d, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -460,7 +498,8 @@ def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, attend, stre
     ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     del graph
     return {"value": job_throughput(world, K, total_T, ms), "unit": UNIT,
-            "h2d_bytes_per_step": int(q_h.numel() * q_h.element_size() + kv_h.numel() * kv_h.element_size()),
+            "h2d_bytes_per_step": int(q_h.numel() * q_h.element_size() + kv_h.numel() * kv_h.element_size()
+                                      + (bits_h.numel() if binv else 0)),
             "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()),
             "ms_per_step": ms / K,
             "note": "q + new position's K/V rows in, encode + attend, output out; one CUDA graph of K steps"}
@@ -578,9 +617,13 @@ def oracle_sample(w, n_heads):
     T = int(w.lengths()[0])
     ws = w.with_(kv_heads=n_kv, q_heads=n_heads, batch=1, ragged=None, seq_len=T)
     kc = synth.uniform_codes(ws, True, T)
-    vc = synth.uniform_codes(ws, False, T)
     kcb = synth.normal_codebook(w, True)
-    vcb = synth.normal_codebook(w, False)
+    if w.v_bits:   # binary values: the bits of the whole KV row, C's columns of the sampled heads
+        vc = synth.value_bits(w, T)
+        vcb = np.ascontiguousarray(synth.binary_value_codebook(w)[:, :n_kv * w.d])
+    else:
+        vc = synth.uniform_codes(ws, False, T)
+        vcb = synth.normal_codebook(w, False)
     q = synth.as_f32(synth.queries(w), w.q_dtype)[:1, :n_heads].astype(np.float64)
     return q, kc, vc, np.array([0, T]), kcb, vcb, n_heads, T
 
@@ -589,7 +632,10 @@ def time_oracle_step(w, sample):
     from oracle import oracle as O
     q, kc, vc, offs, kcb, vcb, n_heads, T = sample
     t0 = time.perf_counter()
-    O.attend_codes(q, kc, vc, offs, kcb, vcb, w.rope_base)
+    if w.v_bits:
+        O.attend_binv(q, kc, vc, offs, kcb, vcb, w.rope_base)
+    else:
+        O.attend_codes(q, kc, vc, offs, kcb, vcb, w.rope_base)
     dt = time.perf_counter() - t0
     tokens = T * n_heads / w.q_heads        # context tokens of the full step this sample covers
     return dt, tokens

@@ -26,6 +26,7 @@ EXPORTS = ("commvq_encode", "commvq_attend_workspace_bytes", "commvq_attend_deco
            "commvq_attend_decode_noalloc", "commvq_em_workspace_bytes", "commvq_em_step",
            "commvq_em_step_soft", "commvq_decompress_workspace_bytes", "commvq_decompress",
            "commvq_dense_decode_workspace_bytes", "commvq_dense_decode",
+           "commvq_attend_binv_workspace_bytes", "commvq_attend_decode_binv",
            "commvq_workspace_error", "commvq_status_string", "commvq_abi_version")
 
 
@@ -80,6 +81,10 @@ def _load():
     lib.commvq_dense_decode_workspace_bytes.restype = SZ
     lib.commvq_dense_decode.argtypes = [CP, P, I32, P, P, I32, P, I32, I64, P, P, P, SZ, OP, P]
     lib.commvq_dense_decode.restype = I32
+    lib.commvq_attend_binv_workspace_bytes.argtypes = [CP, I32, I32, I64]
+    lib.commvq_attend_binv_workspace_bytes.restype = SZ
+    lib.commvq_attend_decode_binv.argtypes = [CP, P, I32, P, P, I32, P, I32, I64, P, P, P, P, P, SZ, I32, P]
+    lib.commvq_attend_decode_binv.restype = I32
     lib.commvq_workspace_error.argtypes = [P, ctypes.POINTER(I32), P]
     lib.commvq_workspace_error.restype = I32
     lib.commvq_status_string.argtypes = [I32]
@@ -328,6 +333,41 @@ def dense_decode(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                    _ptr(seq_offsets), int(B), int(max_T), _ptr(out), _ptr(lse),
                                    _ptr(workspace), workspace.numel(), ctypes.byref(o), _stream(stream)),
            "commvq_dense_decode")
+    return out, lse
+
+
+def attend_binv_workspace_bytes(cfg: Config, n_bits: int, B: int, max_T: int) -> int:
+    cc = cfg.c()
+    return int(LIB.commvq_attend_binv_workspace_bytes(ctypes.byref(cc), int(n_bits), int(B), int(max_T)))
+
+
+def attend_decode_binv(cfg: Config, q: torch.Tensor, k_codes: torch.Tensor, v_bits: torch.Tensor,
+                       seq_offsets: torch.Tensor, max_T: int, k_codebook: torch.Tensor, v_codebook: torch.Tensor,
+                       out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, want_lse: bool = True, prepared: bool = False,
+                       stream=None):
+    """commvq_attend_decode_binv: CommVQ keys, binary values v_bits [total_T, n_bits/8] uint8
+    with codebook C [n_bits, kv_heads * d]. prepared: the workspace holds the key side's state
+    from an earlier call with the same cfg, B, max_T and key codebook. Returns (out, lse)."""
+    if prepared and workspace is None:
+        raise ValueError("prepared=True needs the workspace of an earlier call")
+    B = q.shape[0]
+    n_bits = v_codebook.shape[0]
+    if out is None:
+        out = torch.empty((B, cfg.q_heads, cfg.d), dtype=torch.float32, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, cfg.q_heads), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = attend_binv_workspace_bytes(cfg, n_bits, B, max_T)
+        if n == 0:
+            raise CommVQError(2, "commvq_attend_binv_workspace_bytes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    cc = cfg.c()
+    _check(LIB.commvq_attend_decode_binv(ctypes.byref(cc), _ptr(q), _DT[q.dtype], _ptr(k_codes), _ptr(v_bits),
+                                         int(n_bits), _ptr(seq_offsets), int(B), int(max_T), _ptr(k_codebook),
+                                         _ptr(v_codebook), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                         ATTEND_PREPARED if prepared else 0, _stream(stream)),
+           "commvq_attend_decode_binv")
     return out, lse
 
 

@@ -376,6 +376,41 @@ extern "C" commvq_status commvq_attend_prepare(const commvq_config* cfg, int32_t
 }
 
 namespace commvq {
+int mma_splits(int B, int q_heads, int64_t max_T) {
+  commvq_attend_options o{COMMVQ_ATTN_DECODE_MMA, 0, nullptr, nullptr, 0};
+  return choose_splits(COMMVQ_ATTN_DECODE_MMA, B, q_heads, max_T, &o);
+}
+
+int attend_mma_setup(const commvq_config* cfg, int B, int64_t max_T, unsigned char* ws,
+                     const int64_t* seq_offsets, const void* k_codes, const float* k_codebook, AttendArgs& a) {
+  commvq_attend_options o{COMMVQ_ATTN_DECODE_MMA, 0, nullptr, nullptr, 0};
+  const int S = choose_splits(COMMVQ_ATTN_DECODE_MMA, B, cfg->q_heads, max_T, &o);
+  const WorkspaceLayout L = workspace_layout(cfg, COMMVQ_ATTN_DECODE_MMA, B, max_T, S);
+  a.k_codes = static_cast<const uint8_t*>(k_codes);
+  a.v_codes = static_cast<const uint8_t*>(k_codes);
+  a.seq_offsets = seq_offsets;
+  a.k_codebook = k_codebook;
+  a.v_codebook = k_codebook;
+  a.error_word = reinterpret_cast<int*>(ws);
+  a.partials = reinterpret_cast<Partial*>(ws + L.partials_off);
+  a.k_img = reinterpret_cast<const uint4*>(ws + L.kimg_off);
+  a.v_img = reinterpret_cast<const uint4*>(ws + L.vimg_off);
+  a.scores = reinterpret_cast<float*>(ws + L.scores_off);
+  a.theta = reinterpret_cast<const double*>(ws + L.phase_off);
+  a.rowph = reinterpret_cast<const float4*>(ws + L.phase_off + 64 * sizeof(double));
+  a.advph = a.rowph + 128 * 32;
+  a.max_T = max_T;
+  a.rope_base = cfg->rope_base;
+  a.B = B;
+  a.q_heads = cfg->q_heads;
+  a.kv_heads = cfg->kv_heads;
+  a.R = cfg->R;
+  a.n_codes = cfg->n_codes;
+  return S;
+}
+}  // namespace commvq
+
+namespace commvq {
 commvq_status launch_combine(const AttendArgs& a, int S, cudaStream_t st) {
   if (launch_dependent(combine_kernel, dim3(a.B * a.q_heads, kCombineQuarters), dim3(kCombineThreads), 0, st, a,
                        S) != cudaSuccess)

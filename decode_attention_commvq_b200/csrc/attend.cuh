@@ -51,6 +51,21 @@ bool mma_supported(int R, int q_heads, int kv_heads, int n_codes);
 commvq_status launch_attend_prep(const AttendArgs& a, cudaStream_t st);
 commvq_status launch_attend_mma(const AttendArgs& a, const void* q, commvq_dtype qt, int splits,
                                 cudaStream_t st);
+// Position splits of the decode-and-rotate scores kernel for this batch (the count
+// attend_mma_setup returns).
+int mma_splits(int B, int q_heads, int64_t max_T);
+// AttendArgs for the decode-and-rotate key side in an attention workspace laid out for
+// (cfg, B, max_T) with the DECODE_MMA algorithm; returns the split count.
+int attend_mma_setup(const commvq_config* cfg, int B, int64_t max_T, unsigned char* ws,
+                     const int64_t* seq_offsets, const void* k_codes, const float* k_codebook, AttendArgs& a);
+// The scores kernel alone (maxima in the partials' m, exp2-domain scores in a.scores).
+commvq_status launch_attend_scores(const AttendArgs& a, const void* q, commvq_dtype qt, int splits,
+                                   cudaStream_t st);
+// The score buffer's slot of (sequence b, position t, KV head kv, head column col).
+__host__ __device__ inline int64_t score_slot(int64_t b, int64_t t, int kv, int col, int64_t n_tiles, int KV, int G) {
+  const int tau = static_cast<int>(t % 16);
+  return ((((b * n_tiles + t / 16) * KV + kv) * G + col) * 4 + ((tau & 7) >> 1)) * 4 + (tau & 1) + 2 * (tau >> 3);
+}
 commvq_status launch_attend_table(const AttendArgs& a, const void* q, commvq_dtype qt, int splits,
                                   cudaStream_t st);
 commvq_status launch_combine(const AttendArgs& a, int splits, cudaStream_t st);

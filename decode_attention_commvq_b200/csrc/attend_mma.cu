@@ -694,7 +694,8 @@ attend_values_kernel(AttendArgs a) {
 }
 
 template <int R, int KV, int NC>
-commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt, int S, cudaStream_t st) {
+commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt, int S, cudaStream_t st,
+                            bool with_values) {
   const size_t smem_s = mma_scores_smem_bytes(R, KV, a.n_codes);
   const size_t smem_v = mma_values_smem_bytes(R, KV, a.q_heads, a.n_codes);
   dim3 grid(S, a.B);
@@ -715,6 +716,7 @@ commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt,
     default: return COMMVQ_ERR_UNSUPPORTED;
   }
 #undef COMMVQ_LAUNCH_SCORES
+  if (!with_values) return launch_status();
   {
     auto k = attend_values_kernel<R, KV, NC>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_v) != cudaSuccess)
@@ -728,18 +730,20 @@ commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt,
 }
 
 template <int R, int KV>
-commvq_status launch_mma_r(const AttendArgs& a, const void* q, commvq_dtype qt, int S, cudaStream_t st) {
-  if (a.n_codes == 256) return launch_mma_rk<R, KV, 256>(a, q, qt, S, st);
-  return launch_mma_rk<R, KV, 0>(a, q, qt, S, st);
+commvq_status launch_mma_r(const AttendArgs& a, const void* q, commvq_dtype qt, int S, cudaStream_t st,
+                           bool with_values) {
+  if (a.n_codes == 256) return launch_mma_rk<R, KV, 256>(a, q, qt, S, st, with_values);
+  return launch_mma_rk<R, KV, 0>(a, q, qt, S, st, with_values);
 }
 
 template <int R>
-commvq_status launch_mma_kv(const AttendArgs& a, const void* q, commvq_dtype qt, int S, cudaStream_t st) {
+commvq_status launch_mma_kv(const AttendArgs& a, const void* q, commvq_dtype qt, int S, cudaStream_t st,
+                            bool with_values) {
   switch (a.kv_heads) {
-    case 1: return launch_mma_r<R, 1>(a, q, qt, S, st);
-    case 2: return launch_mma_r<R, 2>(a, q, qt, S, st);
-    case 4: return launch_mma_r<R, 4>(a, q, qt, S, st);
-    case 8: return launch_mma_r<R, 8>(a, q, qt, S, st);
+    case 1: return launch_mma_r<R, 1>(a, q, qt, S, st, with_values);
+    case 2: return launch_mma_r<R, 2>(a, q, qt, S, st, with_values);
+    case 4: return launch_mma_r<R, 4>(a, q, qt, S, st, with_values);
+    case 8: return launch_mma_r<R, 8>(a, q, qt, S, st, with_values);
     default: return COMMVQ_ERR_UNSUPPORTED;
   }
 }
@@ -779,8 +783,14 @@ commvq_status launch_attend_prep(const AttendArgs& a, cudaStream_t st) {
 }
 
 commvq_status launch_attend_mma(const AttendArgs& a, const void* q, commvq_dtype qt, int S, cudaStream_t st) {
-  if (a.R == 1) return launch_mma_kv<1>(a, q, qt, S, st);
-  if (a.R == 2) return launch_mma_kv<2>(a, q, qt, S, st);
+  if (a.R == 1) return launch_mma_kv<1>(a, q, qt, S, st, true);
+  if (a.R == 2) return launch_mma_kv<2>(a, q, qt, S, st, true);
+  return COMMVQ_ERR_UNSUPPORTED;
+}
+
+commvq_status launch_attend_scores(const AttendArgs& a, const void* q, commvq_dtype qt, int S, cudaStream_t st) {
+  if (a.R == 1) return launch_mma_kv<1>(a, q, qt, S, st, false);
+  if (a.R == 2) return launch_mma_kv<2>(a, q, qt, S, st, false);
   return COMMVQ_ERR_UNSUPPORTED;
 }
 

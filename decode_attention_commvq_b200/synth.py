@@ -69,6 +69,7 @@ class Workload:
     em_iters: int = 5                  # per round
     encode_tokens: int = 0             # >0: encode-only workload (tokens x kv_heads rows)
     fit_seed: Optional[int] = None     # seed of the codebook fit and outlier channels
+    v_bits: int = 0                    # > 0: values in the binary code with this many rows
 
     @property
     def cb_seed(self) -> int:
@@ -99,7 +100,8 @@ class Workload:
 
 
 # The workloads, in order: tiny fp32 case, 2-bit 32K layer, 1-bit 128K layer, ragged batch of
-# 16, the encode + codebook-fit workload, and the pages' own g = 64 setting at 2 and 1 bits.
+# 16, the encode + codebook-fit workload, the pages' own g = 64 setting at 2 and 1 bits, and
+# the binary value code.
 WORKLOADS = [
     Workload(name="tiny_fp32_T256_R1_N16", seed=0, R=1, n_codes=16, q_heads=1, kv_heads=1,
              rope_base=10000.0, seq_len=256, kv_dtype="f32", q_dtype="f32", n_outliers=0,
@@ -114,6 +116,9 @@ WORKLOADS = [
     # (1-bit) residual rounds: R * log2(64) / 64 = 1.97 and 1.03 bits per scalar
     Workload(name="pages_g64_2bit_T32768", seed=5, g=64, R=21, n_codes=64, seq_len=32768),
     Workload(name="pages_g64_1bit_T32768", seed=6, fit_seed=5, g=64, R=11, n_codes=64, seq_len=32768),
+    # the pages' binary value code (2048 rows over the 1024-dim KV row: 2 bits per scalar) with
+    # the 2-bit layer's keys
+    Workload(name="llama8b_binv2048_T32768", seed=7, fit_seed=1, R=2, seq_len=32768, v_bits=2048),
 ]
 # The 1-bit layer and the ragged batch take their codebooks (and outlier channels) from
 # the 2-bit layer's fit seed: under sequential residual fitting the R=1 codebook is
@@ -236,3 +241,15 @@ def uniform_codes(w: Workload, key: bool, total_T: int) -> np.ndarray:
     stream = STREAM_KCODES if key else STREAM_VCODES
     c = rng(w.seed, stream, 0).integers(0, w.n_codes, size=(total_T, w.kv_heads, w.R, w.groups))
     return c.astype(np.uint8 if w.code_bytes == 1 else np.uint16)
+
+
+def value_bits(w: Workload, total_T: int) -> np.ndarray:
+    """[total_T, v_bits / 8] uint8 binary value codes, every bit uniform (stream 8, sub 1)."""
+    return rng(w.seed, STREAM_VCODES, 1).integers(0, 256, size=(total_T, w.v_bits // 8), dtype=np.uint8)
+
+
+def binary_value_codebook(w: Workload) -> np.ndarray:
+    """C [v_bits, kv_heads * d] float32, entries N(0, 2 / v_bits): with half the bits set a decoded
+    value row is ~N(0, 1) per scalar (stream 0, sub 4)."""
+    x = rng(w.cb_seed, STREAM_CODEBOOK, 4).standard_normal((w.v_bits, w.kv_heads * w.d))
+    return (x * np.sqrt(2.0 / w.v_bits)).astype(np.float32)

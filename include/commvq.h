@@ -252,6 +252,41 @@ commvq_status commvq_em_step_soft(const commvq_config* cfg, const float* rows, i
                                   float* codebook_round, float tau, double* sse_out,
                                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Binary value code -------------------------------------------------------------------
+ * The paper's value encoding (review, "Assumptions & free parameters"): one bit vector
+ * s_t in {0,1}^n_bits per position over the whole KV dimension (kv_heads * 128 scalars), decoded
+ * as v_t = sum_n s_{t,n} C[n, :]; n_bits / (kv_heads * 128) bits per scalar (1024 -> 1 bit,
+ * 2048 -> 2 bits at 8 KV heads). Keys keep the additive RoPE-commutative code of cfg.
+ */
+
+/* Bytes of device workspace commvq_attend_decode_binv needs. 0 for invalid or unsupported
+ * input. */
+size_t commvq_attend_binv_workspace_bytes(const commvq_config* cfg, int32_t n_bits, int32_t B, int64_t max_T);
+
+/* Decode attention with CommVQ keys and binary values:
+ *   s_t (keys) as in commvq_attend_decode, p = softmax(s),
+ *   out[b,h] = sum_t p_t (s_t^T C)[kvh * 128 : kvh * 128 + 128], kvh = h / (q_heads / kv_heads),
+ *   lse as in commvq_attend_decode.
+ * The softmax weights are folded into the bits first (H_h = sum_t p_t s_t on the tensor cores,
+ * bits expanded to fp16 0 / 1), then H_h is contracted with C in fp32.
+ * v_bits      [total_T, n_bits / 8] uint8, bit n of position t = byte n/8, bit n%8 (least
+ *             significant first), 16-byte aligned.
+ * v_codebook  C [n_bits, kv_heads * 128] float32.
+ * Other arguments as commvq_attend_decode (q, k_codes, seq_offsets, B, max_T, k_codebook, out,
+ * lse, workspace of commvq_attend_binv_workspace_bytes bytes).
+ * Supports the DECODE_MMA key shapes (g = 8, R <= 2, Nc' <= 256, kv_heads in {1, 2, 4, 8}),
+ * q_heads <= 32, n_bits a multiple of 1024 up to 8192.
+ * flags: COMMVQ_ATTEND_PREPARED when this workspace already holds the key side's codebook images
+ * and RoPE tables from an earlier call with the same cfg, B, max_T and k_codebook (the first call
+ * on a workspace passes 0). Codes out of range are clamped and reported as by
+ * commvq_attend_decode (commvq_workspace_error on this workspace). */
+commvq_status commvq_attend_decode_binv(const commvq_config* cfg, const void* q, commvq_dtype q_dtype,
+                                        const void* k_codes, const uint8_t* v_bits, int32_t n_bits,
+                                        const int64_t* seq_offsets, int32_t B, int64_t max_T,
+                                        const float* k_codebook, const float* v_codebook, float* out,
+                                        float* lse, void* workspace, size_t workspace_bytes, int32_t flags,
+                                        void* stream);
+
 /* ---- Decompress-then-attend comparator ----------------------------------------------------
  * The review compares CommVQ's decode latency with a "naive implementation of the same
  * quantization" ("What carries the argument", Table 5: 6x-9.6x lower latency). These two calls

@@ -276,6 +276,26 @@ int oracle_attend(const double* q, const double* khat, const double* vhat, const
   return ORACLE_OK;
 }
 
+/* The paper's binary value code (review, "Assumptions & free parameters": value codebook of
+ * Nc rows over the whole KV dimension, Nc/d bits per scalar): position t stores bits
+ * s_t in {0,1}^Nc and decodes to v_t = sum_n s_{t,n} C[n, :], the row of all KV heads.
+ * bits [T, Nc/8] uint8, bit n of a row = byte n/8, bit n%8 (little-endian);
+ * C [Nc, dkv] fp32; out [T, dkv] fp64. Sums in fp64 in index order. */
+int oracle_decode_bits(const uint8_t* bits, int64_t T, int Nc, const float* C, int dkv, double* out) {
+  if (T < 0 || Nc <= 0 || (Nc % 8) || dkv <= 0 || (T > 0 && (!bits || !C || !out))) return ORACLE_BAD_ARG;
+  for (int64_t t = 0; t < T; ++t) {
+    double* o = out + t * dkv;
+    for (int i = 0; i < dkv; ++i) o[i] = 0.0;
+    const uint8_t* row = bits + t * (Nc / 8);
+    for (int n = 0; n < Nc; ++n) {
+      if (!((row[n >> 3] >> (n & 7)) & 1)) continue;
+      const float* c = C + (int64_t)n * dkv;
+      for (int i = 0; i < dkv; ++i) o[i] += (double)c[i];
+    }
+  }
+  return ORACLE_OK;
+}
+
 /* Dense decode attention over keys that already carry their rotation (the second half of a
  * decompress-then-attend implementation): s_t = q . k_t / sqrt(d), out = softmax(s) . v,
  * lse = log sum e^{s_t}; shapes, GQA mapping, offsets and the empty case as oracle_attend. */

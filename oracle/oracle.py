@@ -50,9 +50,10 @@ def lib():
         _lib.oracle_em_soft_step.argtypes = [P, I64, I, I, I, P, ctypes.c_double, P]
         _lib.oracle_rope.argtypes = [P, P, I64, I, ctypes.c_double, P]
         _lib.oracle_attend_dense.argtypes = [P, P, P, P, I, I, I, I, P, P]
+        _lib.oracle_decode_bits.argtypes = [P, I64, I, P, I, P]
         for f in ("oracle_encode", "oracle_decode", "oracle_scores_plain", "oracle_scores_table",
                   "oracle_attend", "oracle_em_step", "oracle_values_hist", "oracle_em_soft_step",
-                  "oracle_rope", "oracle_attend_dense"):
+                  "oracle_rope", "oracle_attend_dense", "oracle_decode_bits"):
             getattr(_lib, f).restype = ctypes.c_int
     return _lib
 
@@ -197,6 +198,27 @@ def attend_dense(q: np.ndarray, k: np.ndarray, v: np.ndarray, offsets: np.ndarra
                                      _p(_c(offsets, np.int64)), B, Hq, Hkv, d, _p(out), _p(lse)),
            "attend_dense")
     return out, lse
+
+
+def decode_bits(bits: np.ndarray, C: np.ndarray) -> np.ndarray:
+    """The binary value code: bits [T, Nc/8] uint8 (bit n = byte n/8, bit n%8) and value codebook
+    C [Nc, dkv] -> rows [T, dkv] fp64, the sum of the rows of C whose bit is set."""
+    Nc, dkv = C.shape
+    b = _c(bits, np.uint8)
+    T = b.shape[0]
+    out = np.empty((T, dkv), dtype=np.float64)
+    _check(lib().oracle_decode_bits(_p(b), T, Nc, _p(_c(C, np.float32)), dkv, _p(out)), "decode_bits")
+    return out
+
+
+def attend_binv(q: np.ndarray, k_codes: np.ndarray, v_bits: np.ndarray, offsets: np.ndarray,
+                kcb: np.ndarray, C: np.ndarray, base: float):
+    """Decode attention with CommVQ keys (codes [sum T, Hkv, R, d/g]) and binary values
+    (bits [sum T, Nc/8] over all Hkv*d value dims): decode both, then attend."""
+    Hkv = k_codes.shape[1]
+    d = q.shape[-1]
+    vhat = decode_bits(v_bits, C).reshape(-1, Hkv, d)
+    return attend(q, decode(k_codes, kcb), vhat, offsets, base)
 
 
 def attend_codes(q: np.ndarray, k_codes: np.ndarray, v_codes: np.ndarray, offsets: np.ndarray,

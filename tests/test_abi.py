@@ -222,3 +222,37 @@ def test_generic_algo_workspace(api):
     assert api.attend_workspace_bytes(cfg, 1, 32768, splits=4, algo=api.ATTN_GENERIC) == n
     assert api.attend_workspace_bytes(cfg, 1, 32768, algo=api.ATTN_DECODE_MMA) == 0
     assert api.attend_workspace_bytes(_cfg(api, g=64, n_codes=64, R=21, q_heads=64, kv_heads=2), 1, 10) == 0
+
+
+def _binv(api, cfg, n_bits=2048, B=1, max_T=100, q=FAKE, qdt=2, kc=FAKE, bits=FAKE, offs=FAKE, kcb=FAKE,
+          C=FAKE, out=FAKE, ws=FAKE, ws_bytes=1 << 28, flags=0):
+    cc = cfg.c()
+    P = ctypes.c_void_p
+    return api.LIB.commvq_attend_decode_binv(ctypes.byref(cc), P(q), qdt, P(kc), P(bits), n_bits, P(offs), B,
+                                             max_T, P(kcb), P(C), P(out), None, P(ws), ws_bytes, flags, None)
+
+
+def test_binary_value_code_rejects_bad_arguments(api):
+    INVALID, UNSUP, WS = 1, 2, 4
+    cfg = _cfg(api)
+    assert _binv(api, cfg, B=0) == 0
+    assert _binv(api, cfg, n_bits=1000) == UNSUP                     # not a multiple of 1024
+    assert _binv(api, cfg, n_bits=9216) == UNSUP                     # above 8192
+    assert _binv(api, cfg, n_bits=0) == INVALID
+    assert _binv(api, _cfg(api, R=3)) == UNSUP                       # keys off the decode-and-rotate shape
+    assert _binv(api, _cfg(api, q_heads=64, kv_heads=8)) == UNSUP    # more than 32 query heads
+    assert _binv(api, cfg, qdt=7) == INVALID
+    assert _binv(api, cfg, bits=0) == INVALID
+    assert _binv(api, cfg, C=FAKE + 4) == INVALID                    # misaligned codebook
+    assert _binv(api, cfg, max_T=-1) == INVALID
+    assert _binv(api, cfg, ws_bytes=4096) == WS
+
+
+def test_binary_value_code_workspace_holds_the_key_side_and_the_sums(api):
+    """At least the decode-and-rotate workspace plus one split's H [Hq, n_bits] fp32 (the split
+    count falls as the bit count grows, so the size need not grow with the bits)."""
+    cfg = _cfg(api)
+    base = api.attend_workspace_bytes(cfg, 1, 32768, algo=api.ATTN_DECODE_MMA)
+    for n_bits in (1024, 2048, 8192):
+        assert api.attend_binv_workspace_bytes(cfg, n_bits, 1, 32768) >= base + 32 * n_bits * 4
+    assert api.attend_binv_workspace_bytes(cfg, 2048, -1, 10) == 0

@@ -549,3 +549,38 @@ def test_attend_dense_equals_rotating_attend_and_sdpa():
     Q = torch.from_numpy(q[2])[None, :, None, :]
     sd = torch.nn.functional.scaled_dot_product_attention(Q, K, V)[0, :, 0].numpy()
     assert np.abs(out[2] - sd).max() <= 1e-12 * np.abs(sd).max()
+
+
+# ----------------------------------------------------------------------------------------
+# binary value code (the paper's value encoding): s_t in {0,1}^Nc, v_t = s_t^T C
+
+def test_decode_bits_equals_matrix_product_and_bit_order():
+    """Against numpy's unpacked bits times C (a library product), and single set bits pick
+    single rows: byte n/8, bit n%8, least significant first."""
+    rng = np.random.default_rng(71)
+    Nc, dkv, T = 64, 24, 9
+    C = rng.standard_normal((Nc, dkv)).astype(np.float32)
+    bits = rng.integers(0, 256, size=(T, Nc // 8), dtype=np.uint8)
+    S = np.unpackbits(bits, axis=1, bitorder="little").astype(np.float64)
+    assert np.abs(O.decode_bits(bits, C) - S @ C.astype(np.float64)).max() <= 1e-12
+    one = np.zeros((1, Nc // 8), dtype=np.uint8)
+    one[0, 5] = 1 << 3                                   # bit 43
+    assert np.array_equal(O.decode_bits(one, C)[0], C[43].astype(np.float64))
+    assert np.all(O.decode_bits(np.zeros((2, Nc // 8), np.uint8), C) == 0)
+
+
+def test_attend_binv_is_attention_on_decoded_values():
+    rng = np.random.default_rng(72)
+    Hq, Hkv, d, R, G, Nc = 8, 2, 128, 2, 16, 256
+    offs = np.array([0, 40, 97])
+    kcb = rng.standard_normal((R, G, 16, 8)).astype(np.float32)
+    C = (rng.standard_normal((Nc, Hkv * d)) / 8).astype(np.float32)
+    kc = rng.integers(0, 16, size=(97, Hkv, R, G))
+    vb = rng.integers(0, 256, size=(97, Nc // 8), dtype=np.uint8)
+    q = rng.standard_normal((2, Hq, d))
+    out, lse = O.attend_binv(q, kc, vb, offs, kcb, C, 1e4)
+    S = np.unpackbits(vb, axis=1, bitorder="little").astype(np.float64)
+    vhat = (S @ C.astype(np.float64)).reshape(97, Hkv, d)
+    ref, ref_lse = O.attend(q, O.decode(kc, kcb), vhat, offs, 1e4)
+    assert np.abs(out - ref).max() <= 1e-12 * np.abs(ref).max()
+    assert np.allclose(lse, ref_lse, rtol=0, atol=1e-12)
