@@ -7,12 +7,13 @@
 // Because v_t is linear in s_t, the softmax weights can be folded into the bits first:
 //   out_h = (sum_t p_{h,t} s_t) C[:, slice of h's KV head] / sum_t p_{h,t}.
 // Kernel 1 (grid: position splits x 256-bit slices x sequences) forms the per-split sums
-// H_v[h, n] = sum_t 2^(score - m_v) s_t[n] on the tensor cores: A = the weights of all query heads
-// (rows) for 16 positions (k), B = the 16 positions' bits for 8 codebook rows (n), expanded to
-// fp16 0 / 1 in registers. A split is a run of whole splits of the scores kernel, so its maximum
-// m_v is the maximum of their maxima and every weight is at most 1. Kernel 2 (grid: KV heads x
-// 128-row chunks of C) merges the splits' H with log-sum-exp weights and contracts its chunk with
-// C; kernel 3 sums the chunks and divides by the softmax sum.
+// H_v[h, n] = sum_t 2^(score - m_v) s_t[n] with tcgen05 MMAs, as H_v^T = S^T P^T: A = the bits of
+// 128 codebook rows (M) for 16 positions (K), expanded to fp16 0 / 1 and stored into tensor memory;
+// B = the weights of all 32 query-head columns (N) in shared memory; D accumulates in tensor
+// memory. A split is a run of whole splits of the scores kernel, so its maximum m_v is the maximum
+// of their maxima and every weight is at most 1. Kernel 2 (grid: KV heads x 128-row chunks of C)
+// merges the splits' H with log-sum-exp weights and contracts its chunk with C; kernel 3 sums the
+// chunks and divides by the softmax sum.
 #include <math.h>
 
 #include "attend.cuh"
@@ -20,20 +21,15 @@
 namespace commvq {
 namespace {
 
-constexpr int kBvThreads = 512;   // 16 warps: 4 bit groups x 4 position groups
-constexpr int kBvBitGroups = 4;
-constexpr int kBvPosGroups = 4;
-constexpr int kBvBitsPerWarp = 64;
-constexpr int kBvBitsPerCta = kBvBitGroups * kBvBitsPerWarp;   // 256
+constexpr int kBvThreads = 512;   // 16 warps
+constexpr int kBvPosGroups = 4;   // 16-position MMA steps per chunk
+constexpr int kBvBitsPerCta = 256;                              // two M = 128 halves
 constexpr int kBvSliceBytes = kBvBitsPerCta / 8;                // 32
-constexpr int kBvRowBytes = 48;   // padded: the 4 rows a warp reads at once hit distinct banks
 constexpr int kBvMaxHeads = 32;
-constexpr int kBvTile = 16;       // positions per mma k-step (one tile of the scores buffer)
+constexpr int kBvTile = 16;       // positions per MMA K step (one tile of the scores buffer)
 constexpr int kBvChunk = kBvPosGroups * kBvTile;   // positions per pipeline step
 constexpr int kBvStages = 4;
-constexpr int kPStride = kBvChunk + 8;             // halves per weight row (144 B: conflict-free ldmatrix)
 constexpr int kBvMaxSplits = 64;
-constexpr int kHRed = kBvBitsPerWarp + 8;          // floats per head row of the reduction buffer
 constexpr int kBvCRows = 128;                      // rows of C per merge-and-contract CTA
 constexpr int kBvMaxG = 8;
 
@@ -49,18 +45,11 @@ struct BinvArgs {
   float2* ml;                 // [B][Hq] (M, L)
   float* out;
   float* lse;
+  int* error_word;
   int64_t max_T, n_tiles;
   int B, Hq, KV, Nc, S, K, Sv;   // S scores splits, K of them per value split, Sv value splits
 };
 
-struct BvStage {
-  uint8_t bits[kBvChunk][kBvRowBytes];
-  float sc[kBvPosGroups * kBvMaxHeads * kBvTile];   // 4 tiles' score blocks, head h of tile q at 16 (q Hq + h)
-};
-static_assert(sizeof(BvStage) % 16 == 0, "stage alignment");
-constexpr size_t kBvLoopSmem = kBvStages * sizeof(BvStage) + kBvMaxHeads * kPStride * 2 + kBvMaxHeads * 4;
-constexpr size_t kBvRedSmem = (kBvPosGroups - 1) * kBvBitGroups * kBvMaxHeads * kHRed * 4;
-constexpr size_t kBvAccSmem = kBvLoopSmem > kBvRedSmem ? kBvLoopSmem : kBvRedSmem;
 constexpr size_t kBvMcSmem = (kBvCRows * kD + kBvMaxG * kBvMaxSplits + 2 * kBvMaxG * kBvCRows) * 4;
 
 // Value split v of sequence b: scores splits vK .. vK + K - 1 (the same tile-aligned pieces of
@@ -82,40 +71,130 @@ __device__ __forceinline__ void cp_async16_z(void* smem_dst, const void* gmem_sr
                : "memory");
 }
 
-__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// fp16 pair (bit lo, bit hi) as 1.0 / 0.0 (0x3C00 is fp16 1.0)
-__device__ __forceinline__ uint32_t bits_to_h2(uint32_t lo, uint32_t hi) { return lo * 0x3C00u + hi * 0x3C000000u; }
-
 // Position tau of a 16-position tile sits at this offset of the head's 16 scores (the scores
 // kernel's fragment order).
 __device__ __forceinline__ int tile_slot(int tau) { return ((tau & 7) >> 1) * 4 + (tau & 1) + 2 * (tau >> 3); }
 
+// ---------------------------------------------------------------------------------------
+// tcgen05 pieces (PTX ISA 8.6, sm_100a): TMEM allocation, loads and stores, the f16 MMA with its
+// A operand in TMEM and B in shared memory, completion through an mbarrier.
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase of `parity` to complete, giving up after `limit` polls (each poll may
+// itself block for a while). Returns false when it gave up.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit) {
+  for (uint32_t n = 0; n < limit; ++n)
+    if (mbar_test(bar, parity)) return true;
+  return false;
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n" ::"r"(taddr),
+               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+// D[128 x N] (+)= A[128 x 16] (TMEM, fp16) * B[16 x N] (shared memory descriptor, fp16), fp32 D.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B fp16 (formats 0), both
+// K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+constexpr uint32_t kBvIdesc = (1u << 4) | ((32u >> 3) << 17) | ((128u >> 4) << 24);
+// Shared-memory descriptor of a K-major, unswizzled operand: 8-row x 16-byte core matrices,
+// LBO = byte step between the two 8-element K halves, SBO = byte step between 8-row groups,
+// version 1 at bits 46-47.
+__device__ __forceinline__ uint64_t smem_desc_k(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+constexpr int kBvCols = 256;       // TMEM columns: D (2 x 32), A (2 buffers x 2 halves x 32)
+constexpr int kBvColA = 64;
+constexpr uint32_t kBvWaitPolls = 1u << 20;
+// B operand of one buffer: 4 k-steps x [32 heads x 16 positions] fp16, K-major core matrices:
+// (head h, position k of the step) at ks 1024 + (h / 8) 256 + (k / 8) 128 + (h % 8) 16 + (k % 8) 2.
+constexpr int kBvBBytes = kBvPosGroups * kBvMaxHeads * kBvTile * 2;
+constexpr size_t kBvTcSmem = 2 * kBvBBytes + kBvStages * (kBvChunk * kBvSliceBytes + kBvPosGroups * kBvMaxHeads * kBvTile * 4) +
+                             kBvMaxHeads * 4 + 2 * 8 + 16;
+
+// H_v^T[n, h] = sum_t s_t[n] 2^(score_{h,t} - m_v) for the CTA's 256 codebook rows (two M = 128
+// halves) and all 32 head columns, on tcgen05: per 64-position chunk, 16 warps expand the bits to
+// fp16 0 / 1 straight into TMEM (A, one 32-lane quarter and one 16-position step per store), all
+// threads write the weights into shared memory (B), and one thread issues 8 MMAs (2 halves x 4
+// steps) and commits them to the buffer's mbarrier. Two A/B buffers: chunk c + 1 is built while
+// chunk c's MMAs run.
 __global__ void __launch_bounds__(kBvThreads, 1) binv_accumulate_kernel(BinvArgs a) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  BvStage* stage = reinterpret_cast<BvStage*>(smem);
-  __half(*ptile)[kPStride] = reinterpret_cast<__half(*)[kPStride]>(smem + kBvStages * sizeof(BvStage));
-  float* mrow = reinterpret_cast<float*>(smem + kBvStages * sizeof(BvStage) + kBvMaxHeads * kPStride * 2);
-  float* hred = reinterpret_cast<float*>(smem);   // after the loop: [pos group - 1][bit group][head][kHRed]
+  extern __shared__ __align__(1024) unsigned char smem[];
+  unsigned char* bbuf = smem;                                                  // [2][kBvBBytes]
+  unsigned char* stg = smem + 2 * kBvBBytes;                                   // [stages][bits | scores]
+  constexpr int kStgBits = kBvChunk * kBvSliceBytes;                           // 2048
+  constexpr int kStgBytes = kStgBits + kBvPosGroups * kBvMaxHeads * kBvTile * 4;
+  float* mrow = reinterpret_cast<float*>(stg + kBvStages * kStgBytes);
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(mrow + kBvMaxHeads);            // [2]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(mbar + 2);
+
   const int v = blockIdx.x, slice = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bg = warp & (kBvBitGroups - 1), pg = warp / kBvBitGroups;
-  const int g = lane >> 2, i = lane & 3;
   int64_t row0, t_begin, t_end;
   bv_split(a, b, v, row0, t_begin, t_end);
   const int64_t n_c = (t_end - t_begin + kBvChunk - 1) / kBvChunk;
   const uint8_t* bsrc = a.bits + row0 * (a.Nc / 8) + slice * kBvSliceBytes;
   const float* ssrc = a.scores + (static_cast<int64_t>(b) * a.n_tiles + t_begin / kBvTile) * a.Hq * kBvTile;
+
+  if (warp == 0) {   // TMEM for the accumulators and the A buffers (one CTA per SM)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tslot)),
+                 "r"(kBvCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  if (tid == 0) {
+    mbar_init(&mbar[0], 1);
+    mbar_init(&mbar[1], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
   pdl_wait();   // the scores kernel's buffer and maxima are complete from here on
 
-  // the split's maximum per head: the maxima of its K scores splits (16 lanes per head)
-  {
+  {   // the split's maximum per head: the maxima of its K scores splits (16 lanes per head)
     const int h = tid >> 4, l = tid & 15;
     float m = -INFINITY;
     if (h < a.Hq) {
@@ -126,22 +205,20 @@ __global__ void __launch_bounds__(kBvThreads, 1) binv_accumulate_kernel(BinvArgs
     for (int o = 1; o < 16; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (l == 0) mrow[h] = m;
   }
-
-  // chunk c of the split into stage st: 64 positions' 32-byte bit slices, then the 4 tiles'
-  // score blocks (tiles past the split's end are zero-filled, never read as weights)
-  const int n_copies = 2 * kBvChunk + kBvPosGroups * a.Hq * kBvTile / 4;
-  auto issue = [&](int st, int64_t c) {
+  const int n_copies = kStgBits / 16 + kBvPosGroups * a.Hq * kBvTile / 4;
+  auto issue = [&](int st, int64_t c) {   // chunk c into stage st (pieces past the split zero-filled)
     const int64_t t0 = t_begin + c * kBvChunk;
+    unsigned char* dst = stg + st * kStgBytes;
     for (int e = tid; e < n_copies; e += kBvThreads) {
-      if (e < 2 * kBvChunk) {
+      if (e < kStgBits / 16) {
         const int p = e >> 1, h16 = e & 1;
         const bool ok = t0 + p < t_end;
-        cp_async16_z(&stage[st].bits[p][16 * h16], ok ? bsrc + (t0 + p) * (a.Nc / 8) + 16 * h16 : a.bits, ok);
+        cp_async16_z(dst + p * kBvSliceBytes + 16 * h16, ok ? bsrc + (t0 + p) * (a.Nc / 8) + 16 * h16 : a.bits, ok);
       } else {
-        const int j = e - 2 * kBvChunk;                  // 16-byte piece of the 4 score blocks
+        const int j = e - kStgBits / 16;
         const int q = j / (a.Hq * kBvTile / 4);
         const bool ok = t0 + q * kBvTile < t_end;
-        cp_async16_z(&stage[st].sc[4 * j], ok ? ssrc + c * kBvPosGroups * a.Hq * kBvTile + 4 * j : a.scores, ok);
+        cp_async16_z(dst + kStgBits + 16 * j, ok ? ssrc + c * kBvPosGroups * a.Hq * kBvTile + 4 * j : a.scores, ok);
       }
     }
   };
@@ -150,107 +227,109 @@ __global__ void __launch_bounds__(kBvThreads, 1) binv_accumulate_kernel(BinvArgs
     if (s < n_c) issue(s, s);
     cp_async_commit();
   }
-  __syncthreads();   // mrow
+  tc_fence_before();
+  __syncthreads();   // TMEM address, mbarriers, mrow
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
 
-  float H[2][8][4];
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) H[mt][nt][0] = H[mt][nt][1] = H[mt][nt][2] = H[mt][nt][3] = 0.0f;
-  const int ph = tid >> 4, pt = tid & 15;   // weight builder: head row, position column of each tile
+  const int ph = tid >> 4, pt = tid & 15;   // weight builder: head, position column of each step
   const int pslot = tile_slot(pt);
   const float m_h = mrow[ph];
-  const bool two_mt = a.Hq > 16;
+  const uint32_t boff = static_cast<uint32_t>((ph >> 3) * 256 + (pt >> 3) * 128 + (ph & 7) * 16 + (pt & 7) * 2);
+  // bit expansion: this warp's TMEM lane quarter and its two (half, step) units
+  const int quarter = warp & 3;
   float lacc = 0.0f;
-  // ldmatrix row addresses of the weight tile: matrix (lane >> 3) is rows 0-7 / 8-15 of k 0-7,
-  // then rows 0-7 / 8-15 of k 8-15; this warp's k columns are those of its position group
-  const int lrow = (lane & 7) + (((lane >> 3) & 1) << 3), lcol = pg * kBvTile + ((lane >> 4) << 3);
-  const int brow = pg * kBvTile + 2 * i;
+  bool ok = true;
   for (int64_t c = 0; c < n_c; ++c) {
-    const int st = static_cast<int>(c % kBvStages);
-    cp_async_wait<kBvStages - 2>();   // chunk c has landed (this thread's pieces)
-    __syncthreads();                  // ... everyone's; and chunk c - 1 is done with its stage and the weights
+    const int st = static_cast<int>(c % kBvStages), bb = static_cast<int>(c & 1);
+    cp_async_wait<kBvStages - 2>();
+    __syncthreads();   // chunk c landed; chunk c - 1's stage reads are done
     {
       const int64_t cn = c + kBvStages - 1;
       if (cn < n_c) issue(static_cast<int>(cn % kBvStages), cn);
       cp_async_commit();
     }
-    // weights 2^(score - m), fp16, and their fp32 row sums
+    if (c >= 2) {   // the MMAs of chunk c - 2 read buffer bb
+      ok = mbar_wait_bounded(&mbar[bb], static_cast<uint32_t>(((c >> 1) - 1) & 1), kBvWaitPolls) && ok;
+      tc_fence_after();
+    }
+    const unsigned char* sg = stg + st * kStgBytes;
+    const float* sc = reinterpret_cast<const float*>(sg + kStgBits);
+    // weights 2^(score - m), fp16, into B; fp32 row sums
 #pragma unroll
     for (int q = 0; q < kBvPosGroups; ++q) {
       const int64_t t = t_begin + c * kBvChunk + q * kBvTile + pt;
       const bool valid = ph < a.Hq && t < t_end;
-      const float p = valid ? exp2f(stage[st].sc[(q * a.Hq + ph) * kBvTile + pslot] - m_h) : 0.0f;
+      const float p = valid ? exp2f(sc[(q * a.Hq + ph) * kBvTile + pslot] - m_h) : 0.0f;
       lacc += p;
-      ptile[ph][q * kBvTile + pt] = __float2half_rn(p);
+      *reinterpret_cast<__half*>(bbuf + bb * kBvBBytes + q * 1024 + boff) = __float2half_rn(p);
     }
-    __syncthreads();
-    uint32_t A[2][4];
+    fence_async_smem();   // generic-proxy writes of B, read by the tensor cores
+    // bits -> fp16 0 / 1 in TMEM: lane `lane` of quarter `quarter` is codebook row
+    // hb 128 + 32 quarter + lane; column j of a step holds positions 2j (low half) and 2j + 1
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      const unsigned addr = static_cast<unsigned>(__cvta_generic_to_shared(&ptile[mt * 16 + lrow][lcol]));
-      asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                   : "=r"(A[mt][0]), "=r"(A[mt][1]), "=r"(A[mt][2]), "=r"(A[mt][3])
-                   : "r"(addr));
+    for (int u = 0; u < 2; ++u) {
+      const int unit = (warp >> 2) * 2 + u, hb = unit >> 2, ks = unit & 3;
+      const unsigned char* rows = sg + (ks * kBvTile) * kBvSliceBytes + hb * 16 + 4 * quarter;
+      uint32_t col[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(rows + (2 * j) * kBvSliceBytes);
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(rows + (2 * j + 1) * kBvSliceBytes);
+        col[j] = (((w0 >> lane) & 1u) | (((w1 >> lane) & 1u) << 16)) * 0x3C00u;
+      }
+      tmem_st8(tbase + (static_cast<uint32_t>(32 * quarter) << 16) + kBvColA + (bb * 2 + hb) * 32 + ks * 8, col);
     }
-    // the warp's 64 codebook rows: bytes 8 bg .. 8 bg + 7 of its tile's positions' slices
-    const uint2 w0 = *reinterpret_cast<const uint2*>(&stage[st].bits[brow][8 * bg]);
-    const uint2 w1 = *reinterpret_cast<const uint2*>(&stage[st].bits[brow + 1][8 * bg]);
-    const uint2 w2 = *reinterpret_cast<const uint2*>(&stage[st].bits[brow + 8][8 * bg]);
-    const uint2 w3 = *reinterpret_cast<const uint2*>(&stage[st].bits[brow + 9][8 * bg]);
+    tc_wait_st();
+    tc_fence_before();
+    ok = __syncthreads_and(ok) != 0;   // B and A of chunk c are complete; every wait succeeded
+    if (!ok) break;                    // (uniform) a wait gave up: issue nothing more
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t bsa = smem_u32(bbuf + bb * kBvBBytes);
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int sh = (nt & 3) * 8 + g;   // bit nt * 8 + g of the 64-bit slice
-      const uint32_t x0 = nt < 4 ? w0.x : w0.y, x1 = nt < 4 ? w1.x : w1.y;
-      const uint32_t x2 = nt < 4 ? w2.x : w2.y, x3 = nt < 4 ? w3.x : w3.y;
-      const uint32_t b0 = bits_to_h2((x0 >> sh) & 1u, (x1 >> sh) & 1u);
-      const uint32_t b1 = bits_to_h2((x2 >> sh) & 1u, (x3 >> sh) & 1u);
-      mma_f16(H[0][nt], A[0], b0, b1);
-      if (two_mt) mma_f16(H[1][nt], A[1], b0, b1);
+      for (int ks = 0; ks < kBvPosGroups; ++ks) {
+        const uint64_t bd = smem_desc_k(bsa + ks * 1024, 128, 256);
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb)
+          umma_f16_ts(tbase + hb * 32, tbase + kBvColA + (bb * 2 + hb) * 32 + ks * 8, bd, kBvIdesc,
+                      (c > 0 || ks > 0) ? 1u : 0u);
+      }
+      umma_commit(&mbar[bb]);
     }
   }
   cp_async_wait<0>();
-  __syncthreads();   // the stages are free: the reduction buffer overlays them
+  // the last commit covers every MMA issued before it
+  if (n_c > 0 && ok) {
+    const int64_t cl = n_c - 1;
+    ok = mbar_wait_bounded(&mbar[cl & 1], static_cast<uint32_t>((cl >> 1) & 1), kBvWaitPolls);
+  }
+  tc_fence_after();
+  ok = __syncthreads_and(ok) != 0;
+  if (!ok && tid == 0) atomicOr(a.error_word, kErrWaitLimit);
 
-  // row sums: the 16 builders of a head are 16 consecutive lanes
 #pragma unroll
   for (int o = 1; o < 16; o <<= 1) lacc += __shfl_xor_sync(0xffffffffu, lacc, o);
   const int64_t base = (static_cast<int64_t>(b) * a.Sv + v) * a.Hq;
   if (slice == 0 && pt == 0 && ph < a.Hq) a.mlpart[base + ph] = make_float2(m_h, lacc);
-  // the four position groups' sums: groups 1-3 through shared memory into group 0
-  if (pg > 0) {
-    float* dst = hred + ((pg - 1) * kBvBitGroups + bg) * kBvMaxHeads * kHRed;
+  if (warp < 8) {   // warps 0-3: rows 0-127 (D of half 0), warps 4-7: rows 128-255
+    const int hb = warp >> 2;
+    const bool have = n_c > 0 && ok;   // uniform
+    uint32_t r[32];
+    if (have) {
+      tmem_ld32(tbase + (static_cast<uint32_t>(32 * quarter) << 16) + hb * 32, r);
+      tc_wait_ld();
+    }
+    float* dst = a.hpart + base * a.Nc + slice * kBvBitsPerCta + hb * 128 + 32 * quarter + lane;
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr)
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-          *reinterpret_cast<float2*>(dst + (mt * 16 + g + 8 * rr) * kHRed + nt * 8 + 2 * i) =
-              make_float2(H[mt][nt][2 * rr], H[mt][nt][2 * rr + 1]);
+    for (int h = 0; h < kBvMaxHeads; ++h)
+      if (h < a.Hq) dst[static_cast<int64_t>(h) * a.Nc] = have ? __uint_as_float(r[h]) : 0.0f;
   }
+  tc_fence_before();
   __syncthreads();
-  if (pg == 0) {
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int h = mt * 16 + g + 8 * rr;
-        if (h >= a.Hq) continue;
-        float* dst = a.hpart + (base + h) * a.Nc + slice * kBvBitsPerCta + bg * kBvBitsPerWarp;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          float2 sum = make_float2(H[mt][nt][2 * rr], H[mt][nt][2 * rr + 1]);
-#pragma unroll
-          for (int q = 0; q < kBvPosGroups - 1; ++q) {
-            const float2 o = *reinterpret_cast<const float2*>(
-                hred + ((q * kBvBitGroups + bg) * kBvMaxHeads + h) * kHRed + nt * 8 + 2 * i);
-            sum.x += o.x;
-            sum.y += o.y;
-          }
-          *reinterpret_cast<float2*>(dst + nt * 8 + 2 * i) = sum;
-        }
-      }
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tbase), "r"(kBvCols) : "memory");
   }
 }
 
@@ -260,7 +339,7 @@ __global__ void __launch_bounds__(kBvThreads, 1) binv_accumulate_kernel(BinvArgs
 // The chunk's rows of C are copied into shared memory before the wait on the previous kernel.
 // The chunk-0 CTA also stores (M, L = sum_v 2^(m_v - M) l_v).
 __global__ void __launch_bounds__(256) binv_merge_contract_kernel(BinvArgs a) {
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(1024) unsigned char smem[];
   float* cs = reinterpret_cast<float*>(smem);                 // [kBvCRows][128]
   float* wts = cs + kBvCRows * kD;                            // [kBvMaxG][kBvMaxSplits]
   float* hc = wts + kBvMaxG * kBvMaxSplits;                   // [kBvMaxG][kBvCRows]
@@ -447,6 +526,7 @@ extern "C" commvq_status commvq_attend_decode_binv(const commvq_config* cfg, con
   BinvArgs v{};
   v.scores = a.scores;
   v.partials = a.partials;
+  v.error_word = a.error_word;
   v.seq_offsets = seq_offsets;
   v.bits = v_bits;
   v.C = v_codebook;
@@ -466,11 +546,11 @@ extern "C" commvq_status commvq_attend_decode_binv(const commvq_config* cfg, con
   v.K = L.K;
   v.Sv = L.Sv;
   if (cudaFuncSetAttribute(binv_accumulate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kBvAccSmem)) != cudaSuccess ||
+                           static_cast<int>(kBvTcSmem)) != cudaSuccess ||
       cudaFuncSetAttribute(binv_merge_contract_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kBvMcSmem)) != cudaSuccess)
     return COMMVQ_ERR_CUDA;
-  if (launch_dependent(binv_accumulate_kernel, dim3(L.Sv, n_bits / kBvBitsPerCta, B), dim3(kBvThreads), kBvAccSmem,
+  if (launch_dependent(binv_accumulate_kernel, dim3(L.Sv, n_bits / kBvBitsPerCta, B), dim3(kBvThreads), kBvTcSmem,
                        st, v) != cudaSuccess)
     return COMMVQ_ERR_CUDA;
   if (launch_dependent(binv_merge_contract_kernel, dim3(B * cfg->kv_heads, n_bits / kBvCRows), dim3(256), kBvMcSmem,

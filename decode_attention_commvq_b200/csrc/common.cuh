@@ -18,6 +18,7 @@ constexpr int kPairs = kG / 2; // RoPE pairs per group
 
 // Device error word bits (first 4 bytes of an attention workspace).
 constexpr int kErrCodeRange = 1;
+constexpr int kErrWaitLimit = 2;   // a bounded wait on asynchronous tensor-core work gave up
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

@@ -345,7 +345,8 @@ commvq_status commvq_dense_decode(const commvq_config* cfg, const void* q, commv
 
 /* The device error word in an attention workspace: synchronises `stream`, copies the word
  * to the host and writes it to *device_error (0 = none; bit 0 = a code >= Nc' was seen
- * and clamped). Returns COMMVQ_ERR_DEVICE_CHECK when the word is non-zero. */
+ * and clamped; bit 1 = a bounded wait for the tensor cores' asynchronous work gave up, the
+ * output of that call is not valid). Returns COMMVQ_ERR_DEVICE_CHECK when the word is non-zero. */
 commvq_status commvq_workspace_error(const void* workspace, int32_t* device_error, void* stream);
 
 /* Static description of a status code. */
