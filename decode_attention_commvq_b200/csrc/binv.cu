@@ -22,15 +22,12 @@ namespace commvq {
 namespace {
 
 constexpr int kBvThreads = 512;   // 16 warps
-constexpr int kBvPosGroups = 4;   // 16-position MMA steps per chunk
 constexpr int kBvBitsPerCta = 256;                              // two M = 128 halves
 constexpr int kBvSliceBytes = kBvBitsPerCta / 8;                // 32
 constexpr int kBvMaxHeads = 32;
 constexpr int kBvTile = 16;       // positions per MMA K step (one tile of the scores buffer)
-constexpr int kBvChunk = kBvPosGroups * kBvTile;   // positions per pipeline step
-constexpr int kBvStages = 4;
 constexpr int kBvMaxSplits = 64;
-constexpr int kBvCRows = 128;                      // rows of C per merge-and-contract CTA
+constexpr int kBvCRows = 64;                       // rows of C per merge-and-contract CTA
 constexpr int kBvMaxG = 8;
 
 struct BinvArgs {
@@ -39,18 +36,23 @@ struct BinvArgs {
   const int64_t* seq_offsets;
   const uint8_t* bits;        // [total_T, Nc / 8]
   const float* C;             // [Nc, KV * 128]
+  unsigned char* wts;         // [B][n_tiles] 1.5 KB blocks: weight digits, the MMA's B layout
+  float* mvec;                // [B][Sv][Hq] value-split maxima m_v
+  float* lpart;               // [B][Sv][P][Hq] partial sums of the weights
   float* hpart;               // [B][Sv][Hq][Nc]
-  float2* mlpart;             // [B][Sv][Hq] (m, l)
   float* opart;               // [B][Hq][Nc / kBvCRows][128]
   float2* ml;                 // [B][Hq] (M, L)
   float* out;
   float* lse;
   int* error_word;
   int64_t max_T, n_tiles;
-  int B, Hq, KV, Nc, S, K, Sv;   // S scores splits, K of them per value split, Sv value splits
+  int B, Hq, KV, Nc, S, K, Sv, P;   // S scores splits, K of them per value split, Sv value splits,
+                                    // P weight-kernel parts per value split
 };
 
-constexpr size_t kBvMcSmem = (kBvCRows * kD + kBvMaxG * kBvMaxSplits + 2 * kBvMaxG * kBvCRows) * 4;
+// C chunk, split weights, merged H, the second half's contraction, split maxima and sums
+constexpr size_t kBvMcSmem =
+    (kBvCRows * kD + kBvMaxG * kBvMaxSplits + kBvMaxG * kBvCRows + kBvMaxG * kD + 2 * kBvMaxG * kBvMaxSplits) * 4;
 
 // Value split v of sequence b: scores splits vK .. vK + K - 1 (the same tile-aligned pieces of
 // ceil(T_b / S) positions).
@@ -71,9 +73,6 @@ __device__ __forceinline__ void cp_async16_z(void* smem_dst, const void* gmem_sr
                : "memory");
 }
 
-// Position tau of a 16-position tile sits at this offset of the head's 16 scores (the scores
-// kernel's fragment order).
-__device__ __forceinline__ int tile_slot(int tau) { return ((tau & 7) >> 1) * 4 + (tau & 1) + 2 * (tau >> 3); }
 
 // ---------------------------------------------------------------------------------------
 // tcgen05 pieces (PTX ISA 8.6, sm_100a): TMEM allocation, loads and stores, the f16 MMA with its
@@ -123,12 +122,13 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
       : "r"(taddr)
       : "memory");
 }
-// D[128 x N] (+)= A[128 x 16] (TMEM, fp16) * B[16 x N] (shared memory descriptor, fp16), fp32 D.
-__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
+// D[128 x N] (+)= A[128 x 32] (TMEM, unsigned 8-bit) * B[32 x N] (shared memory descriptor,
+// unsigned 8-bit), int32 D.
+__device__ __forceinline__ void umma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -137,193 +137,303 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
-// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B fp16 (formats 0), both
-// K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
-constexpr uint32_t kBvIdesc = (1u << 4) | ((32u >> 3) << 17) | ((128u >> 4) << 24);
+// Instruction descriptor, kind::i8: D int32 (bits 4-5 = 2), A and B unsigned 8-bit (formats 0),
+// both K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+constexpr uint32_t kBvIdesc = (2u << 4) | ((32u >> 3) << 17) | ((128u >> 4) << 24);
 // Shared-memory descriptor of a K-major, unswizzled operand: 8-row x 16-byte core matrices,
-// LBO = byte step between the two 8-element K halves, SBO = byte step between 8-row groups,
+// LBO = byte step between the two 16-byte K halves, SBO = byte step between 8-row groups,
 // version 1 at bits 46-47.
 __device__ __forceinline__ uint64_t smem_desc_k(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
          (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
-constexpr int kBvCols = 256;       // TMEM columns: D (2 x 32), A (2 buffers x 2 halves x 32)
-constexpr int kBvColA = 64;
+// Weights as 24-bit fixed point q = round(p (2^24 - 1)) in three 8-bit digits (most significant
+// first): the MMA sums s_t[n] x digit exactly in int32 (at most 2^8 x positions per split), and
+// H = (D0 2^16 + D1 2^8 + D2) / (2^24 - 1) carries each weight to 2^-25 absolute, as good as
+// fp16 down to 2^-14 and better below.
+constexpr float kBvQScale = 16777215.0f;
+constexpr int kBvDigits = 3;
+constexpr int kBvWTile = kBvDigits * 512;   // weight bytes per 16-position tile
+constexpr int kBvCols = 512;       // TMEM columns: D (2 halves x 3 digits x 32), A (2 buffers x 2 halves x 32)
+constexpr int kBvColA = 2 * kBvDigits * 32;
+constexpr int kBvCk = 128;         // positions per chunk (4 MMA K steps of 32)
+constexpr int kBvStep = 32;
+constexpr int kBvRing = 6;         // chunk stages in shared memory
+constexpr int kBvDist = 3;         // chunks in flight ahead of the one being expanded
 constexpr uint32_t kBvWaitPolls = 1u << 20;
-// B operand of one buffer: 4 k-steps x [32 heads x 16 positions] fp16, K-major core matrices:
-// (head h, position k of the step) at ks 1024 + (h / 8) 256 + (k / 8) 128 + (h % 8) 16 + (k % 8) 2.
-constexpr int kBvBBytes = kBvPosGroups * kBvMaxHeads * kBvTile * 2;
-constexpr size_t kBvTcSmem = 2 * kBvBBytes + kBvStages * (kBvChunk * kBvSliceBytes + kBvPosGroups * kBvMaxHeads * kBvTile * 4) +
-                             kBvMaxHeads * 4 + 2 * 8 + 16;
+constexpr int kBvPlane = kBvCk * 16;                                      // one 16-byte half of every slice
+constexpr int kBvStageBytes = 2 * kBvPlane + (kBvCk / kBvTile) * kBvWTile;   // bits + 8 weight tiles
+constexpr size_t kBvTcSmem = static_cast<size_t>(kBvRing) * kBvStageBytes + kBvRing * 8 + 16;
 
-// H_v^T[n, h] = sum_t s_t[n] 2^(score_{h,t} - m_v) for the CTA's 256 codebook rows (two M = 128
-// halves) and all 32 head columns, on tcgen05: per 64-position chunk, 16 warps expand the bits to
-// fp16 0 / 1 straight into TMEM (A, one 32-lane quarter and one 16-position step per store), all
-// threads write the weights into shared memory (B), and one thread issues 8 MMAs (2 halves x 4
-// steps) and commits them to the buffer's mbarrier. Two A/B buffers: chunk c + 1 is built while
-// chunk c's MMAs run.
+// Weights once per value split: p = 2^(score - m_v), its three digits in 1.5 KB blocks per
+// 16-position tile laid out as the MMA's B operand (digit d, head h, position k of the tile at
+// d 512 + (h / 8) 128 + (h % 8) 16 + k; heads >= Hq and positions past the sequence are 0), the
+// split's maxima, and fp32 partial sums of p per part. Grid: value splits x parts x sequences;
+// thread (h, j) takes positions 2j, 2j + 1 of each tile of its part.
+__global__ void __launch_bounds__(256) binv_weights_kernel(BinvArgs a) {
+  __shared__ float mrow[kBvMaxHeads];
+  const int v = blockIdx.x, part = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, h = tid >> 3, j = tid & 7;
+  int64_t row0, t_begin, t_end;
+  bv_split(a, b, v, row0, t_begin, t_end);
+  const int64_t n_tl = (t_end - t_begin + kBvTile - 1) / kBvTile;
+  const int64_t per = (n_tl + a.P - 1) / a.P;
+  const int64_t tl0 = min(n_tl, part * per), tl1 = min(n_tl, tl0 + per);
+  pdl_wait();
+  {   // the split's maximum per head: the maxima of its K scores splits (8 lanes per head)
+    float m = -INFINITY;
+    if (h < a.Hq) {
+      const Partial* ph = a.partials + (static_cast<int64_t>(b) * a.Hq + h) * a.S;
+      for (int s = v * a.K + j; s < min(a.S, (v + 1) * a.K); s += 8) m = fmaxf(m, ph[s].m);
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (j == 0) mrow[h] = m;
+  }
+  __syncthreads();
+  const float m = mrow[h];
+  // the scores buffer holds position tau of a tile at ((tau % 8) / 2) 4 + tau % 2 + 2 (tau / 8):
+  // positions 2j and 2j + 1 are neighbours
+  const int slot0 = (j & 3) * 4 + 2 * (j >> 2);
+  const uint32_t woff = static_cast<uint32_t>((h >> 3) * 128 + (h & 7) * 16 + 2 * j);
+  float lsum = 0.0f;
+  const float* sbase = a.scores + (static_cast<int64_t>(b) * a.n_tiles + t_begin / kBvTile) * a.Hq * kBvTile +
+                       h * kBvTile + slot0;
+  unsigned char* wbase = a.wts + (static_cast<int64_t>(b) * a.n_tiles + t_begin / kBvTile) * kBvWTile + woff;
+  for (int64_t tl = tl0; tl < tl1; tl += 4) {   // four tiles' loads in flight
+    float2 f[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      f[u] = (h < a.Hq && tl + u < tl1)
+                 ? *reinterpret_cast<const float2*>(sbase + (tl + u) * a.Hq * kBvTile)
+                 : make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (tl + u >= tl1) break;
+      const int64_t t0 = t_begin + (tl + u) * kBvTile;
+      const bool hv = h < a.Hq;
+      const float p0 = (hv && t0 + 2 * j < t_end) ? exp2f(f[u].x - m) : 0.0f;
+      const float p1 = (hv && t0 + 2 * j + 1 < t_end) ? exp2f(f[u].y - m) : 0.0f;
+      lsum += p0 + p1;
+      const uint32_t q0 = __float2uint_rn(p0 * kBvQScale), q1 = __float2uint_rn(p1 * kBvQScale);
+      unsigned char* w = wbase + (tl + u) * kBvWTile;
+#pragma unroll
+      for (int d = 0; d < kBvDigits; ++d) {
+        const int sh = 8 * (kBvDigits - 1 - d);
+        *reinterpret_cast<uint16_t*>(w + d * 512) =
+            static_cast<uint16_t>(((q0 >> sh) & 0xFFu) | (((q1 >> sh) & 0xFFu) << 8));
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  if (j == 0 && h < a.Hq) {
+    a.lpart[((static_cast<int64_t>(b) * a.Sv + v) * a.P + part) * a.Hq + h] = lsum;
+    if (part == 0) a.mvec[(static_cast<int64_t>(b) * a.Sv + v) * a.Hq + h] = m;
+  }
+}
+
+// 32 x 32 bit transpose across a warp: lane p holds w with bit l = row l at position p; returns,
+// in lane l, the word whose bit p = row l at position p. Five butterfly exchanges; at block size
+// jj a lane keeps its own half of every 2jj-bit block and takes the partner's other half, moved
+// by a rotation (left by jj in the lower lane, right by jj in the upper).
+struct BitTranspose {
+  uint32_t keep[5], rot[5];
+  __device__ __forceinline__ explicit BitTranspose(int lane) {
+    const uint32_t masks[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+      const int jj = 16 >> k;
+      keep[k] = (lane & jj) ? ~masks[k] : masks[k];
+      rot[k] = (lane & jj) ? 32u - jj : static_cast<uint32_t>(jj);
+    }
+  }
+  __device__ __forceinline__ uint32_t operator()(uint32_t x) const {
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+      const uint32_t t = __shfl_xor_sync(0xffffffffu, x, 16 >> k);
+      const uint32_t u = __funnelshift_l(t, t, rot[k]);
+      x = (x & keep[k]) | (u & ~keep[k]);
+    }
+    return x;
+  }
+};
+
+// H_v^T[n, h] = sum_t s_t[n] q_{h,t} for the CTA's 256 codebook rows (two M = 128 halves) and 32
+// head columns on tcgen05 (kind::i8, exact int32 sums). Per 128-position chunk: cp.async brings
+// the bits and the weight tiles into a ring stage; each warp turns two 32-position x 32-row bit
+// blocks (its TMEM lane quarter) into bytes 0 / 1 through a warp bit transpose and a nibble
+// spread, and stores them into TMEM (A). 24 MMAs per chunk (4 steps x 2 halves x 3 digits),
+// spread over four issuing warps, take their B operand (a digit plane) from the stage; each
+// issuing warp commits its MMAs to the stage's mbarrier. The wait for chunk c - 2 before chunk
+// c's stores frees both the A buffer and the stage that chunk c + 3 is copied into. One CTA
+// barrier per chunk.
 __global__ void __launch_bounds__(kBvThreads, 1) binv_accumulate_kernel(BinvArgs a) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  unsigned char* bbuf = smem;                                                  // [2][kBvBBytes]
-  unsigned char* stg = smem + 2 * kBvBBytes;                                   // [stages][bits | scores]
-  constexpr int kStgBits = kBvChunk * kBvSliceBytes;                           // 2048
-  constexpr int kStgBytes = kStgBits + kBvPosGroups * kBvMaxHeads * kBvTile * 4;
-  float* mrow = reinterpret_cast<float*>(stg + kBvStages * kStgBytes);
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(mrow + kBvMaxHeads);            // [2]
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(mbar + 2);
+  unsigned char* ring = smem;                                                     // [kBvRing][stage]
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + kBvRing * kBvStageBytes);   // [kBvRing]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(mbar + kBvRing);
 
   const int v = blockIdx.x, slice = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int64_t row0, t_begin, t_end;
   bv_split(a, b, v, row0, t_begin, t_end);
-  const int64_t n_c = (t_end - t_begin + kBvChunk - 1) / kBvChunk;
-  const uint8_t* bsrc = a.bits + row0 * (a.Nc / 8) + slice * kBvSliceBytes;
-  const float* ssrc = a.scores + (static_cast<int64_t>(b) * a.n_tiles + t_begin / kBvTile) * a.Hq * kBvTile;
+  const int len = static_cast<int>(t_end - t_begin);   // at most max_T / S * K positions
+  const int n_c = (len + kBvCk - 1) / kBvCk;
+  const int64_t rowb = a.Nc / 8;
+  const uint8_t* bsrc = a.bits + (row0 + t_begin) * rowb + slice * kBvSliceBytes;   // the split's first row
+  const unsigned char* wsrc = a.wts + (static_cast<int64_t>(b) * a.n_tiles + t_begin / kBvTile) * kBvWTile;
 
-  if (warp == 0) {   // TMEM for the accumulators and the A buffers (one CTA per SM)
+  if (warp == 0) {   // all of TMEM: one CTA per SM
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tslot)),
                  "r"(kBvCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
-  if (tid == 0) {
-    mbar_init(&mbar[0], 1);
-    mbar_init(&mbar[1], 1);
+  if (tid == 0) {   // a chunk's four issuing warps each commit once
+    for (int s = 0; s < kBvRing; ++s) mbar_init(&mbar[s], 4);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  pdl_wait();   // the scores kernel's buffer and maxima are complete from here on
+  pdl_wait();   // the weight tiles are complete from here on
 
-  {   // the split's maximum per head: the maxima of its K scores splits (16 lanes per head)
-    const int h = tid >> 4, l = tid & 15;
-    float m = -INFINITY;
-    if (h < a.Hq) {
-      const Partial* ph = a.partials + (static_cast<int64_t>(b) * a.Hq + h) * a.S;
-      for (int s = v * a.K + l; s < min(a.S, (v + 1) * a.K); s += 16) m = fmaxf(m, ph[s].m);
-    }
-#pragma unroll
-    for (int o = 1; o < 16; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (l == 0) mrow[h] = m;
-  }
-  const int n_copies = kStgBits / 16 + kBvPosGroups * a.Hq * kBvTile / 4;
-  auto issue = [&](int st, int64_t c) {   // chunk c into stage st (pieces past the split zero-filled)
-    const int64_t t0 = t_begin + c * kBvChunk;
-    unsigned char* dst = stg + st * kStgBytes;
-    for (int e = tid; e < n_copies; e += kBvThreads) {
-      if (e < kStgBits / 16) {
-        const int p = e >> 1, h16 = e & 1;
-        const bool ok = t0 + p < t_end;
-        cp_async16_z(dst + p * kBvSliceBytes + 16 * h16, ok ? bsrc + (t0 + p) * (a.Nc / 8) + 16 * h16 : a.bits, ok);
-      } else {
-        const int j = e - kStgBits / 16;
-        const int q = j / (a.Hq * kBvTile / 4);
-        const bool ok = t0 + q * kBvTile < t_end;
-        cp_async16_z(dst + kStgBits + 16 * j, ok ? ssrc + c * kBvPosGroups * a.Hq * kBvTile + 4 * j : a.scores, ok);
-      }
-    }
+  // Each thread copies two 16-byte pieces of every chunk: threads 0-255 one piece of bits
+  // (position tid / 2, half tid % 2) and weight piece tid + 256, threads 256-511 weight pieces
+  // tid - 256 and tid + 256 (a chunk holds 256 bit pieces and 768 weight pieces of 16 bytes).
+  constexpr int kTilePieces = kBvWTile / 16;   // 96 per weight tile
+  const bool bits_piece = tid < 256;
+  const int w0 = bits_piece ? -1 : tid - 256, w1 = tid + 256;
+  const int p_lim0 = bits_piece ? tid >> 1 : (w0 / kTilePieces) * kBvTile;   // position that must exist
+  const int p_lim1 = (w1 / kTilePieces) * kBvTile;
+  const uint8_t* src0 = bits_piece ? bsrc + (tid >> 1) * rowb + 16 * (tid & 1) : wsrc + 16 * w0;
+  const unsigned char* src1 = wsrc + 16 * w1;
+  const int64_t step0 = bits_piece ? kBvCk * rowb : (kBvCk / kBvTile) * kBvWTile;   // per chunk
+  constexpr int64_t step1 = (kBvCk / kBvTile) * kBvWTile;
+  const int doff0 = bits_piece ? (tid & 1) * kBvPlane + (tid >> 1) * 16 : 2 * kBvPlane + 16 * w0;
+  const int doff1 = 2 * kBvPlane + 16 * w1;
+  auto issue = [&](int c, int st) {   // chunk c into stage st (pieces past the split zero-filled)
+    unsigned char* dst = ring + st * kBvStageBytes;
+    const int pos = c * kBvCk;
+    const bool ok0 = pos + p_lim0 < len, ok1 = pos + p_lim1 < len;
+    cp_async16_z(dst + doff0, ok0 ? src0 + c * step0 : a.wts, ok0);
+    cp_async16_z(dst + doff1, ok1 ? src1 + c * step1 : a.wts, ok1);
   };
 #pragma unroll
-  for (int s = 0; s < kBvStages - 1; ++s) {
+  for (int s = 0; s < kBvDist; ++s) {
     if (s < n_c) issue(s, s);
     cp_async_commit();
   }
   tc_fence_before();
-  __syncthreads();   // TMEM address, mbarriers, mrow
+  __syncthreads();   // TMEM address
   tc_fence_after();
   const uint32_t tbase = *tslot;
-
-  const int ph = tid >> 4, pt = tid & 15;   // weight builder: head, position column of each step
-  const int pslot = tile_slot(pt);
-  const float m_h = mrow[ph];
-  const uint32_t boff = static_cast<uint32_t>((ph >> 3) * 256 + (pt >> 3) * 128 + (ph & 7) * 16 + (pt & 7) * 2);
-  // bit expansion: this warp's TMEM lane quarter and its two (half, step) units
   const int quarter = warp & 3;
-  float lacc = 0.0f;
+  const uint32_t tq = tbase + (static_cast<uint32_t>(32 * quarter) << 16);
+  if (warp < 4) {   // zero the accumulators: every MMA then adds, in whatever order they run
+    uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int c8 = 0; c8 < kBvColA / 8; ++c8) tmem_st8(tq + c8 * 8, z);
+    tc_wait_st();
+  }
+  cp_async_wait<kBvDist - 1>();   // chunk 0 (this thread's pieces)
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();   // mbarriers, zeroed accumulators, chunk 0
+  tc_fence_after();
+  const BitTranspose transpose(lane);
+  // this warp's two 32 x 32 bit blocks: rows hb 128 + 32 quarter + lane, positions 32 step + 0..31
+  const int grp = warp >> 2;
+  uint32_t lds_off[2], col_off[2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int idx = grp * 2 + u, hb = idx >> 2, step = idx & 3;
+    lds_off[u] = static_cast<uint32_t>(hb * kBvPlane + (kBvStep * step + lane) * 16 + 4 * quarter);
+    col_off[u] = static_cast<uint32_t>(kBvColA + hb * 32 + step * 8);
+  }
+  // MMA issue, spread over the four warps 0, 4, 8, 12: warp 4g takes group g's units (half g / 2,
+  // steps 2 (g % 2) and 2 (g % 2) + 1) for all three digits. Descriptors of stage 0; a stage,
+  // step or digit moves only the start-address field (addresses stay below 2^18 bytes).
+  const int ghb = grp >> 1, gs0 = 2 * (grp & 1);
+  const uint64_t desc0 = smem_desc_k(smem_u32(ring + 2 * kBvPlane), kBvWTile, 128);
   bool ok = true;
-  for (int64_t c = 0; c < n_c; ++c) {
-    const int st = static_cast<int>(c % kBvStages), bb = static_cast<int>(c & 1);
-    cp_async_wait<kBvStages - 2>();
-    __syncthreads();   // chunk c landed; chunk c - 1's stage reads are done
-    {
-      const int64_t cn = c + kBvStages - 1;
-      if (cn < n_c) issue(static_cast<int>(cn % kBvStages), cn);
-      cp_async_commit();
-    }
-    if (c >= 2) {   // the MMAs of chunk c - 2 read buffer bb
-      ok = mbar_wait_bounded(&mbar[bb], static_cast<uint32_t>(((c >> 1) - 1) & 1), kBvWaitPolls) && ok;
+  // ring positions: chunk c in stage st, chunk c - 2 in stage stw with mbarrier phase parity pw
+  // (starting from chunk -2: stage kBvRing - 2, parity 1), chunk c + kBvDist in stage sti
+  int st = 0, stw = kBvRing - 2, sti = kBvDist;
+  uint32_t pw = 1;
+  for (int c = 0; c < n_c; ++c) {
+    const uint32_t bbc = static_cast<uint32_t>(c & 1) * 64;
+    const unsigned char* sg = ring + st * kBvStageBytes;
+    if (c >= 2) {   // chunk c - 2's MMAs are done: its A buffer, and chunk c - 3's stage, are free
+      ok = mbar_wait_bounded(&mbar[stw], pw, kBvWaitPolls) && ok;
       tc_fence_after();
     }
-    const unsigned char* sg = stg + st * kStgBytes;
-    const float* sc = reinterpret_cast<const float*>(sg + kStgBits);
-    // weights 2^(score - m), fp16, into B; fp32 row sums
-#pragma unroll
-    for (int q = 0; q < kBvPosGroups; ++q) {
-      const int64_t t = t_begin + c * kBvChunk + q * kBvTile + pt;
-      const bool valid = ph < a.Hq && t < t_end;
-      const float p = valid ? exp2f(sc[(q * a.Hq + ph) * kBvTile + pslot] - m_h) : 0.0f;
-      lacc += p;
-      *reinterpret_cast<__half*>(bbuf + bb * kBvBBytes + q * 1024 + boff) = __float2half_rn(p);
-    }
-    fence_async_smem();   // generic-proxy writes of B, read by the tensor cores
-    // bits -> fp16 0 / 1 in TMEM: lane `lane` of quarter `quarter` is codebook row
-    // hb 128 + 32 quarter + lane; column j of a step holds positions 2j (low half) and 2j + 1
+    if (c + kBvDist < n_c) issue(c + kBvDist, sti);   // into chunk c - 3's stage
+    cp_async_commit();
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int unit = (warp >> 2) * 2 + u, hb = unit >> 2, ks = unit & 3;
-      const unsigned char* rows = sg + (ks * kBvTile) * kBvSliceBytes + hb * 16 + 4 * quarter;
-      uint32_t col[8];
+      const uint32_t x = transpose(*reinterpret_cast<const uint32_t*>(sg + lds_off[u]));
+      uint32_t col[8];   // byte k of column g: position 4g + k
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(rows + (2 * j) * kBvSliceBytes);
-        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(rows + (2 * j + 1) * kBvSliceBytes);
-        col[j] = (((w0 >> lane) & 1u) | (((w1 >> lane) & 1u) << 16)) * 0x3C00u;
-      }
-      tmem_st8(tbase + (static_cast<uint32_t>(32 * quarter) << 16) + kBvColA + (bb * 2 + hb) * 32 + ks * 8, col);
+      for (int g = 0; g < 8; ++g) col[g] = (((x >> (4 * g)) & 0xFu) * 0x00204081u) & 0x01010101u;
+      tmem_st8(tq + col_off[u] + bbc, col);
     }
     tc_wait_st();
+    cp_async_wait<kBvDist - 1>();   // chunk c + 1 (this thread's pieces)
+    fence_async_smem();              // cp.async writes -> the tensor cores' reads of the weights
     tc_fence_before();
-    ok = __syncthreads_and(ok) != 0;   // B and A of chunk c are complete; every wait succeeded
+    ok = __syncthreads_and(ok) != 0;   // A of chunk c stored, chunk c + 1 landed, every wait succeeded
     if (!ok) break;                    // (uniform) a wait gave up: issue nothing more
-    if (tid == 0) {
+    if ((warp & 3) == 0 && lane == 0) {
       tc_fence_after();
-      const uint32_t bsa = smem_u32(bbuf + bb * kBvBBytes);
+      const uint64_t dst = desc0 + static_cast<uint64_t>((st * kBvStageBytes) >> 4);
 #pragma unroll
-      for (int ks = 0; ks < kBvPosGroups; ++ks) {
-        const uint64_t bd = smem_desc_k(bsa + ks * 1024, 128, 256);
+      for (int k = 0; k < 2; ++k) {
+        const int step = gs0 + k;
 #pragma unroll
-        for (int hb = 0; hb < 2; ++hb)
-          umma_f16_ts(tbase + hb * 32, tbase + kBvColA + (bb * 2 + hb) * 32 + ks * 8, bd, kBvIdesc,
-                      (c > 0 || ks > 0) ? 1u : 0u);
+        for (int d = 0; d < kBvDigits; ++d)   // two consecutive tiles make the step's K = 32: LBO = one tile
+          umma_i8_ts(tbase + (ghb * kBvDigits + d) * 32, tbase + kBvColA + bbc + ghb * 32 + step * 8,
+                     dst + static_cast<uint64_t>(((2 * step) * kBvWTile + d * 512) >> 4), kBvIdesc, 1u);
       }
-      umma_commit(&mbar[bb]);
+      umma_commit(&mbar[st]);
+    }
+    st = st + 1 == kBvRing ? 0 : st + 1;
+    sti = sti + 1 == kBvRing ? 0 : sti + 1;
+    if (++stw == kBvRing) {
+      stw = 0;
+      pw ^= 1u;
     }
   }
   cp_async_wait<0>();
-  // the last commit covers every MMA issued before it
-  if (n_c > 0 && ok) {
-    const int64_t cl = n_c - 1;
-    ok = mbar_wait_bounded(&mbar[cl & 1], static_cast<uint32_t>((cl >> 1) & 1), kBvWaitPolls);
+  if (n_c > 0 && ok) {   // the last commit covers every MMA issued before it
+    const int cl = n_c - 1;
+    ok = mbar_wait_bounded(&mbar[cl % kBvRing], static_cast<uint32_t>((cl / kBvRing) & 1), kBvWaitPolls);
   }
   tc_fence_after();
   ok = __syncthreads_and(ok) != 0;
   if (!ok && tid == 0) atomicOr(a.error_word, kErrWaitLimit);
 
-#pragma unroll
-  for (int o = 1; o < 16; o <<= 1) lacc += __shfl_xor_sync(0xffffffffu, lacc, o);
-  const int64_t base = (static_cast<int64_t>(b) * a.Sv + v) * a.Hq;
-  if (slice == 0 && pt == 0 && ph < a.Hq) a.mlpart[base + ph] = make_float2(m_h, lacc);
-  if (warp < 8) {   // warps 0-3: rows 0-127 (D of half 0), warps 4-7: rows 128-255
+  if (warp < 8) {   // warps 0-3: rows 0-127 (half 0), warps 4-7: rows 128-255
     const int hb = warp >> 2;
     const bool have = n_c > 0 && ok;   // uniform
-    uint32_t r[32];
+    float hsum[32];
+#pragma unroll
+    for (int h = 0; h < 32; ++h) hsum[h] = 0.0f;
     if (have) {
-      tmem_ld32(tbase + (static_cast<uint32_t>(32 * quarter) << 16) + hb * 32, r);
-      tc_wait_ld();
+#pragma unroll
+      for (int d = 0; d < kBvDigits; ++d) {
+        uint32_t r[32];
+        tmem_ld32(tq + (hb * kBvDigits + d) * 32, r);
+        tc_wait_ld();
+        const float wd = d == 0 ? 65536.0f : (d == 1 ? 256.0f : 1.0f);
+#pragma unroll
+        for (int h = 0; h < 32; ++h) hsum[h] = fmaf(static_cast<float>(r[h]), wd, hsum[h]);
+      }
     }
+    const int64_t base = (static_cast<int64_t>(b) * a.Sv + v) * a.Hq;
     float* dst = a.hpart + base * a.Nc + slice * kBvBitsPerCta + hb * 128 + 32 * quarter + lane;
 #pragma unroll
     for (int h = 0; h < kBvMaxHeads; ++h)
-      if (h < a.Hq) dst[static_cast<int64_t>(h) * a.Nc] = have ? __uint_as_float(r[h]) : 0.0f;
+      if (h < a.Hq) dst[static_cast<int64_t>(h) * a.Nc] = hsum[h] * (1.0f / kBvQScale);
   }
   tc_fence_before();
   __syncthreads();
@@ -344,6 +454,8 @@ __global__ void __launch_bounds__(256) binv_merge_contract_kernel(BinvArgs a) {
   float* wts = cs + kBvCRows * kD;                            // [kBvMaxG][kBvMaxSplits]
   float* hc = wts + kBvMaxG * kBvMaxSplits;                   // [kBvMaxG][kBvCRows]
   float* half_out = hc + kBvMaxG * kBvCRows;                  // [kBvMaxG][128]
+  float* msplit = half_out + kBvMaxG * kD;                    // [kBvMaxG][kBvMaxSplits]
+  float* lsplit = msplit + kBvMaxG * kBvMaxSplits;            // [kBvMaxG][kBvMaxSplits]
   const int bkv = blockIdx.x, chunk = blockIdx.y;
   const int b = bkv / a.KV, kv = bkv % a.KV, G = a.Hq / a.KV;
   const int tid = threadIdx.x;
@@ -358,36 +470,45 @@ __global__ void __launch_bounds__(256) binv_merge_contract_kernel(BinvArgs a) {
     cp_async_commit();
   }
   pdl_wait();
-  const float2* mlb = a.mlpart + static_cast<int64_t>(b) * a.Sv * a.Hq + kv * G;
+  for (int e = tid; e < G * a.Sv; e += 256) {   // each (head, split): its maximum and weight sum
+    const int h = e / a.Sv, s = e % a.Sv;
+    const int64_t bs = static_cast<int64_t>(b) * a.Sv + s;
+    const float* lp = a.lpart + bs * a.P * a.Hq + kv * G + h;
+    float l = 0.0f;
+#pragma unroll 16
+    for (int q = 0; q < a.P; ++q) l += lp[static_cast<int64_t>(q) * a.Hq];
+    msplit[h * kBvMaxSplits + s] = a.mvec[bs * a.Hq + kv * G + h];
+    lsplit[h * kBvMaxSplits + s] = l;
+  }
+  __syncthreads();
   if (tid < G) {
     float M = -INFINITY;
-    for (int s = 0; s < a.Sv; ++s) M = fmaxf(M, mlb[static_cast<int64_t>(s) * a.Hq + tid].x);
+    for (int s = 0; s < a.Sv; ++s) M = fmaxf(M, msplit[tid * kBvMaxSplits + s]);
     float L = 0.0f;
     for (int s = 0; s < a.Sv; ++s) {
-      const float2 m_l = mlb[static_cast<int64_t>(s) * a.Hq + tid];
-      const float w = M == -INFINITY ? 0.0f : exp2f(m_l.x - M);
+      const float w = M == -INFINITY ? 0.0f : exp2f(msplit[tid * kBvMaxSplits + s] - M);
       wts[tid * kBvMaxSplits + s] = w;
-      L = fmaf(w, m_l.y, L);
+      L = fmaf(w, lsplit[tid * kBvMaxSplits + s], L);
     }
     if (chunk == 0) a.ml[static_cast<int64_t>(b) * a.Hq + kv * G + tid] = make_float2(M, L);
   }
   __syncthreads();
-  // merged H of the chunk: element (h, n), n fastest (coalesced); four independent partial sums
+  // merged H of the chunk: element (h, n), n fastest (coalesced); eight split sums in flight
   for (int e = tid; e < G * kBvCRows; e += 256) {
     const int h = e / kBvCRows, n = e % kBvCRows;
     const float* src = a.hpart + (static_cast<int64_t>(b) * a.Sv * a.Hq + kv * G + h) * a.Nc + n0 + n;
     const int64_t step = static_cast<int64_t>(a.Hq) * a.Nc;
     const float* w = wts + h * kBvMaxSplits;
-    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
-    int s = 0;
-    for (; s + 4 <= a.Sv; s += 4) {
-      s0 = fmaf(w[s], src[s * step], s0);
-      s1 = fmaf(w[s + 1], src[(s + 1) * step], s1);
-      s2 = fmaf(w[s + 2], src[(s + 2) * step], s2);
-      s3 = fmaf(w[s + 3], src[(s + 3) * step], s3);
+    float acc = 0.0f;
+    for (int s0 = 0; s0 < a.Sv; s0 += 8) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = s0 + u < a.Sv ? src[(s0 + u) * step] : 0.0f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (s0 + u < a.Sv) acc = fmaf(w[s0 + u], x[u], acc);
     }
-    for (; s < a.Sv; ++s) s0 = fmaf(w[s], src[s * step], s0);
-    hc[h * kBvCRows + n] = (s0 + s1) + (s2 + s3);
+    hc[h * kBvCRows + n] = acc;
   }
   cp_async_wait<0>();
   __syncthreads();
@@ -444,9 +565,17 @@ void bv_geometry(int B, int Nc, int S, int& K, int& Sv) {
   Sv = (S + K - 1) / K;
 }
 
+// Parts per value split in the weights kernel: about two CTAs per SM in all.
+int bv_parts(int B, int Sv) {
+  const DeviceInfo di = current_device_info();
+  const int sms = di.sms > 0 ? di.sms : 148;
+  int P = 2 * sms / (B * Sv);
+  return P < 1 ? 1 : (P > 16 ? 16 : P);
+}
+
 struct BvLayout {
-  size_t attend_bytes, hpart_off, mlpart_off, opart_off, ml_off, total;
-  int S, K, Sv;
+  size_t attend_bytes, wts_off, mvec_off, lpart_off, hpart_off, opart_off, ml_off, total;
+  int S, K, Sv, P;
 };
 
 BvLayout bv_layout(const commvq_config* cfg, int Nc, int B, int64_t max_T, const commvq_attend_options* o) {
@@ -454,9 +583,13 @@ BvLayout bv_layout(const commvq_config* cfg, int Nc, int B, int64_t max_T, const
   L.attend_bytes = commvq_attend_workspace_bytes(cfg, B, max_T, o);
   L.S = mma_splits(B > 0 ? B : 1, cfg->q_heads, max_T);
   bv_geometry(B > 0 ? B : 1, Nc, L.S, L.K, L.Sv);
-  L.hpart_off = round_up(L.attend_bytes, 256);
-  L.mlpart_off = round_up(L.hpart_off + static_cast<size_t>(B) * L.Sv * cfg->q_heads * Nc * sizeof(float), 256);
-  L.opart_off = round_up(L.mlpart_off + static_cast<size_t>(B) * L.Sv * cfg->q_heads * sizeof(float2), 256);
+  L.P = bv_parts(B > 0 ? B : 1, L.Sv);
+  const size_t n_tiles = static_cast<size_t>((max_T + kBvTile - 1) / kBvTile);
+  L.wts_off = round_up(L.attend_bytes, 1024);
+  L.mvec_off = round_up(L.wts_off + static_cast<size_t>(B) * n_tiles * kBvWTile, 256);
+  L.lpart_off = round_up(L.mvec_off + static_cast<size_t>(B) * L.Sv * cfg->q_heads * sizeof(float), 256);
+  L.hpart_off = round_up(L.lpart_off + static_cast<size_t>(B) * L.Sv * L.P * cfg->q_heads * sizeof(float), 256);
+  L.opart_off = round_up(L.hpart_off + static_cast<size_t>(B) * L.Sv * cfg->q_heads * Nc * sizeof(float), 256);
   L.ml_off = round_up(L.opart_off + static_cast<size_t>(B) * cfg->q_heads * (Nc / kBvCRows) * kD * sizeof(float), 256);
   L.total = round_up(L.ml_off + static_cast<size_t>(B) * cfg->q_heads * sizeof(float2), 256);
   return L;
@@ -531,7 +664,9 @@ extern "C" commvq_status commvq_attend_decode_binv(const commvq_config* cfg, con
   v.bits = v_bits;
   v.C = v_codebook;
   v.hpart = reinterpret_cast<float*>(ws + L.hpart_off);
-  v.mlpart = reinterpret_cast<float2*>(ws + L.mlpart_off);
+  v.wts = ws + L.wts_off;
+  v.mvec = reinterpret_cast<float*>(ws + L.mvec_off);
+  v.lpart = reinterpret_cast<float*>(ws + L.lpart_off);
   v.opart = reinterpret_cast<float*>(ws + L.opart_off);
   v.ml = reinterpret_cast<float2*>(ws + L.ml_off);
   v.out = out;
@@ -545,10 +680,13 @@ extern "C" commvq_status commvq_attend_decode_binv(const commvq_config* cfg, con
   v.S = L.S;
   v.K = L.K;
   v.Sv = L.Sv;
+  v.P = L.P;
   if (cudaFuncSetAttribute(binv_accumulate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kBvTcSmem)) != cudaSuccess ||
       cudaFuncSetAttribute(binv_merge_contract_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kBvMcSmem)) != cudaSuccess)
+    return COMMVQ_ERR_CUDA;
+  if (launch_dependent(binv_weights_kernel, dim3(L.Sv, L.P, B), dim3(256), 0, st, v) != cudaSuccess)
     return COMMVQ_ERR_CUDA;
   if (launch_dependent(binv_accumulate_kernel, dim3(L.Sv, n_bits / kBvBitsPerCta, B), dim3(kBvThreads), kBvTcSmem,
                        st, v) != cudaSuccess)
