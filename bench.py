@@ -444,37 +444,47 @@ def run_ours(args, w, rank, world, dev):
 
 def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, attend, stream, dev, torch, api,
             synth, world, dist):
-    """Per step: pinned host -> device copy of the step's query and the new position's K/V
-    rows, encode of the new position into the cache (position T-1 of sequence 0), decode
+    """Per step: one pinned host -> device copy of the step's inputs (the query, the new
+    position's K and V rows, and for the binary value code its bits), encode of the new position
+    into the cache (position T-1 of sequence 0; the K and V encodes run on two streams), decode
     attention, device -> host copy of the output."""
     K, W = args.steps, args.warmup
     n_copies = len(kcs)
-    q_h = torch.from_numpy(synth.queries(w).view(np.int16) if w.q_dtype == "bf16"
-                           else synth.queries(w).astype(np.float32)).pin_memory()
+    binv = w.v_bits > 0
+    q_np = synth.queries(w).view(np.int16) if w.q_dtype == "bf16" else synth.queries(w).astype(np.float32)
     kv_new = np.stack([synth.kv_rows(w, True, 1, sub=1000, dtype="f16"),
                        synth.kv_rows(w, False, 1, sub=1000, dtype="f16")])   # [2, 1, Hkv, d]
-    kv_h = torch.from_numpy(kv_new).pin_memory()
-    binv = w.v_bits > 0
-    bits_h = torch.from_numpy(synth.value_bits(w, 1)).pin_memory() if binv else None
-    bits_d = torch.empty(bits_h.shape, dtype=torch.uint8, device=dev) if binv else None
+    parts = [q_np, kv_new] + ([synth.value_bits(w, 1)] if binv else [])
+    sizes = [int(x.nbytes) for x in parts]
+    offsets = np.concatenate([[0], np.cumsum([(n + 255) // 256 * 256 for n in sizes])])   # 256-byte aligned
+    stage_h = torch.zeros(int(offsets[-1]), dtype=torch.uint8).pin_memory()
+    for x, o, n in zip(parts, offsets, sizes):
+        stage_h[int(o):int(o) + n] = torch.from_numpy(np.ascontiguousarray(x).view(np.uint8).reshape(-1))
+    stage_d = torch.empty_like(stage_h, device=dev)
+
+    def view(k, dtype, shape):
+        return stage_d[int(offsets[k]):int(offsets[k]) + sizes[k]].view(dtype).view(shape)
+
+    q_d = view(0, torch.bfloat16 if w.q_dtype == "bf16" else torch.float32, q_np.shape)
+    kv_d = view(1, torch.float16, kv_new.shape)
+    bits_d = view(2, torch.uint8, (1, w.v_bits // 8)) if binv else None
     out_h = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32).pin_memory()
-    q_d = torch.empty(q_h.shape, dtype=q_h.dtype, device=dev)
-    kv_d = torch.empty(kv_h.shape, dtype=kv_h.dtype, device=dev)
     out_d = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32, device=dev)
     last = int(w.offsets()[1]) - 1
-    qv = q_d.view(torch.bfloat16) if w.q_dtype == "bf16" else q_d
+    side = torch.cuda.Stream(device=dev)
 
     def step(i):
         kc, vc = kcs[i % n_copies], vcs[i % n_copies]
-        q_d.copy_(q_h, non_blocking=True)
-        kv_d.copy_(kv_h, non_blocking=True)
+        stage_d.copy_(stage_h, non_blocking=True)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):   # the value row's code, beside the key row's
+            if binv:   # the value encoder is a learned network: its bits arrive from the host
+                vc[last:last + 1].copy_(bits_d, non_blocking=True)
+            else:
+                api.encode(cfg, kv_d[1], vcb, codes=vc[last:last + 1], stream=side)
         api.encode(cfg, kv_d[0], kcb, codes=kc[last:last + 1], stream=stream)
-        if binv:   # the value encoder is a learned network: its bits arrive from the host
-            bits_d.copy_(bits_h, non_blocking=True)
-            vc[last:last + 1].copy_(bits_d, non_blocking=True)
-        else:
-            api.encode(cfg, kv_d[1], vcb, codes=vc[last:last + 1], stream=stream)
-        attend(kc, vc, qv, out_d, None, i=i)
+        stream.wait_stream(side)
+        attend(kc, vc, q_d, out_d, None, i=i)
         out_h.copy_(out_d, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -498,11 +508,11 @@ def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, attend, stre
     ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     del graph
     return {"value": job_throughput(world, K, total_T, ms), "unit": UNIT,
-            "h2d_bytes_per_step": int(q_h.numel() * q_h.element_size() + kv_h.numel() * kv_h.element_size()
-                                      + (bits_h.numel() if binv else 0)),
+            "h2d_bytes_per_step": int(stage_h.numel()),
             "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()),
             "ms_per_step": ms / K,
-            "note": "q + new position's K/V rows in, encode + attend, output out; one CUDA graph of K steps"}
+            "note": "one copy of q + the new position's K/V rows (+ value bits) in, encode (K and V on two "
+                    "streams) + attend, output out; one CUDA graph of K steps"}
 
 
 # ---------------------------------------------------------------------------------------
