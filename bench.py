@@ -73,16 +73,19 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-KERNEL_SOURCES = {"attend_table_kernel": "attend_table.cu",
-                  "attend_scores_kernel+attend_values_kernel": "attend_mma.cu",
-                  "attend_generic_kernel": "attend_generic.cu",
-                  "dense_decode_kernel": "naive.cu"}
+KERNEL_SOURCES = {"attend_table_kernel": ("attend_table.cu",),
+                  "attend_scores_kernel+attend_values_kernel": ("attend_mma.cu",),
+                  "attend_scores_kernel+binv_*": ("attend_mma.cu", "binv.cu"),
+                  "attend_generic_kernel": ("attend_generic.cu",),
+                  "dense_decode_kernel": ("naive.cu",)}
 
 
 def kernel_source_sha(kernel: str):
-    src = os.path.join(ROOT, "decode_attention_commvq_b200", "csrc", KERNEL_SOURCES[kernel])
-    with open(src, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "decode_attention_commvq_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, workload_name: str):

@@ -187,3 +187,24 @@ def test_prepared_workspace_reuse(api, gpu):
     out1, lse1 = _run(api, w, q, kc, bits, offs, kcb, C, gpu, workspace=ws, prepared=True)
     assert np.array_equal(out0, out1) and np.array_equal(lse0, lse1)
     assert api.workspace_error(ws) == 0
+
+
+def test_many_waves_of_ctas(api, gpu):
+    """8192 value bits (32 slices of 256 rows) for 20 sequences of 1 KV head x 8 query heads:
+    ~640 CTAs of the bit-plane kernel, several per SM in turn, each holding all of tensor
+    memory while it runs."""
+    rng = np.random.default_rng(77)
+    lens = rng.integers(1, 300, size=20)
+    w = synth.Workload(name="binv_waves", seed=77, R=2, n_codes=256, q_heads=8, kv_heads=1, batch=20,
+                       seq_len=300, n_outliers=0, codebook="normal", v_bits=8192)
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    N = int(offs[-1])
+    kcb = synth.normal_codebook(w, True)
+    kc = synth.uniform_codes(w, True, N)
+    bits = synth.value_bits(w, N)
+    C = synth.binary_value_codebook(w)
+    q = synth.queries(w)
+    out, lse = _run(api, w, q, kc, bits, offs, kcb, C, gpu)
+    ref, ref_lse = O.attend_binv(q_as_f64(w, q), kc, bits, offs, kcb, C, w.rope_base)
+    assert rel_err(out, ref) <= tol_for(w)
+    assert np.allclose(lse, ref_lse, rtol=1e-3, atol=5e-3)
