@@ -404,8 +404,8 @@ def run_ours(args, w, rank, world, dev):
         kname, launches_per_step = "dense_decode_kernel", 4   # decompress prep, decompress, dense, merge
         alg_bytes = 2 * k_rows.numel() * k_rows.element_size()
     else:
-        if binv:   # scores, bit accumulation, split merge, contraction with C
-            kname, launches_per_step = "attend_scores_kernel+binv_*", 4
+        if binv:   # scores, weights, bit-plane sums, merge and contraction with C, final division
+            kname, launches_per_step = "attend_scores_kernel+binv_*", 5
         else:
             kname, launches_per_step = main_kernel(api, cfg, args.algo)
         if not prepared and kname.startswith("attend_scores"):
