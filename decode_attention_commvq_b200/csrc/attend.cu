@@ -46,7 +46,8 @@ constexpr int kMaxSplits = 4096;
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(AttendArgs a, int S) {
   __shared__ float4 acc_s[kCombineGroups][8];
   __shared__ float ml_s[kCombineGroups][2];
-  pdl_wait();   // launched as a dependent of the kernel that writes the partials
+  pdl_trigger();   // the next decode step's scores kernel may copy its codebook image meanwhile
+  pdl_wait();      // launched as a dependent of the kernel that writes the partials
   const int bh = blockIdx.x, quarter = blockIdx.y;
   const int tid = threadIdx.x, grp = tid >> 3, gl = tid & 7;
   const Partial* p = a.partials + static_cast<int64_t>(bh) * S;

@@ -266,6 +266,15 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
   split_range(a, b, s, S, row0, t_begin, t_end);
   Partial* part = a.partials + static_cast<int64_t>(b) * a.q_heads * S + s;   // + h * S
 
+  // The prepared codebook image and advance phasors are not written by the kernel this one may
+  // be a programmatic dependent of (the previous decode step's combine): copy them first, then
+  // wait for that kernel before touching anything else.
+  if (t_begin < t_end) {
+    for (int p = tid; p < 32 * Nc; p += kMmaThreads) cp_async16(cbk + p, a.k_img + p);
+    if (tid < kD / 4) cp_async16(reinterpret_cast<uint4*>(advs) + tid, reinterpret_cast<const uint4*>(a.advph) + tid);
+  }
+  cp_async_commit();
+  pdl_wait();
   if (t_begin >= t_end) {
     for (int h = tid; h < a.q_heads; h += kMmaThreads) part[static_cast<int64_t>(h) * S].m = -INFINITY;
     return;
@@ -289,11 +298,8 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
       cp_async16(wstage + buf * kWarpStage + (row * kRowPieces + (piece ^ (row & kRowSwz))) * 16, src + p * 16);
     }
   };
-  // Set-up: asynchronous copies of the prepared codebook image and advance phasors, then the
-  // warp's first rows; meanwhile the query fragments and the split's base phasor are formed.
-  for (int p = tid; p < 32 * Nc; p += kMmaThreads) cp_async16(cbk + p, a.k_img + p);
-  if (tid < kD / 4) cp_async16(reinterpret_cast<uint4*>(advs) + tid, reinterpret_cast<const uint4*>(a.advph) + tid);
-  cp_async_commit();
+  // Set-up: the warp's first rows (the image is on its way); meanwhile the query fragments and
+  // the split's base phasor are formed.
   if (t_begin + warp * kRows < t_end) issue_rows(0, t_begin);
   cp_async_commit();
   // Query fragments of this sequence in the mma k-order: entry (kv, k-step st, lane) holds, for
@@ -707,7 +713,8 @@ commvq_status launch_mma_rk(const AttendArgs& a, const void* q, commvq_dtype qt,
     auto k = attend_scores_kernel<R, KV, NC, T>;                                               \
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s) != cudaSuccess) \
       return COMMVQ_ERR_CUDA;                                                                      \
-    k<<<grid, kMmaThreads, smem_s, st>>>(a, static_cast<const T*>(q));                             \
+    if (launch_dependent(k, grid, dim3(kMmaThreads), smem_s, st, a, static_cast<const T*>(q)) != cudaSuccess) \
+      return COMMVQ_ERR_CUDA;                                                                      \
   }
   switch (qt) {
     case COMMVQ_F32: COMMVQ_LAUNCH_SCORES(float) break;

@@ -542,6 +542,7 @@ __global__ void __launch_bounds__(256) binv_merge_contract_kernel(BinvArgs a) {
 // out[b, h, :] = sum over chunks / L; lse = (M + log2 L) ln 2 (-inf and a zero row when empty).
 __global__ void __launch_bounds__(kD) binv_finalize_kernel(BinvArgs a) {
   const int bh = blockIdx.x, d = threadIdx.x;
+  pdl_trigger();   // the next decode step's scores kernel may copy its codebook image meanwhile
   pdl_wait();
   const int nch = a.Nc / kBvCRows;
   const float* src = a.opart + static_cast<int64_t>(bh) * nch * kD + d;
