@@ -6,14 +6,19 @@
 //
 // Because v_t is linear in s_t, the softmax weights can be folded into the bits first:
 //   out_h = (sum_t p_{h,t} s_t) C[:, slice of h's KV head] / sum_t p_{h,t}.
-// Kernel 1 (grid: position splits x 256-bit slices x sequences) forms the per-split sums
-// H_v[h, n] = sum_t 2^(score - m_v) s_t[n] with tcgen05 MMAs, as H_v^T = S^T P^T: A = the bits of
-// 128 codebook rows (M) for 16 positions (K), expanded to fp16 0 / 1 and stored into tensor memory;
-// B = the weights of all 32 query-head columns (N) in shared memory; D accumulates in tensor
-// memory. A split is a run of whole splits of the scores kernel, so its maximum m_v is the maximum
-// of their maxima and every weight is at most 1. Kernel 2 (grid: KV heads x 128-row chunks of C)
-// merges the splits' H with log-sum-exp weights and contracts its chunk with C; kernel 3 sums the
-// chunks and divides by the softmax sum.
+// After the scores kernel, four kernels:
+// * weights (grid: value splits x parts x sequences): p = 2^(score - m_v) once per value split, as
+//   24-bit fixed point in three 8-bit digits laid out as an MMA operand. A value split is a run
+//   of whole splits of the scores kernel, so m_v is the maximum of their maxima and p <= 1.
+// * accumulate (grid: value splits x 256-bit slices x sequences): the per-split sums
+//   H_v^T[n, h] = sum_t s_t[n] p_{h,t} with tcgen05 kind::i8 MMAs and exact int32 sums: A = the
+//   bits of 128 codebook rows (M) for 32 positions (K) as bytes 0 / 1 in tensor memory, B = one
+//   digit plane of the weights of all 32 query-head columns (N) in shared memory, D in tensor
+//   memory.
+// * merge and contract (grid: KV heads x 64-row chunks of C): the splits' H merged with
+//   log-sum-exp weights and contracted with the chunk of C.
+// * finalize (grid: sequences x query heads): the chunks summed in order and divided by the
+//   softmax sum.
 #include <math.h>
 
 #include "attend.cuh"

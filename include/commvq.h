@@ -267,8 +267,9 @@ size_t commvq_attend_binv_workspace_bytes(const commvq_config* cfg, int32_t n_bi
  *   s_t (keys) as in commvq_attend_decode, p = softmax(s),
  *   out[b,h] = sum_t p_t (s_t^T C)[kvh * 128 : kvh * 128 + 128], kvh = h / (q_heads / kv_heads),
  *   lse as in commvq_attend_decode.
- * The softmax weights are folded into the bits first (H_h = sum_t p_t s_t on the tensor cores,
- * bits expanded to fp16 0 / 1), then H_h is contracted with C in fp32.
+ * The softmax weights are folded into the bits first, H_h = sum_t p_t s_t on the tensor cores
+ * (int8 MMAs: bits as bytes 0 / 1, each weight as 24-bit fixed point in three 8-bit digits,
+ * exact int32 sums; a weight carries 2^-25 absolute error), then H_h is contracted with C in fp32.
  * v_bits      [total_T, n_bits / 8] uint8, bit n of position t = byte n/8, bit n%8 (least
  *             significant first), 16-byte aligned.
  * v_codebook  C [n_bits, kv_heads * 128] float32.

@@ -3,10 +3,11 @@ over the whole KV dimension, v_t = s_t^T C): commvq_attend_decode_binv against t
 attention on decoded values, within the attention bounds of the other parity tests (2e-3 fp32
 query / 5e-3 bf16 query, max relative error per (b, h)).
 
-The key side is the decode-and-rotate scores kernel (same error as there); on the value side the
-softmax weights enter the tensor cores as fp16 (relative rounding <= 2^-11 each, independent
-signs), H = sum_t p_t s_t is accumulated in fp32 and contracted with the fp32 C in fp32, so the
-value side adds less than the fp16 value codebook of the CommVQ value path."""
+The key side is the decode-and-rotate scores kernel (same error as there). On the value side
+each softmax weight enters the tensor cores as 24-bit fixed point (absolute error <= 2^-25,
+i.e. at most fp16's relative 2^-11 for weights >= 2^-14), H = sum_t p_t s_t is summed exactly in
+int32 and contracted with the fp32 C in fp32, so the value side adds less than the fp16 value
+codebook of the CommVQ value path."""
 import numpy as np
 import pytest
 import torch
