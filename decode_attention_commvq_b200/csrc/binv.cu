@@ -498,19 +498,19 @@ __global__ void __launch_bounds__(256) binv_merge_contract_kernel(BinvArgs a) {
     if (chunk == 0) a.ml[static_cast<int64_t>(b) * a.Hq + kv * G + tid] = make_float2(M, L);
   }
   __syncthreads();
-  // merged H of the chunk: element (h, n), n fastest (coalesced); eight split sums in flight
+  // merged H of the chunk: element (h, n), n fastest (coalesced); sixteen split sums in flight
   for (int e = tid; e < G * kBvCRows; e += 256) {
     const int h = e / kBvCRows, n = e % kBvCRows;
     const float* src = a.hpart + (static_cast<int64_t>(b) * a.Sv * a.Hq + kv * G + h) * a.Nc + n0 + n;
     const int64_t step = static_cast<int64_t>(a.Hq) * a.Nc;
     const float* w = wts + h * kBvMaxSplits;
     float acc = 0.0f;
-    for (int s0 = 0; s0 < a.Sv; s0 += 8) {
-      float x[8];
+    for (int s0 = 0; s0 < a.Sv; s0 += 16) {
+      float x[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = s0 + u < a.Sv ? src[(s0 + u) * step] : 0.0f;
+      for (int u = 0; u < 16; ++u) x[u] = s0 + u < a.Sv ? src[(s0 + u) * step] : 0.0f;
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
+      for (int u = 0; u < 16; ++u)
         if (s0 + u < a.Sv) acc = fmaf(w[s0 + u], x[u], acc);
     }
     hc[h * kBvCRows + n] = acc;
@@ -571,12 +571,12 @@ void bv_geometry(int B, int Nc, int S, int& K, int& Sv) {
   Sv = (S + K - 1) / K;
 }
 
-// Parts per value split in the weights kernel: about two CTAs per SM in all.
+// Parts per value split in the weights kernel: about four CTAs per SM in all.
 int bv_parts(int B, int Sv) {
   const DeviceInfo di = current_device_info();
   const int sms = di.sms > 0 ? di.sms : 148;
-  int P = 2 * sms / (B * Sv);
-  return P < 1 ? 1 : (P > 16 ? 16 : P);
+  int P = 4 * sms / (B * Sv);
+  return P < 1 ? 1 : (P > 32 ? 32 : P);
 }
 
 struct BvLayout {
