@@ -48,3 +48,28 @@ def test_two_term_rotated_keys_keep_a_margin():
         two_term = max(two_term, rel_err(o2, ref))
     assert two_term <= 0.8 * TOL_BF16, two_term
     assert one_term > two_term
+
+
+def test_binary_value_weights_in_three_digits_add_almost_nothing():
+    """The binary value code's value side, emulated: each softmax weight p = 2^(s - m) <= 1 as
+    24-bit fixed point q = round(p (2^24 - 1)) in three 8-bit digits, the bit-plane sums
+    sum_t s_t[n] q_t exact in integers, the contraction with C in fp64 (the kernel's is fp32).
+    Against the exact attention on decoded values the output moves by far less than the bf16
+    tolerance: each weight is carried to 2^-25 absolute, so the relative change of the output is
+    at most ~2^-25 x (positions / sum of weights). Here it is 1.0e-7; fp16 weights would give
+    2.3e-5."""
+    rng = np.random.default_rng(79)
+    T, Nc, d = 3000, 2048, 128
+    s = rng.standard_normal(T) * 3.0                       # log2-domain scores, a few units apart
+    p = np.exp2(s - s.max())                               # split maximum: every weight <= 1
+    q = np.rint(p * (2 ** 24 - 1)).astype(np.int64)
+    digits = [(q >> sh) & 0xFF for sh in (16, 8, 0)]
+    assert np.array_equal(digits[0] * 65536 + digits[1] * 256 + digits[2], q)
+    bits = rng.integers(0, 2, size=(T, Nc), dtype=np.int64)
+    C = rng.standard_normal((Nc, d)) * np.sqrt(2.0 / Nc)
+    H_int = sum(bits.T @ dg * (256 ** (2 - i)) for i, dg in enumerate(digits))   # exact integers
+    out = (H_int / (2 ** 24 - 1)) @ C / p.sum()
+    ref = (bits.T @ p) @ C / p.sum()
+    err = np.abs(out - ref).max() / np.abs(ref).max()
+    assert err < 1e-5
+    assert err < TOL_BF16 / 100
