@@ -18,6 +18,9 @@
  *    per scalar (Eq. 21); the codebook is fit by EM (Algorithm 1, Eq. 20).
  *  - machine review, "If this is right": softmax weights multiply the value codes
  *    before the codebook multiply.
+ *  - machine review, "Assumptions & free parameters" and referee minor comment 4: the
+ *    paper's own value code is a bit vector s in {0,1}^Nc over a codebook of Nc rows
+ *    (Nc / d bits per scalar), decoded as s^T C (oracle_decode_bits).
  * Readings where the pages are silent (each is listed in the design notes):
  *  - a stored key pair (a, b) is the reconstructed 2-vector; its block is
  *    [[a, -b], [b, a]] (the pages' form with x = a, y = -b), so every stored pair
