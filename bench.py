@@ -75,6 +75,7 @@ def measured_peaks():
 
 KERNEL_SOURCES = {"attend_table_kernel": ("attend_table.cu",),
                   "attend_scores_kernel+attend_values_kernel": ("attend_mma.cu",),
+                  "fast_keys_kernel+fast_values_kernel": ("attend_fast.cu",),
                   "attend_scores_kernel+binv_*": ("attend_mma.cu", "binv.cu"),
                   "attend_generic_kernel": ("attend_generic.cu",),
                   "dense_decode_kernel": ("naive.cu",)}
@@ -111,6 +112,10 @@ def main_kernel(api, cfg, algo):
             cfg.q_heads % cfg.kv_heads == 0 and cfg.q_heads // cfg.kv_heads <= 8
         run = api.ATTN_DECODE_MMA if mma_ok else (api.ATTN_TABLE if g8 and cfg.R <= 4 else api.ATTN_GENERIC)
     if run == api.ATTN_DECODE_MMA:
+        fast = cfg.g == 8 and cfg.R <= 2 and cfg.n_codes <= 256 and cfg.kv_heads in (2, 4, 8) and \
+            cfg.q_heads % cfg.kv_heads == 0 and cfg.q_heads // cfg.kv_heads <= 8
+        if fast:
+            return "fast_keys_kernel+fast_values_kernel", 3     # keys, values, merge
         return "attend_scores_kernel+attend_values_kernel", 3   # scores, values, merge
     if run == api.ATTN_GENERIC:
         return "attend_generic_kernel", 3                       # phasor tables, generic, merge
@@ -408,7 +413,7 @@ def run_ours(args, w, rank, world, dev):
             kname, launches_per_step = "attend_scores_kernel+binv_*", 5
         else:
             kname, launches_per_step = main_kernel(api, cfg, args.algo)
-        if not prepared and kname.startswith("attend_scores"):
+        if not prepared and (kname.startswith("attend_scores") or kname.startswith("fast_keys")):
             launches_per_step += 1   # the prep kernel
         alg_bytes = code_bytes + (vcb.numel() * vcb.element_size() if binv else 0)
     achieved = alg_bytes / (kern_ms / 1e3) / 1e9
@@ -449,7 +454,7 @@ def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, attend, stre
             synth, world, dist):
     """Per step: one pinned host -> device copy of the step's inputs (the query, the new
     position's K and V rows, and for the binary value code its bits), encode of the new position
-    into the cache (position T-1 of sequence 0; the K and V encodes run on two streams), decode
+    into the cache (position T-1 of sequence 0; its K and V rows in one encode launch), decode
     attention, device -> host copy of the output."""
     K, W = args.steps, args.warmup
     n_copies = len(kcs)
@@ -474,19 +479,15 @@ def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, attend, stre
     out_h = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32).pin_memory()
     out_d = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32, device=dev)
     last = int(w.offsets()[1]) - 1
-    side = torch.cuda.Stream(device=dev)
 
     def step(i):
         kc, vc = kcs[i % n_copies], vcs[i % n_copies]
         stage_d.copy_(stage_h, non_blocking=True)
-        side.wait_stream(stream)
-        with torch.cuda.stream(side):   # the value row's code, beside the key row's
-            if binv:   # the value encoder is a learned network: its bits arrive from the host
-                vc[last:last + 1].copy_(bits_d, non_blocking=True)
-            else:
-                api.encode(cfg, kv_d[1], vcb, codes=vc[last:last + 1], stream=side)
-        api.encode(cfg, kv_d[0], kcb, codes=kc[last:last + 1], stream=stream)
-        stream.wait_stream(side)
+        if binv:   # the value encoder is a learned network: its bits arrive from the host
+            vc[last:last + 1].copy_(bits_d, non_blocking=True)
+            api.encode(cfg, kv_d[0], kcb, codes=kc[last:last + 1], stream=stream)
+        else:      # the new key and value rows in one launch
+            api.encode_kv(cfg, kv_d[0], kv_d[1], kcb, vcb, kc[last:last + 1], vc[last:last + 1], stream=stream)
         attend(kc, vc, q_d, out_d, None, i=i)
         out_h.copy_(out_d, non_blocking=True)
 
@@ -514,8 +515,8 @@ def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, attend, stre
             "h2d_bytes_per_step": int(stage_h.numel()),
             "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()),
             "ms_per_step": ms / K,
-            "note": "one copy of q + the new position's K/V rows (+ value bits) in, encode (K and V on two "
-                    "streams) + attend, output out; one CUDA graph of K steps"}
+            "note": "one copy of q + the new position's K/V rows (+ value bits) in, encode (K and V rows in one "
+                    "launch) + attend, output out; one CUDA graph of K steps"}
 
 
 # ---------------------------------------------------------------------------------------

@@ -22,7 +22,7 @@ ATTEND_PREPARED = 1
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "WORKSPACE", 5: "DEVICE_CHECK"}
 
-EXPORTS = ("commvq_encode", "commvq_attend_workspace_bytes", "commvq_attend_decode", "commvq_attend_prepare",
+EXPORTS = ("commvq_encode", "commvq_encode_kv", "commvq_attend_workspace_bytes", "commvq_attend_decode", "commvq_attend_prepare",
            "commvq_attend_decode_noalloc", "commvq_em_workspace_bytes", "commvq_em_step",
            "commvq_em_step_soft", "commvq_decompress_workspace_bytes", "commvq_decompress",
            "commvq_dense_decode_workspace_bytes", "commvq_dense_decode",
@@ -59,6 +59,8 @@ def _load():
     OP = ctypes.POINTER(CAttendOptions)
     lib.commvq_encode.argtypes = [CP, P, I32, I64, P, P, P, P, P]
     lib.commvq_encode.restype = I32
+    lib.commvq_encode_kv.argtypes = [CP, P, P, I32, I64, P, P, P, P, P, P]
+    lib.commvq_encode_kv.restype = I32
     lib.commvq_attend_workspace_bytes.argtypes = [CP, I32, I64, OP]
     lib.commvq_attend_workspace_bytes.restype = SZ
     lib.commvq_attend_decode.argtypes = [CP, P, I32, P, P, P, I32, I64, P, P, P, P, P, SZ, OP, P]
@@ -158,6 +160,20 @@ def encode(cfg: Config, x: torch.Tensor, codebook: torch.Tensor, codes: Optional
                              _ptr(codes), _ptr(near_ties), _ptr(residual_out), _stream(stream)),
            "commvq_encode")
     return codes
+
+
+def encode_kv(cfg: Config, k_x: torch.Tensor, v_x: torch.Tensor, k_codebook: torch.Tensor,
+              v_codebook: torch.Tensor, k_codes: torch.Tensor, v_codes: torch.Tensor,
+              near_ties: Optional[torch.Tensor] = None, stream=None):
+    """commvq_encode_kv: the key rows k_x and value rows v_x [T, kv_heads, d] (same shape and dtype)
+    into k_codes / v_codes [T, kv_heads, R, d/g] in one launch."""
+    if k_x.shape != v_x.shape or k_x.dtype != v_x.dtype:
+        raise ValueError("k_x and v_x must have the same shape and dtype")
+    cc = cfg.c()
+    _check(LIB.commvq_encode_kv(ctypes.byref(cc), _ptr(k_x), _ptr(v_x), _DT[k_x.dtype], int(k_x.shape[0]),
+                                _ptr(k_codebook), _ptr(v_codebook), _ptr(k_codes), _ptr(v_codes), _ptr(near_ties),
+                                _stream(stream)), "commvq_encode_kv")
+    return k_codes, v_codes
 
 
 def _opts(algo: int, splits: int, events=None, flags: int = 0) -> CAttendOptions:

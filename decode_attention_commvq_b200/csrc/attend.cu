@@ -50,6 +50,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(AttendArgs a, 
   pdl_wait();      // launched as a dependent of the kernel that writes the partials
   const int bh = blockIdx.x, quarter = blockIdx.y;
   const int tid = threadIdx.x, grp = tid >> 3, gl = tid & 7;
+  if (bh == 0 && quarter == 0 && tid == 0 && a.error_word) publish_error(a.error_word);   // the call's last kernel
   const Partial* p = a.partials + static_cast<int64_t>(bh) * S;
   const int dim4 = quarter * 8 + gl;   // float4 index within o[128]
 
@@ -180,22 +181,41 @@ int partial_slots(const commvq_config* cfg, int algo, int S) {
 struct WorkspaceLayout {
   size_t partials_off, kimg_off, vimg_off, phase_off, scores_off, tables_off, total;
 };
-constexpr size_t kPhaseBytes = 64 * sizeof(double) + 128 * 64 * 8 + 64 * 8;   // theta, rows, advance
+// theta, rows, advance: attend_mma.cu's tables (128 offset rows); the fast kernels' (64 rows) fit
+constexpr size_t kPhaseBytes = 64 * sizeof(double) + 128 * 64 * 8 + 64 * 8;
 
-WorkspaceLayout workspace_layout(const commvq_config* cfg, int algo, int B, int64_t max_T, int S) {
+void set_phase_tables(AttendArgs& a, unsigned char* base, bool fast) {
+  a.theta = reinterpret_cast<const double*>(base);
+  a.rowph = reinterpret_cast<const float4*>(base + 64 * sizeof(double));
+  a.advph = a.rowph + (fast ? 64 * 64 / 2 : 128 * 32);   // float4 units: 64 x 64 (cos, sin) or 128 x 32
+}
+
+bool use_fast(const commvq_config* cfg) {
+  return fast_supported(cfg->g, cfg->R, cfg->q_heads, cfg->kv_heads, cfg->n_codes);
+}
+
+// The prepared state (codebook images, RoPE tables) depends only on cfg and the codebooks, so
+// it sits at fixed offsets right after the header: a workspace prepared once stays valid for
+// any B, max_T and split count that fit in it. Per-call buffers (partials, scores) follow.
+// fast: the fast kernels' image size (128 KB each); otherwise attend_mma.cu's (512 Nc' bytes).
+WorkspaceLayout workspace_layout(const commvq_config* cfg, int algo, int B, int64_t max_T, int S, bool fast) {
   WorkspaceLayout L{};
-  L.partials_off = kHeaderBytes;
-  size_t end = L.partials_off + static_cast<size_t>(B) * cfg->q_heads * partial_slots(cfg, algo, S) * sizeof(Partial);
+  size_t end = kHeaderBytes;
+  if (algo == COMMVQ_ATTN_DECODE_MMA) {
+    const size_t img = fast ? static_cast<size_t>(131072) : static_cast<size_t>(512) * cfg->n_codes;
+    L.kimg_off = end;
+    L.vimg_off = round_up(L.kimg_off + img, 256);
+    L.phase_off = round_up(L.vimg_off + img, 256);
+    end = round_up(L.phase_off + kPhaseBytes, 256);
+  }
+  L.partials_off = end;
+  end = L.partials_off + static_cast<size_t>(B) * cfg->q_heads * partial_slots(cfg, algo, S) * sizeof(Partial);
   if (algo == COMMVQ_ATTN_GENERIC) {
     L.tables_off = round_up(end, 256);
     end = L.tables_off + generic_tables_bytes(max_T);
   }
   if (algo == COMMVQ_ATTN_DECODE_MMA) {
-    const size_t img = static_cast<size_t>(512) * cfg->n_codes;
-    L.kimg_off = round_up(end, 256);
-    L.vimg_off = round_up(L.kimg_off + img, 256);
-    L.phase_off = round_up(L.vimg_off + img, 256);
-    L.scores_off = round_up(L.phase_off + kPhaseBytes, 256);
+    L.scores_off = round_up(end, 256);
     end = L.scores_off + static_cast<size_t>(B) * ((max_T + 15) / 16 * 16) * cfg->q_heads * sizeof(float);
   }
   L.total = round_up(end, 256);
@@ -229,7 +249,7 @@ extern "C" size_t commvq_attend_workspace_bytes(const commvq_config* cfg, int32_
   const int algo = resolve_algo(cfg, options);
   if (!algo_supported(cfg, algo)) return 0;
   const int S = choose_splits(algo, B > 0 ? B : 1, cfg->q_heads, max_T, options);
-  return workspace_layout(cfg, algo, B, max_T, S).total;
+  return workspace_layout(cfg, algo, B, max_T, S, algo == COMMVQ_ATTN_DECODE_MMA && use_fast(cfg)).total;
 }
 
 extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const void* q,
@@ -262,7 +282,12 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
 
   const DeviceInfo di = current_device_info();
   if (di.device < 0) return COMMVQ_ERR_CUDA;
-  if (run == COMMVQ_ATTN_DECODE_MMA) {
+  const bool fast = run == COMMVQ_ATTN_DECODE_MMA && use_fast(cfg);
+  if (fast) {
+    if (fast_keys_smem_bytes(cfg->R, cfg->kv_heads) > di.smem_optin ||
+        fast_values_smem_bytes(cfg->R, cfg->kv_heads, cfg->q_heads) > di.smem_optin)
+      return COMMVQ_ERR_UNSUPPORTED;
+  } else if (run == COMMVQ_ATTN_DECODE_MMA) {
     if (mma_scores_smem_bytes(cfg->R, cfg->kv_heads, cfg->n_codes) > di.smem_optin ||
         mma_values_smem_bytes(cfg->R, cfg->kv_heads, cfg->q_heads, cfg->n_codes) > di.smem_optin)
       return COMMVQ_ERR_UNSUPPORTED;
@@ -271,7 +296,7 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
   }
 
   const int S = choose_splits(run, B, cfg->q_heads, max_T, options);
-  const WorkspaceLayout L = workspace_layout(cfg, run, B, max_T, S);
+  const WorkspaceLayout L = workspace_layout(cfg, run, B, max_T, S, fast);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   AttendArgs a{};
   a.k_codes = static_cast<const uint8_t*>(k_codes);
@@ -287,9 +312,7 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
     a.k_img = reinterpret_cast<const uint4*>(ws + L.kimg_off);
     a.v_img = reinterpret_cast<const uint4*>(ws + L.vimg_off);
     a.scores = reinterpret_cast<float*>(ws + L.scores_off);
-    a.theta = reinterpret_cast<const double*>(ws + L.phase_off);
-    a.rowph = reinterpret_cast<const float4*>(ws + L.phase_off + 64 * sizeof(double));
-    a.advph = a.rowph + 128 * 32;
+    set_phase_tables(a, ws + L.phase_off, fast);
   }
   a.main_start = options ? options->main_start : nullptr;
   a.main_stop = options ? options->main_stop : nullptr;
@@ -304,19 +327,24 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool prepared = options && (options->flags & COMMVQ_ATTEND_PREPARED);
   commvq_status rc;
-  if (run == COMMVQ_ATTN_DECODE_MMA) {
+  if (fast) {
     if (!prepared) {
-      rc = launch_attend_prep(a, st);   // also clears the error word
+      rc = launch_fast_prep(a, st);   // also clears the error words
       if (rc != COMMVQ_OK) return rc;
-    } else if (cfg->n_codes < 256 &&   // codes can be out of range: this call's word starts clear
-               cudaMemsetAsync(a.error_word, 0, sizeof(int), st) != cudaSuccess) {
-      return COMMVQ_ERR_CUDA;
-    }
+    }   // else: the previous call's merge left the running error word clear
+    // the keys kernel copies the prepared state before its dependency wait: launch it as a
+    // programmatic dependent only when the kernel before it is not the one writing that state
+    rc = launch_attend_fast(a, q, q_dtype, S, st, prepared);
+  } else if (run == COMMVQ_ATTN_DECODE_MMA) {
+    if (!prepared) {
+      rc = launch_attend_prep(a, st);   // also clears the error words
+      if (rc != COMMVQ_OK) return rc;
+    }   // else: the previous call's merge left the running error word clear
     rc = launch_attend_mma(a, q, q_dtype, S, st);
   } else if (run == COMMVQ_ATTN_GENERIC) {
     rc = launch_attend_generic(a, cfg, q, q_dtype, S, ws + L.tables_off, st);   // clears the error word
   } else {
-    if (cudaMemsetAsync(a.error_word, 0, sizeof(int), st) != cudaSuccess) return COMMVQ_ERR_CUDA;
+    if (cudaMemsetAsync(a.error_word, 0, 2 * sizeof(int), st) != cudaSuccess) return COMMVQ_ERR_CUDA;
     // Timing events around the main kernel (external event nodes when the stream is captured).
     if (a.main_start && record_event(a.main_start, st) != cudaSuccess)
       return COMMVQ_ERR_CUDA;
@@ -354,18 +382,17 @@ extern "C" commvq_status commvq_attend_prepare(const commvq_config* cfg, int32_t
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   if (run != COMMVQ_ATTN_DECODE_MMA)
-    return cudaMemsetAsync(workspace, 0, sizeof(int), st) == cudaSuccess ? COMMVQ_OK : COMMVQ_ERR_CUDA;
+    return cudaMemsetAsync(workspace, 0, 2 * sizeof(int), st) == cudaSuccess ? COMMVQ_OK : COMMVQ_ERR_CUDA;
   const int S = choose_splits(run, B, cfg->q_heads, max_T, options);
-  const WorkspaceLayout L = workspace_layout(cfg, run, B, max_T, S);
+  const bool fast = use_fast(cfg);
+  const WorkspaceLayout L = workspace_layout(cfg, run, B, max_T, S, fast);
   AttendArgs a{};
   a.k_codebook = k_codebook;
   a.v_codebook = v_codebook;
   a.error_word = static_cast<int*>(workspace);
   a.k_img = reinterpret_cast<const uint4*>(ws + L.kimg_off);
   a.v_img = reinterpret_cast<const uint4*>(ws + L.vimg_off);
-  a.theta = reinterpret_cast<const double*>(ws + L.phase_off);
-  a.rowph = reinterpret_cast<const float4*>(ws + L.phase_off + 64 * sizeof(double));
-  a.advph = a.rowph + 128 * 32;
+  set_phase_tables(a, ws + L.phase_off, fast);
   a.max_T = max_T;
   a.rope_base = cfg->rope_base;
   a.B = B;
@@ -373,7 +400,7 @@ extern "C" commvq_status commvq_attend_prepare(const commvq_config* cfg, int32_t
   a.kv_heads = cfg->kv_heads;
   a.R = cfg->R;
   a.n_codes = cfg->n_codes;
-  return launch_attend_prep(a, st);
+  return fast ? launch_fast_prep(a, st) : launch_attend_prep(a, st);
 }
 
 namespace commvq {
@@ -386,7 +413,7 @@ int attend_mma_setup(const commvq_config* cfg, int B, int64_t max_T, unsigned ch
                      const int64_t* seq_offsets, const void* k_codes, const float* k_codebook, AttendArgs& a) {
   commvq_attend_options o{COMMVQ_ATTN_DECODE_MMA, 0, nullptr, nullptr, 0};
   const int S = choose_splits(COMMVQ_ATTN_DECODE_MMA, B, cfg->q_heads, max_T, &o);
-  const WorkspaceLayout L = workspace_layout(cfg, COMMVQ_ATTN_DECODE_MMA, B, max_T, S);
+  const WorkspaceLayout L = workspace_layout(cfg, COMMVQ_ATTN_DECODE_MMA, B, max_T, S, false);
   a.k_codes = static_cast<const uint8_t*>(k_codes);
   a.v_codes = static_cast<const uint8_t*>(k_codes);
   a.seq_offsets = seq_offsets;
@@ -397,9 +424,7 @@ int attend_mma_setup(const commvq_config* cfg, int B, int64_t max_T, unsigned ch
   a.k_img = reinterpret_cast<const uint4*>(ws + L.kimg_off);
   a.v_img = reinterpret_cast<const uint4*>(ws + L.vimg_off);
   a.scores = reinterpret_cast<float*>(ws + L.scores_off);
-  a.theta = reinterpret_cast<const double*>(ws + L.phase_off);
-  a.rowph = reinterpret_cast<const float4*>(ws + L.phase_off + 64 * sizeof(double));
-  a.advph = a.rowph + 128 * 32;
+  set_phase_tables(a, ws + L.phase_off, false);
   a.max_T = max_T;
   a.rope_base = cfg->rope_base;
   a.B = B;
@@ -439,7 +464,7 @@ extern "C" const char* commvq_status_string(commvq_status s) {
     case COMMVQ_ERR_UNSUPPORTED: return "shape or type not supported by this build";
     case COMMVQ_ERR_CUDA: return "CUDA runtime error";
     case COMMVQ_ERR_WORKSPACE: return "workspace missing or too small";
-    case COMMVQ_ERR_DEVICE_CHECK: return "device recorded a data error (code out of range)";
+    case COMMVQ_ERR_DEVICE_CHECK: return "device recorded a data error (code or sequence length out of range)";
     default: return "unknown status";
   }
 }

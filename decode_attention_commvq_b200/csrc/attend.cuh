@@ -69,6 +69,17 @@ __host__ __device__ inline int64_t score_slot(int64_t b, int64_t t, int kv, int 
 commvq_status launch_attend_table(const AttendArgs& a, const void* q, commvq_dtype qt, int splits,
                                   cudaStream_t st);
 commvq_status launch_combine(const AttendArgs& a, int splits, cudaStream_t st);
+// The fast decode-and-rotate kernels (attend_fast.cu): KV heads in {2, 4, 8}, up to 8 query heads
+// per KV head, R <= 2, Nc' <= 256, g = 8. Their prepared state is 128 KB per codebook image, RoPE
+// tables theta [64] fp64, offset rows [64][64] (cos, sin) and the 64-position advance [64].
+bool fast_supported(int g, int R, int q_heads, int kv_heads, int n_codes);
+size_t fast_keys_smem_bytes(int R, int KV);
+size_t fast_values_smem_bytes(int R, int KV, int q_heads);
+commvq_status launch_fast_prep(const AttendArgs& a, cudaStream_t st);
+// dependent: launch the keys kernel as a programmatic dependent of the previous kernel (only when
+// that kernel does not write the prepared state).
+commvq_status launch_attend_fast(const AttendArgs& a, const void* q, commvq_dtype qt, int splits, cudaStream_t st,
+                                 bool dependent);
 bool generic_supported(const commvq_config* cfg);
 int generic_warps_per_kv(int kv_heads);
 size_t generic_tables_bytes(int64_t max_T);

@@ -30,7 +30,7 @@ constexpr int kGenMaxG = 16;       // query heads per KV head
 // e^{i 128 h theta_p}, both from fp64 angles, in the packed layout of put_phasor.
 __global__ void generic_prep_kernel(float4* rowph, float4* coarse, int n_hi, double rope_base, int* error_word) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e == 0 && blockIdx.y == 0) *error_word = 0;
+  if (e == 0 && blockIdx.y == 0) error_word[0] = error_word[1] = 0;
   const int p = e % (kD / 2), row = e / (kD / 2);
   const double th = pow(rope_base, -2.0 * p / kD);
   double sn, cs;
@@ -105,9 +105,8 @@ __global__ void __launch_bounds__(kGenThreads) attend_generic_kernel(GenericArgs
   const int kv = warp / wpk, sub = warp % wpk;
   const int j = (4 * lane) / a.g, off = (4 * lane) % a.g;
 
-  const int64_t row0 = a.seq_offsets[b];
-  int64_t Tb = a.seq_offsets[b + 1] - row0;
-  Tb = Tb < 0 ? 0 : (Tb > a.max_T ? a.max_T : Tb);
+  int64_t row0;
+  const int64_t Tb = sequence_rows(a.seq_offsets, b, a.max_T, running_error(a.error_word), row0);
   int64_t per = (Tb + S - 1) / S;
   const int64_t t_begin = min(Tb, static_cast<int64_t>(s) * per);
   const int64_t t_end = min(Tb, t_begin + per);
@@ -177,7 +176,7 @@ __global__ void __launch_bounds__(kGenThreads) attend_generic_kernel(GenericArgs
     }
   }
   err = __syncthreads_or(err);
-  if (err && threadIdx.x == 0) atomicOr(a.error_word, kErrCodeRange);
+  if (err && threadIdx.x == 0) atomicOr(running_error(a.error_word), kErrCodeRange);
 }
 
 }  // namespace

@@ -111,9 +111,7 @@ __device__ __forceinline__ float qval<__nv_bfloat16>(const __nv_bfloat16* q, int
 // Position range of split s of sequence b: tile-aligned pieces of ceil(T_b / S).
 __device__ __forceinline__ void split_range(const AttendArgs& a, int b, int s, int S, int64_t& row0,
                                             int64_t& t_begin, int64_t& t_end) {
-  row0 = a.seq_offsets[b];
-  int64_t Tb = a.seq_offsets[b + 1] - row0;
-  Tb = Tb < 0 ? 0 : (Tb > a.max_T ? a.max_T : Tb);
+  const int64_t Tb = sequence_rows(a.seq_offsets, b, a.max_T, running_error(a.error_word), row0);
   int64_t per = (Tb + S - 1) / S;
   per = (per + kTileT - 1) / kTileT * kTileT;
   t_begin = min(Tb, static_cast<int64_t>(s) * per);
@@ -175,7 +173,7 @@ constexpr int kPhaseRows = kStageT;
 __global__ void prep_kernel(AttendArgs a, int R) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   const int Nc = a.n_codes;
-  if (e == 0 && blockIdx.y == 0) *a.error_word = 0;   // the device error word starts clear
+  if (e == 0 && blockIdx.y == 0) a.error_word[0] = a.error_word[1] = 0;   // both error words start clear
   const double rope_base = a.rope_base;
   double* theta = const_cast<double*>(a.theta);
   float4* rowph = const_cast<float4*>(a.rowph);
@@ -475,7 +473,7 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
   }
   if (kCheck) {
     err = __syncthreads_or(err);
-    if (err && tid == 0) atomicOr(a.error_word, kErrCodeRange);
+    if (err && tid == 0) atomicOr(running_error(a.error_word), kErrCodeRange);
   }
 }
 
@@ -695,7 +693,7 @@ attend_values_kernel(AttendArgs a) {
   }
   if (kCheck) {
     err = __syncthreads_or(err);
-    if (err && tid == 0) atomicOr(a.error_word, kErrCodeRange);
+    if (err && tid == 0) atomicOr(running_error(a.error_word), kErrCodeRange);
   }
 }
 

@@ -51,6 +51,10 @@ extern "C" commvq_status commvq_attend_decode_noalloc(
     const void* v_codes, const int64_t* seq_offsets, int32_t B, int64_t max_T,
     const float* k_codebook, const float* v_codebook, float* out, float* lse,
     const commvq_attend_options* options, void* stream) {
+  // Prepared state would have to survive in the shared array from an earlier call, which any
+  // other call on the device (another layer's codebooks, another rope base) may have
+  // overwritten since: this entry point always rebuilds it.
+  if (options && (options->flags & COMMVQ_ATTEND_PREPARED)) return COMMVQ_ERR_INVALID_ARG;
   if (B == 0)   // nothing to run: let the regular call validate the rest and return
     return commvq_attend_decode(cfg, q, q_dtype, k_codes, v_codes, seq_offsets, B, max_T, k_codebook,
                                 v_codebook, out, lse, nullptr, 0, options, stream);
@@ -62,8 +66,9 @@ extern "C" commvq_status commvq_attend_decode_noalloc(
   void* scratch = nullptr;
   const commvq_status rc = scratch_address(&scratch);
   if (rc != COMMVQ_OK) return rc;
-  // The regular call clears the scratch's error word; everything else it reads from the
-  // scratch is written earlier in the same call, so a previous call's leftovers do not matter.
+  // Without COMMVQ_ATTEND_PREPARED the regular call clears the scratch's error words and writes
+  // everything else it reads from the scratch earlier in the same call, so a previous call's
+  // leftovers do not matter.
   return commvq_attend_decode(cfg, q, q_dtype, k_codes, v_codes, seq_offsets, B, max_T, k_codebook,
                               v_codebook, out, lse, scratch, kNoAllocScratchBytes, options, stream);
 }

@@ -68,9 +68,8 @@ attend_table_kernel(AttendArgs a, const QT* __restrict__ q) {
   const int S = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kvh = h / (a.q_heads / a.kv_heads);
-  const int64_t row0 = a.seq_offsets[b];
-  int64_t Tb = a.seq_offsets[b + 1] - row0;
-  Tb = Tb < 0 ? 0 : (Tb > a.max_T ? a.max_T : Tb);
+  int64_t row0;
+  const int64_t Tb = sequence_rows(a.seq_offsets, b, a.max_T, running_error(a.error_word), row0);
   const int64_t per = (Tb + S - 1) / S;
   const int64_t t_begin = min(Tb, static_cast<int64_t>(s) * per);
   const int64_t t_end = min(Tb, t_begin + per);
@@ -264,7 +263,7 @@ attend_table_kernel(AttendArgs a, const QT* __restrict__ q) {
   }
   if (kCheck) {
     err = __syncthreads_or(err);
-    if (err && tid == 0) atomicOr(a.error_word, kErrCodeRange);
+    if (err && tid == 0) atomicOr(running_error(a.error_word), kErrCodeRange);
   }
 }
 

@@ -63,9 +63,7 @@ constexpr size_t kBvMcSmem =
 // ceil(T_b / S) positions).
 __device__ __forceinline__ void bv_split(const BinvArgs& a, int b, int v, int64_t& row0, int64_t& t_begin,
                                          int64_t& t_end) {
-  row0 = a.seq_offsets[b];
-  int64_t Tb = a.seq_offsets[b + 1] - row0;
-  Tb = Tb < 0 ? 0 : (Tb > a.max_T ? a.max_T : Tb);
+  const int64_t Tb = sequence_rows(a.seq_offsets, b, a.max_T, running_error(a.error_word), row0);
   int64_t per = (Tb + a.S - 1) / a.S;
   per = (per + kBvTile - 1) / kBvTile * kBvTile;
   t_begin = min(Tb, static_cast<int64_t>(v) * a.K * per);
@@ -365,6 +363,7 @@ __global__ void __launch_bounds__(kBvThreads, 1) binv_accumulate_kernel(BinvArgs
   // (starting from chunk -2: stage kBvRing - 2, parity 1), chunk c + kBvDist in stage sti
   int st = 0, stw = kBvRing - 2, sti = kBvDist;
   uint32_t pw = 1;
+  int last_issued = -1;   // the last chunk whose MMAs were issued and committed (uniform)
   for (int c = 0; c < n_c; ++c) {
     const uint32_t bbc = static_cast<uint32_t>(c & 1) * 64;
     const unsigned char* sg = ring + st * kBvStageBytes;
@@ -401,6 +400,7 @@ __global__ void __launch_bounds__(kBvThreads, 1) binv_accumulate_kernel(BinvArgs
       }
       umma_commit(&mbar[st]);
     }
+    last_issued = c;
     st = st + 1 == kBvRing ? 0 : st + 1;
     sti = sti + 1 == kBvRing ? 0 : sti + 1;
     if (++stw == kBvRing) {
@@ -409,13 +409,18 @@ __global__ void __launch_bounds__(kBvThreads, 1) binv_accumulate_kernel(BinvArgs
     }
   }
   cp_async_wait<0>();
-  if (n_c > 0 && ok) {   // the last commit covers every MMA issued before it
-    const int cl = n_c - 1;
-    ok = mbar_wait_bounded(&mbar[cl % kBvRing], static_cast<uint32_t>((cl / kBvRing) & 1), kBvWaitPolls);
+  // The last commit covers every MMA issued before it. It is waited for on the normal path and
+  // after a give-up alike (again bounded), so that TMEM is not read or freed while MMAs of this
+  // CTA may still write it. Its mbarrier phase is unambiguous: every earlier use of that stage
+  // (chunk last_issued - kBvRing) was waited for before chunk last_issued was issued.
+  if (last_issued >= 0) {
+    const bool done = mbar_wait_bounded(&mbar[last_issued % kBvRing],
+                                        static_cast<uint32_t>((last_issued / kBvRing) & 1), kBvWaitPolls);
+    ok = ok && done;
   }
   tc_fence_after();
   ok = __syncthreads_and(ok) != 0;
-  if (!ok && tid == 0) atomicOr(a.error_word, kErrWaitLimit);
+  if (!ok && tid == 0) atomicOr(running_error(a.error_word), kErrWaitLimit);
 
   if (warp < 8) {   // warps 0-3: rows 0-127 (half 0), warps 4-7: rows 128-255
     const int hb = warp >> 2;
@@ -549,6 +554,7 @@ __global__ void __launch_bounds__(kD) binv_finalize_kernel(BinvArgs a) {
   const int bh = blockIdx.x, d = threadIdx.x;
   pdl_trigger();   // the next decode step's scores kernel may copy its codebook image meanwhile
   pdl_wait();
+  if (bh == 0 && d == 0) publish_error(a.error_word);   // every kernel of the call has finished
   const int nch = a.Nc / kBvCRows;
   const float* src = a.opart + static_cast<int64_t>(bh) * nch * kD + d;
   float s = 0.0f;
@@ -654,11 +660,9 @@ extern "C" commvq_status commvq_attend_decode_binv(const commvq_config* cfg, con
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   commvq_status rc = COMMVQ_OK;
   if (!(flags & COMMVQ_ATTEND_PREPARED)) {
-    rc = launch_attend_prep(a, st);   // also clears the error word
+    rc = launch_attend_prep(a, st);   // also clears the error words
     if (rc != COMMVQ_OK) return rc;
-  } else if (cfg->n_codes < 256 && cudaMemsetAsync(a.error_word, 0, sizeof(int), st) != cudaSuccess) {
-    return COMMVQ_ERR_CUDA;
-  }
+  }   // else: the previous call's last kernel left the running error word clear
   rc = launch_attend_scores(a, q, q_dtype, S, st);
   if (rc != COMMVQ_OK) return rc;
 

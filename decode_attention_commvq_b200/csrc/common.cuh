@@ -19,6 +19,31 @@ constexpr int kPairs = kG / 2; // RoPE pairs per group
 // Device error word bits (first 4 bytes of an attention workspace).
 constexpr int kErrCodeRange = 1;
 constexpr int kErrWaitLimit = 2;   // a bounded wait on asynchronous tensor-core work gave up
+constexpr int kErrLength = 4;      // a sequence length outside [0, max_T] (taken as clamped)
+
+// An attention call's kernels OR their error bits into the running word (int 1 of the
+// workspace); the call's last kernel publishes it as the error word (int 0) and clears the
+// running word for the next call. Both kernels run in stream order, so the publication never
+// races with a setter.
+__device__ __forceinline__ int* running_error(int* error_word) { return error_word + 1; }
+__device__ __forceinline__ void publish_error(int* error_word) {
+  error_word[0] = error_word[1];
+  error_word[1] = 0;
+}
+
+// Rows of sequence b: seq_offsets[b] .. seq_offsets[b+1]-1, at most max_T of them. A length
+// outside [0, max_T] is clamped, and thread 0 of the calling CTA ORs kErrLength into *err_bits
+// (nullable: no report).
+__device__ __forceinline__ int64_t sequence_rows(const int64_t* seq_offsets, int b, int64_t max_T,
+                                                 int* err_bits, int64_t& row0) {
+  row0 = seq_offsets[b];
+  const int64_t Tb = seq_offsets[b + 1] - row0;
+  if (Tb < 0 || Tb > max_T) {
+    if (threadIdx.x == 0 && err_bits) atomicOr(err_bits, kErrLength);
+    return Tb < 0 ? 0 : max_T;
+  }
+  return Tb;
+}
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

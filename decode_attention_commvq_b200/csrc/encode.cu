@@ -18,12 +18,29 @@ namespace {
 
 constexpr int kTileFloats = 8192;   // codebook floats staged per pass (32 KB)
 
+// One tensor's encode: rows, codebook, codes out, residual out (nullable). A launch covers one
+// or two of them (blockIdx.z), e.g. a decode step's new key row and value row together.
+template <typename XT>
+struct EncodeJob {
+  const XT* x;
+  const float* cb;
+  void* codes;
+  float* residual_out;
+};
+template <typename XT>
+struct EncodeJobs {
+  EncodeJob<XT> job[2];
+};
+
 // GG: scalars per group (8, 16, 32 or 64). Each thread encodes kRows rows of one group.
 template <typename XT, bool kTrack, int GG>
 __global__ void __launch_bounds__(kThreads)
-encode_kernel(const XT* __restrict__ x, int64_t n_rows, int d, int R, int n_codes,
-              const float* __restrict__ cb, void* __restrict__ codes, int code_bytes,
-              unsigned long long* __restrict__ near_ties, float* __restrict__ residual_out) {
+encode_kernel(EncodeJobs<XT> jobs, int64_t n_rows, int d, int R, int n_codes, int code_bytes,
+              unsigned long long* __restrict__ near_ties) {
+  const XT* __restrict__ x = jobs.job[blockIdx.z].x;
+  const float* __restrict__ cb = jobs.job[blockIdx.z].cb;
+  void* __restrict__ codes = jobs.job[blockIdx.z].codes;
+  float* __restrict__ residual_out = jobs.job[blockIdx.z].residual_out;
   constexpr int kRows = GG == 8 ? 2 : 1;
   constexpr int kTile = kTileFloats / GG;   // entries per pass
   __shared__ float4 tile[kTileFloats / 4];
@@ -115,9 +132,15 @@ constexpr int kWarpUnitsPerBlock = 8;
 
 template <typename XT, bool kTrack, int GG>
 __global__ void __launch_bounds__(32 * kWarpUnitsPerBlock)
-encode_warp_kernel(const XT* __restrict__ x, int64_t n_rows, int d, int R, int n_codes,
-                   const float* __restrict__ cb, void* __restrict__ codes, int code_bytes,
-                   unsigned long long* __restrict__ near_ties, float* __restrict__ residual_out) {
+encode_warp_kernel(EncodeJobs<XT> jobs, int64_t n_rows, int d, int R, int n_codes, int code_bytes,
+                   unsigned long long* __restrict__ near_ties) {
+  // a following kernel launched as a programmatic dependent (a decode step's attention) may start
+  // its own set-up now; it waits for this grid before it reads the codes
+  pdl_trigger();
+  const XT* __restrict__ x = jobs.job[blockIdx.z].x;
+  const float* __restrict__ cb = jobs.job[blockIdx.z].cb;
+  void* __restrict__ codes = jobs.job[blockIdx.z].codes;
+  float* __restrict__ residual_out = jobs.job[blockIdx.z].residual_out;
   const int G = d / GG;
   const int lane = threadIdx.x & 31;
   const int64_t unit = static_cast<int64_t>(blockIdx.x) * kWarpUnitsPerBlock + (threadIdx.x >> 5);
@@ -175,40 +198,69 @@ encode_warp_kernel(const XT* __restrict__ x, int64_t n_rows, int d, int R, int n
 constexpr int64_t kWarpEncodeMaxUnits = 4096;
 
 template <typename XT, int GG>
-void launch_encode_g(const XT* x, int64_t n_rows, int d, int R, int n_codes, const float* cb,
-                     void* codes, int code_bytes, unsigned long long* near_ties, float* residual_out,
-                     cudaStream_t s) {
+void launch_encode_g(const EncodeJobs<XT>& jobs, int n_jobs, int64_t n_rows, int d, int R, int n_codes,
+                     int code_bytes, unsigned long long* near_ties, cudaStream_t s) {
   const int64_t units = n_rows * (d / GG);
   if (units <= kWarpEncodeMaxUnits) {
     const unsigned blocks = static_cast<unsigned>((units + kWarpUnitsPerBlock - 1) / kWarpUnitsPerBlock);
+    const dim3 grid(blocks, 1, n_jobs);
     if (near_ties)
-      encode_warp_kernel<XT, true, GG><<<blocks, 32 * kWarpUnitsPerBlock, 0, s>>>(
-          x, n_rows, d, R, n_codes, cb, codes, code_bytes, near_ties, residual_out);
+      encode_warp_kernel<XT, true, GG><<<grid, 32 * kWarpUnitsPerBlock, 0, s>>>(jobs, n_rows, d, R, n_codes,
+                                                                                code_bytes, near_ties);
     else
-      encode_warp_kernel<XT, false, GG><<<blocks, 32 * kWarpUnitsPerBlock, 0, s>>>(
-          x, n_rows, d, R, n_codes, cb, codes, code_bytes, nullptr, residual_out);
+      encode_warp_kernel<XT, false, GG><<<grid, 32 * kWarpUnitsPerBlock, 0, s>>>(jobs, n_rows, d, R, n_codes,
+                                                                                 code_bytes, nullptr);
     return;
   }
   const int64_t per_block = kThreads * (GG == 8 ? 2 : 1);
-  dim3 grid(static_cast<unsigned>((n_rows + per_block - 1) / per_block), d / GG);
+  dim3 grid(static_cast<unsigned>((n_rows + per_block - 1) / per_block), d / GG, n_jobs);
   if (near_ties)
-    encode_kernel<XT, true, GG><<<grid, kThreads, 0, s>>>(x, n_rows, d, R, n_codes, cb, codes,
-                                                          code_bytes, near_ties, residual_out);
+    encode_kernel<XT, true, GG><<<grid, kThreads, 0, s>>>(jobs, n_rows, d, R, n_codes, code_bytes, near_ties);
   else
-    encode_kernel<XT, false, GG><<<grid, kThreads, 0, s>>>(x, n_rows, d, R, n_codes, cb, codes,
-                                                           code_bytes, nullptr, residual_out);
+    encode_kernel<XT, false, GG><<<grid, kThreads, 0, s>>>(jobs, n_rows, d, R, n_codes, code_bytes, nullptr);
 }
 
 template <typename XT>
-void launch_encode(const XT* x, int64_t n_rows, int d, int g, int R, int n_codes, const float* cb,
-                   void* codes, int code_bytes, unsigned long long* near_ties, float* residual_out,
-                   cudaStream_t s) {
+void launch_encode(const EncodeJobs<XT>& jobs, int n_jobs, int64_t n_rows, int d, int g, int R, int n_codes,
+                   int code_bytes, unsigned long long* near_ties, cudaStream_t s) {
   switch (g) {
-    case 8: launch_encode_g<XT, 8>(x, n_rows, d, R, n_codes, cb, codes, code_bytes, near_ties, residual_out, s); break;
-    case 16: launch_encode_g<XT, 16>(x, n_rows, d, R, n_codes, cb, codes, code_bytes, near_ties, residual_out, s); break;
-    case 32: launch_encode_g<XT, 32>(x, n_rows, d, R, n_codes, cb, codes, code_bytes, near_ties, residual_out, s); break;
-    default: launch_encode_g<XT, 64>(x, n_rows, d, R, n_codes, cb, codes, code_bytes, near_ties, residual_out, s); break;
+    case 8: launch_encode_g<XT, 8>(jobs, n_jobs, n_rows, d, R, n_codes, code_bytes, near_ties, s); break;
+    case 16: launch_encode_g<XT, 16>(jobs, n_jobs, n_rows, d, R, n_codes, code_bytes, near_ties, s); break;
+    case 32: launch_encode_g<XT, 32>(jobs, n_jobs, n_rows, d, R, n_codes, code_bytes, near_ties, s); break;
+    default: launch_encode_g<XT, 64>(jobs, n_jobs, n_rows, d, R, n_codes, code_bytes, near_ties, s); break;
   }
+}
+
+// Host checks shared by the one- and two-tensor calls: OK, INVALID_ARG or UNSUPPORTED.
+commvq_status check_encode(const commvq_config* cfg, commvq_dtype x_dtype, int64_t n_tokens) {
+  if (!cfg) return COMMVQ_ERR_INVALID_ARG;
+  const int d = cfg->d, g = cfg->g, R = cfg->R, Nc = cfg->n_codes, H = cfg->kv_heads;
+  if (d <= 0 || g <= 0 || d % g || g % 2 || R < 1 || Nc < 1 || H < 1 || n_tokens < 0)
+    return COMMVQ_ERR_INVALID_ARG;
+  if (cfg->code_bytes != (Nc <= 256 ? 1 : 2)) return COMMVQ_ERR_INVALID_ARG;
+  if (Nc > 65536) return COMMVQ_ERR_INVALID_ARG;
+  if ((g != 8 && g != 16 && g != 32 && g != 64) || R > 32) return COMMVQ_ERR_UNSUPPORTED;
+  if (x_dtype != COMMVQ_F32 && x_dtype != COMMVQ_F16) return COMMVQ_ERR_UNSUPPORTED;
+  const int64_t n_rows = n_tokens * H;
+  if (n_tokens > 0 && (n_rows / H != n_tokens || (n_rows + kThreads) / kThreads > INT32_MAX))
+    return COMMVQ_ERR_INVALID_ARG;
+  return COMMVQ_OK;
+}
+
+commvq_status run_encode(const commvq_config* cfg, commvq_dtype x_dtype, int64_t n_tokens, const void* const* x,
+                         const float* const* cb, void* const* codes, float* const* residual, int n_jobs,
+                         unsigned long long* near_ties, cudaStream_t s) {
+  const int64_t n_rows = n_tokens * cfg->kv_heads;
+  if (x_dtype == COMMVQ_F32) {
+    EncodeJobs<float> jobs{};
+    for (int k = 0; k < n_jobs; ++k) jobs.job[k] = {static_cast<const float*>(x[k]), cb[k], codes[k], residual[k]};
+    launch_encode(jobs, n_jobs, n_rows, cfg->d, cfg->g, cfg->R, cfg->n_codes, cfg->code_bytes, near_ties, s);
+  } else {
+    EncodeJobs<__half> jobs{};
+    for (int k = 0; k < n_jobs; ++k) jobs.job[k] = {static_cast<const __half*>(x[k]), cb[k], codes[k], residual[k]};
+    launch_encode(jobs, n_jobs, n_rows, cfg->d, cfg->g, cfg->R, cfg->n_codes, cfg->code_bytes, near_ties, s);
+  }
+  return launch_status();
 }
 
 }  // namespace
@@ -220,27 +272,33 @@ extern "C" commvq_status commvq_encode(const commvq_config* cfg, const void* x, 
                                        int64_t n_tokens, const float* codebook, void* codes,
                                        unsigned long long* near_ties, float* residual_out,
                                        void* stream) {
-  if (!cfg) return COMMVQ_ERR_INVALID_ARG;
-  const int d = cfg->d, g = cfg->g, R = cfg->R, Nc = cfg->n_codes, H = cfg->kv_heads;
-  if (d <= 0 || g <= 0 || d % g || g % 2 || R < 1 || Nc < 1 || H < 1 || n_tokens < 0)
-    return COMMVQ_ERR_INVALID_ARG;
-  if (cfg->code_bytes != (Nc <= 256 ? 1 : 2)) return COMMVQ_ERR_INVALID_ARG;
-  if (Nc > 65536) return COMMVQ_ERR_INVALID_ARG;
-  if ((g != 8 && g != 16 && g != 32 && g != 64) || R > 32) return COMMVQ_ERR_UNSUPPORTED;
-  if (x_dtype != COMMVQ_F32 && x_dtype != COMMVQ_F16) return COMMVQ_ERR_UNSUPPORTED;
+  const commvq_status cs = check_encode(cfg, x_dtype, n_tokens);
+  if (cs != COMMVQ_OK) return cs;
   if (n_tokens == 0) return COMMVQ_OK;
   if (!x || !codebook || !codes) return COMMVQ_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(codebook, 16) || !aligned(near_ties, 8) || !aligned(residual_out, 16))
     return COMMVQ_ERR_INVALID_ARG;
-  const int64_t n_rows = n_tokens * H;
-  if (n_rows / H != n_tokens || (n_rows + kThreads) / kThreads > INT32_MAX)
+  const void* xs[1] = {x};
+  const float* cbs[1] = {codebook};
+  void* cs1[1] = {codes};
+  float* rs[1] = {residual_out};
+  return run_encode(cfg, x_dtype, n_tokens, xs, cbs, cs1, rs, 1, near_ties, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" commvq_status commvq_encode_kv(const commvq_config* cfg, const void* k_x, const void* v_x,
+                                          commvq_dtype x_dtype, int64_t n_tokens, const float* k_codebook,
+                                          const float* v_codebook, void* k_codes, void* v_codes,
+                                          unsigned long long* near_ties, void* stream) {
+  const commvq_status cs = check_encode(cfg, x_dtype, n_tokens);
+  if (cs != COMMVQ_OK) return cs;
+  if (n_tokens == 0) return COMMVQ_OK;
+  if (!k_x || !v_x || !k_codebook || !v_codebook || !k_codes || !v_codes) return COMMVQ_ERR_INVALID_ARG;
+  if (!aligned(k_x, 16) || !aligned(v_x, 16) || !aligned(k_codebook, 16) || !aligned(v_codebook, 16) ||
+      !aligned(near_ties, 8))
     return COMMVQ_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (x_dtype == COMMVQ_F32)
-    launch_encode(static_cast<const float*>(x), n_rows, d, g, R, Nc, codebook, codes, cfg->code_bytes,
-                  near_ties, residual_out, s);
-  else
-    launch_encode(static_cast<const __half*>(x), n_rows, d, g, R, Nc, codebook, codes, cfg->code_bytes,
-                  near_ties, residual_out, s);
-  return launch_status();
+  const void* xs[2] = {k_x, v_x};
+  const float* cbs[2] = {k_codebook, v_codebook};
+  void* cs2[2] = {k_codes, v_codes};
+  float* rs[2] = {nullptr, nullptr};
+  return run_encode(cfg, x_dtype, n_tokens, xs, cbs, cs2, rs, 2, near_ties, static_cast<cudaStream_t>(stream));
 }

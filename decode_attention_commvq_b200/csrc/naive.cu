@@ -167,9 +167,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decompress_kernel(DecompArgs a
   auto chunk_of = [&](int64_t w, int64_t& rec0, int& rows, int& h) {
     const int b = static_cast<int>(w / a.n_hi);
     h = static_cast<int>(w % a.n_hi);
-    const int64_t row0 = a.seq_offsets[b];
-    int64_t Tb = a.seq_offsets[b + 1] - row0;
-    Tb = Tb < 0 ? 0 : (Tb > a.max_T ? a.max_T : Tb);
+    int64_t row0;
+    const int64_t Tb = sequence_rows(a.seq_offsets, b, a.max_T, a.error_word, row0);
     const int64_t t0 = static_cast<int64_t>(h) * kChunk;
     rows = t0 >= Tb ? 0 : static_cast<int>(min(static_cast<int64_t>(kChunk), Tb - t0));
     rec0 = (row0 + t0) * KV;
@@ -264,6 +263,7 @@ struct DenseArgs {
   const void* v;
   const int64_t* seq_offsets;
   Partial* partials;
+  int* error_word;
   int64_t max_T;
   int B;
   int q_heads;
@@ -338,9 +338,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_decode_kernel(DenseArg
   const int g = lane >> 2, i = lane & 3;
   const int kv = warp / kWpk, sub = warp % kWpk;
 
-  const int64_t row0 = a.seq_offsets[b];
-  int64_t Tb = a.seq_offsets[b + 1] - row0;
-  Tb = Tb < 0 ? 0 : (Tb > a.max_T ? a.max_T : Tb);
+  int64_t row0;
+  const int64_t Tb = sequence_rows(a.seq_offsets, b, a.max_T, running_error(a.error_word), row0);
   int64_t per = (Tb + S - 1) / S;
   per = (per + 15) / 16 * 16;
   const int64_t t_begin = min(Tb, static_cast<int64_t>(s) * per);
@@ -702,6 +701,7 @@ extern "C" commvq_status commvq_dense_decode(const commvq_config* cfg, const voi
   d.v = v;
   d.seq_offsets = seq_offsets;
   d.partials = reinterpret_cast<Partial*>(ws + kHeader);
+  d.error_word = static_cast<int*>(workspace);
   d.max_T = max_T;
   d.B = B;
   d.q_heads = cfg->q_heads;
@@ -709,6 +709,7 @@ extern "C" commvq_status commvq_dense_decode(const commvq_config* cfg, const voi
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   void* start = options ? options->main_start : nullptr;
   void* stop = options ? options->main_stop : nullptr;
+  if (cudaMemsetAsync(d.error_word, 0, 2 * sizeof(int), st) != cudaSuccess) return COMMVQ_ERR_CUDA;
   if (start && record_event(start, st) != cudaSuccess)
     return COMMVQ_ERR_CUDA;
   const commvq_status rc = kv_dtype == COMMVQ_F16 ? launch_dense_kv<__half>(d, q, q_dtype, S, st)
@@ -720,6 +721,7 @@ extern "C" commvq_status commvq_dense_decode(const commvq_config* cfg, const voi
   c.out = out;
   c.lse = lse;
   c.partials = d.partials;
+  c.error_word = d.error_word;
   c.B = B;
   c.q_heads = cfg->q_heads;
   return launch_combine(c, S * kWpk, st);

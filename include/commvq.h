@@ -35,9 +35,9 @@
  *
  * Errors: arguments are validated on the host before any launch; a failed check returns
  * a status and launches nothing. A launch failure returns COMMVQ_ERR_CUDA. Data errors
- * found on the device (a code >= Nc') never trap: the kernel clamps the code, records
- * the error in the workspace's error word and carries on; read it with
- * commvq_workspace_error().
+ * found on the device (a code >= Nc', a sequence length outside [0, max_T]) never trap:
+ * the kernel clamps the value, records the error in the workspace's error word and carries
+ * on; read it with commvq_workspace_error().
  */
 #ifndef COMMVQ_H_
 #define COMMVQ_H_
@@ -55,7 +55,7 @@ typedef enum {
   COMMVQ_ERR_UNSUPPORTED = 2,   /* valid CommVQ shape this build does not implement */
   COMMVQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
   COMMVQ_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
-  COMMVQ_ERR_DEVICE_CHECK = 5   /* the device recorded a data error (code out of range) */
+  COMMVQ_ERR_DEVICE_CHECK = 5   /* the device recorded a data error (code or length out of range) */
 } commvq_status;
 
 typedef enum { COMMVQ_F32 = 0, COMMVQ_F16 = 1, COMMVQ_BF16 = 2 } commvq_dtype;
@@ -84,7 +84,9 @@ typedef struct {
 enum {
   /* The workspace already holds this configuration's and these codebooks' prepared state,
      written by commvq_attend_prepare (or by an earlier commvq_attend_decode without the
-     flag) with the same cfg, B, max_T, algo and splits; the call skips rewriting it. */
+     flag) with the same cfg and algo; the call skips rewriting it. The prepared state sits at
+     fixed offsets at the start of the workspace, so B, max_T and splits may differ between the
+     preparing call and later ones (the workspace must be large enough for each call). */
   COMMVQ_ATTEND_PREPARED = 1
 };
 
@@ -121,6 +123,22 @@ commvq_status commvq_encode(const commvq_config* cfg, const void* x, commvq_dtyp
                             int64_t n_tokens, const float* codebook, void* codes,
                             unsigned long long* near_ties, float* residual_out, void* stream);
 
+/* commvq_encode of a key tensor and a value tensor of the same shape in one launch (the abstract:
+ * the encoder turns every fresh K and V vector into codes): a decode step's new positions, whose
+ * two small encodes would otherwise be two launches. Each tensor is encoded exactly as
+ * commvq_encode encodes it (same codes, bit for bit) against its own codebook.
+ * k_x, v_x          [n_tokens, kv_heads, d] in x_dtype (F32 or F16), 16-byte aligned.
+ * k_codebook, v_codebook  [R, d/g, Nc', g] float32, 16-byte aligned.
+ * k_codes, v_codes  [n_tokens, kv_heads, R, d/g] out, code_bytes per element.
+ * near_ties         nullable device counter; both tensors' near-tie decisions are ADDED to it.
+ * When the next kernel on the stream is launched as a programmatic dependent (the attention of a
+ * decode step with COMMVQ_ATTEND_PREPARED), it may start its set-up while this encode runs; it
+ * reads the codes only after the encode has finished. Limits and errors as commvq_encode. */
+commvq_status commvq_encode_kv(const commvq_config* cfg, const void* k_x, const void* v_x,
+                               commvq_dtype x_dtype, int64_t n_tokens, const float* k_codebook,
+                               const float* v_codebook, void* k_codes, void* v_codes,
+                               unsigned long long* near_ties, void* stream);
+
 /* Bytes of device workspace commvq_attend_decode needs for B sequences whose longest
  * has max_T cached rows (options may be NULL = defaults). Returns 0 for invalid input. */
 size_t commvq_attend_workspace_bytes(const commvq_config* cfg, int32_t B, int64_t max_T,
@@ -145,14 +163,18 @@ size_t commvq_attend_workspace_bytes(const commvq_config* cfg, int32_t B, int64_
  * k_codes, v_codes  [total_T, kv_heads, R, d/g], code_bytes per element (uint16 above 256
  *             entries, GENERIC only), 16-byte aligned; total_T = seq_offsets[B].
  * seq_offsets [B+1] int64 device array, non-decreasing, seq_offsets[0] = 0, every
- *             T_b <= max_T (a longer sequence is truncated to max_T rows: the caller
- *             must pass the true maximum).
+ *             0 <= T_b <= max_T. A length outside that range is clamped to it (a longer
+ *             sequence is truncated to max_T rows, a negative one read as empty) and bit 2
+ *             of the device error word is set.
  * k_codebook, v_codebook [R, d/g, Nc', g] float32, 16-byte aligned.
  * out         [B, q_heads, d] float32 out, 16-byte aligned.
  * lse         [B, q_heads] float32 out, nullable.
  * workspace   device buffer of at least commvq_attend_workspace_bytes(...) bytes,
- *             256-byte aligned; its first 64 bytes hold the device error word, which this
- *             call clears. Calls that share a workspace must be ordered on one stream.
+ *             256-byte aligned; its first 64 bytes hold the device error word (int 0) and
+ *             the running word the call's kernels set bits in (int 1); the call's last
+ *             kernel copies the running word to the error word and clears it. Calls that
+ *             share a workspace must be ordered on one stream. A call that returned an error
+ *             status leaves the workspace's prepared state unspecified: prepare it again.
  * options     nullable (defaults: AUTO algorithm, library-chosen splits, no flags). With
  *             COMMVQ_ATTEND_PREPARED the workspace's prepared state (see commvq_attend_prepare)
  *             is used as it stands; otherwise the call writes it first.
@@ -173,11 +195,11 @@ commvq_status commvq_attend_decode(const commvq_config* cfg, const void* q, comm
 
 /* Write the state of commvq_attend_decode that depends only on cfg and the codebooks into
  * the workspace: for the decode-and-rotate algorithm, the fp16 codebook images and the RoPE
- * phasor tables; it also clears the device error word. Later commvq_attend_decode calls with
- * the same cfg, B, max_T, algo, splits, codebooks and workspace pass COMMVQ_ATTEND_PREPARED in
- * options->flags and skip this work (it is the same for every decode step of a layer). The
- * prepared state stays valid until the workspace or the codebooks change. With the table
- * algorithm there is no such state and the call only clears the error word.
+ * phasor tables; it also clears the device error words. Later commvq_attend_decode calls with
+ * the same cfg, algo, codebooks and workspace pass COMMVQ_ATTEND_PREPARED in options->flags and
+ * skip this work (it is the same for every decode step of a layer, whatever the step's B and
+ * max_T). The prepared state stays valid until the workspace or the codebooks change. With the
+ * table algorithm there is no such state and the call only clears the error words.
  * Arguments and errors as in commvq_attend_decode. */
 commvq_status commvq_attend_prepare(const commvq_config* cfg, int32_t B, int64_t max_T,
                                     const float* k_codebook, const float* v_codebook,
@@ -201,6 +223,9 @@ commvq_status commvq_attend_prepare(const commvq_config* cfg, int32_t B, int64_t
  * - Sharing: all calls on a device use the same array and it keeps the last call's
  *   contents. Each call rewrites everything it reads, so results do not depend on earlier
  *   calls, but calls that overlap on the GPU (different streams without ordering) race.
+ * - COMMVQ_ATTEND_PREPARED in options->flags is rejected with COMMVQ_ERR_INVALID_ARG: the
+ *   prepared state would live in the shared array, where any other call on the device may
+ *   have replaced it, so every call rebuilds it (one small kernel).
  * - Device data checks: codes >= Nc' are still clamped, but the error word lives in the
  *   internal array and is not reported by this entry point. */
 commvq_status commvq_attend_decode_noalloc(const commvq_config* cfg, const void* q,
@@ -307,12 +332,14 @@ size_t commvq_decompress_workspace_bytes(const commvq_config* cfg, int64_t max_T
  * commvq_attend_decode: pair p = channels (2p, 2p+1), theta_p = rope_base^(-2p/d)).
  * k_codes, v_codes  [total_T, kv_heads, R, d/g] uint8, total_T = seq_offsets[B].
  * seq_offsets       [B+1] int64 device array as in commvq_attend_decode; rows past
- *                   max_T positions of a sequence are not written.
+ *                   max_T positions of a sequence are not written (and set bit 2 of the
+ *                   error word, as a negative length does).
  * out_dtype         COMMVQ_BF16 or COMMVQ_F16.
  * k_out, v_out      [total_T, kv_heads, d] of out_dtype, 16-byte aligned.
  * workspace         >= commvq_decompress_workspace_bytes(cfg, max_T) bytes, 256-byte aligned;
  *                   its first 4 bytes are the device error word (bit 0: a code >= Nc' was
- *                   seen and clamped), cleared by this call.
+ *                   seen and clamped; bit 2: a sequence length outside [0, max_T]), cleared
+ *                   by this call.
  * Precision: entries are held in fp16 and summed in fp16; keys are rotated in fp32 with
  * phasors from fp64 angles; one final rounding to out_dtype.
  * Supports d = 128, g = 8, R <= 2, Nc' <= 256. */
@@ -334,6 +361,9 @@ size_t commvq_dense_decode_workspace_bytes(const commvq_config* cfg, int32_t B, 
  *         tensor-core products.
  * k, v    [total_T, kv_heads, d] in kv_dtype (F16 or BF16), 16-byte aligned.
  * seq_offsets, B, max_T, out, lse: as in commvq_attend_decode.
+ * workspace >= commvq_dense_decode_workspace_bytes(...) bytes, 256-byte aligned; its first 4
+ *         bytes are the device error word (bit 2: a sequence length outside [0, max_T], clamped),
+ *         written by this call (read it with commvq_workspace_error).
  * options nullable: splits (0 = library choice) and the main_start / main_stop events, recorded
  *         around the attention kernel (before the split combine).
  * Precision: fp32 accumulation; softmax weights are rounded to kv_dtype for the second product.
@@ -347,7 +377,8 @@ commvq_status commvq_dense_decode(const commvq_config* cfg, const void* q, commv
 /* The device error word in an attention workspace: synchronises `stream`, copies the word
  * to the host and writes it to *device_error (0 = none; bit 0 = a code >= Nc' was seen
  * and clamped; bit 1 = a bounded wait for the tensor cores' asynchronous work gave up, the
- * output of that call is not valid). Returns COMMVQ_ERR_DEVICE_CHECK when the word is non-zero. */
+ * output of that call is not valid; bit 2 = a sequence length outside [0, max_T] was
+ * clamped). Returns COMMVQ_ERR_DEVICE_CHECK when the word is non-zero. */
 commvq_status commvq_workspace_error(const void* workspace, int32_t* device_error, void* stream);
 
 /* Static description of a status code. */

@@ -2,6 +2,8 @@
  * CommVQ CPU oracle -- TEST INFRASTRUCTURE ONLY.
  *
  * Plain, slow, single-threaded C that states what the CommVQ hot path computes.
+ * (The Python face may run several calls at once on disjoint rows or heads; each call
+ * is the same single-threaded code.)
  * Only the tests, the smoke check and the bench's CPU-baseline leg may load it;
  * the library's product path never does. It shares no code, header, table or
  * constant with the CUDA library.
@@ -383,6 +385,41 @@ int oracle_em_step(const float* rows, int64_t N, int d, int g, int n_codes, floa
   free(sum);
   free(cnt);
   if (sse_out) *sse_out = sse;
+  return ORACLE_OK;
+}
+
+/* The M-step of oracle_em_step on given assignments (Algorithm 1 / Eq. 20's closed-form
+ * update): entry (j, c) becomes (float)(S / m), S the fp64 sum of the m fp32 sub-vectors
+ * assigned to it, summed in (row, group) order; an entry with m = 0 keeps its value.
+ * codes [N, d/g] int32 in [0, Nc'). With the assignments oracle_em_step makes (the encoder's
+ * rule against the same codebook) the result is oracle_em_step's, bit for bit: the same sums
+ * in the same order. */
+int oracle_em_update(const float* rows, int64_t N, int d, int g, int n_codes, const int32_t* codes,
+                     float* cb) {
+  if (!valid_shape(d, g, 1, n_codes) || N < 0 || !rows || !cb || (N > 0 && !codes)) return ORACLE_BAD_ARG;
+  const int G = d / g;
+  double* sum = (double*)calloc((size_t)G * n_codes * g, sizeof(double));
+  int64_t* cnt = (int64_t*)calloc((size_t)G * n_codes, sizeof(int64_t));
+  if (!sum || !cnt) { free(sum); free(cnt); return ORACLE_NO_MEM; }
+  for (int64_t n = 0; n < N; ++n)
+    for (int j = 0; j < G; ++j) {
+      const float* x = rows + n * d + (int64_t)j * g;
+      const int32_t c = codes[n * G + j];
+      if (c < 0 || c >= n_codes) { free(sum); free(cnt); return ORACLE_BAD_ARG; }
+      cnt[(int64_t)j * n_codes + c] += 1;
+      for (int k = 0; k < g; ++k) sum[((int64_t)j * n_codes + c) * g + k] += (double)x[k];
+    }
+  for (int j = 0; j < G; ++j)
+    for (int c = 0; c < n_codes; ++c) {
+      int64_t m = cnt[(int64_t)j * n_codes + c];
+      if (m == 0) continue;
+      for (int k = 0; k < g; ++k) {
+        int64_t at = ((int64_t)j * n_codes + c) * g + k;
+        cb[at] = (float)(sum[at] / (double)m);
+      }
+    }
+  free(sum);
+  free(cnt);
   return ORACLE_OK;
 }
 

@@ -13,6 +13,7 @@ import ctypes
 import os
 import subprocess
 import time
+from concurrent.futures import ThreadPoolExecutor
 from typing import Optional
 
 import numpy as np
@@ -51,9 +52,10 @@ def lib():
         _lib.oracle_rope.argtypes = [P, P, I64, I, ctypes.c_double, P]
         _lib.oracle_attend_dense.argtypes = [P, P, P, P, I, I, I, I, P, P]
         _lib.oracle_decode_bits.argtypes = [P, I64, I, P, I, P]
+        _lib.oracle_em_update.argtypes = [P, I64, I, I, I, P, P]
         for f in ("oracle_encode", "oracle_decode", "oracle_scores_plain", "oracle_scores_table",
                   "oracle_attend", "oracle_em_step", "oracle_values_hist", "oracle_em_soft_step",
-                  "oracle_rope", "oracle_attend_dense", "oracle_decode_bits"):
+                  "oracle_rope", "oracle_attend_dense", "oracle_decode_bits", "oracle_em_update"):
             getattr(_lib, f).restype = ctypes.c_int
     return _lib
 
@@ -71,8 +73,34 @@ def _check(rc: int, what: str):
         raise RuntimeError(f"oracle {what} failed with status {rc}")
 
 
-def encode(x: np.ndarray, cb: np.ndarray, want_residual: bool = False):
+def host_threads() -> int:
+    """Cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _pieces(n: int, threads: int):
+    """[start, stop) ranges splitting n items into at most `threads` contiguous pieces."""
+    k = max(1, min(int(threads), n))
+    edges = [n * i // k for i in range(k + 1)]
+    return [(edges[i], edges[i + 1]) for i in range(k) if edges[i + 1] > edges[i]]
+
+
+def _run_pieces(fn, pieces):
+    """Run fn(a, b) for every piece, on threads when there are several (each call is one
+    single-threaded C call on disjoint data; ctypes releases the GIL around it)."""
+    if len(pieces) <= 1:
+        return [fn(a, b) for a, b in pieces]
+    with ThreadPoolExecutor(len(pieces)) as ex:
+        return list(ex.map(lambda ab: fn(*ab), pieces))
+
+
+def encode(x: np.ndarray, cb: np.ndarray, want_residual: bool = False, threads: int = 1):
     """Residual nearest-codeword codes of rows x[..., d] against cb [R, d/g, Nc', g].
+    threads > 1 splits the rows into contiguous pieces encoded at once (each row's result does
+    not depend on the others, so the output is the same).
 
     Returns (codes [..., R, d/g] int32, near_tie_count[, residual [..., d] fp32])."""
     R, G, Nc, g = cb.shape
@@ -83,13 +111,18 @@ def encode(x: np.ndarray, cb: np.ndarray, want_residual: bool = False):
     cbf = _c(cb, np.float32)
     codes = np.empty((n, R, G), dtype=np.int32)
     res = np.empty((n, d), dtype=np.float32) if want_residual else None
-    ties = ctypes.c_int64(0)
-    _check(lib().oracle_encode(_p(xf), n, d, g, R, Nc, _p(cbf), _p(codes), _p(res),
-                               ctypes.byref(ties)), "encode")
+
+    def piece(a, b):   # rows a..b-1: their own codes, residuals and near-tie count
+        ties = ctypes.c_int64(0)
+        _check(lib().oracle_encode(_p(xf[a:b]), b - a, d, g, R, Nc, _p(cbf), _p(codes[a:b]),
+                                   None if res is None else _p(res[a:b]), ctypes.byref(ties)), "encode")
+        return int(ties.value)
+
+    ties = sum(_run_pieces(piece, _pieces(n, threads)))
     codes = codes.reshape(*lead, R, G)
     if want_residual:
-        return codes, int(ties.value), res.reshape(*lead, d)
-    return codes, int(ties.value)
+        return codes, ties, res.reshape(*lead, d)
+    return codes, ties
 
 
 def decode(codes: np.ndarray, cb: np.ndarray) -> np.ndarray:
@@ -222,9 +255,28 @@ def attend_binv(q: np.ndarray, k_codes: np.ndarray, v_bits: np.ndarray, offsets:
 
 
 def attend_codes(q: np.ndarray, k_codes: np.ndarray, v_codes: np.ndarray, offsets: np.ndarray,
-                 kcb: np.ndarray, vcb: np.ndarray, base: float):
-    """Decode attention straight from codes [sum T, Hkv, R, d/g]: decode, then attend."""
-    return attend(q, decode(k_codes, kcb), decode(v_codes, vcb), offsets, base)
+                 kcb: np.ndarray, vcb: np.ndarray, base: float, threads: int = 1):
+    """Decode attention straight from codes [sum T, Hkv, R, d/g]: decode, then attend.
+    threads > 1 attends the KV heads' query groups at once (each (b, h) result is computed on
+    its own, so the output is the same)."""
+    Hkv = k_codes.shape[1]
+    if threads <= 1 or Hkv == 1:
+        return attend(q, decode(k_codes, kcb), decode(v_codes, vcb), offsets, base)
+    B, Hq, d = q.shape
+    G = Hq // Hkv
+    out = np.empty((B, Hq, d), dtype=np.float64)
+    lse = np.empty((B, Hq), dtype=np.float64)
+
+    def piece(a, b):   # KV heads a..b-1 and their query heads, decoded one head at a time
+        for kvh in range(a, b):
+            khat = decode(k_codes[:, kvh:kvh + 1], kcb)
+            vhat = decode(v_codes[:, kvh:kvh + 1], vcb)
+            o, l = attend(q[:, kvh * G:(kvh + 1) * G], khat, vhat, offsets, base)
+            out[:, kvh * G:(kvh + 1) * G] = o
+            lse[:, kvh * G:(kvh + 1) * G] = l
+
+    _run_pieces(piece, _pieces(Hkv, threads))
+    return out, lse
 
 
 def em_step(rows: np.ndarray, cb_round: np.ndarray):
@@ -262,10 +314,24 @@ def forgy_init(rows: np.ndarray, idx: np.ndarray, g: int) -> np.ndarray:
                                 dtype=np.float32)
 
 
-def fit_codebook(rows: np.ndarray, R: int, g: int, n_codes: int, iters: int, init_indices):
+def em_update(rows: np.ndarray, cb_round: np.ndarray, codes: np.ndarray) -> np.ndarray:
+    """The EM step's closed-form update on given assignments codes [N, d/g]: a new codebook."""
+    G, Nc, g = cb_round.shape
+    rf = _c(rows, np.float32)
+    cb = _c(cb_round, np.float32).copy()
+    _check(lib().oracle_em_update(_p(rf), rf.shape[0], G * g, g, Nc, _p(_c(codes, np.int32)), _p(cb)),
+           "em_update")
+    return cb
+
+
+def fit_codebook(rows: np.ndarray, R: int, g: int, n_codes: int, iters: int, init_indices,
+                 threads: int = 1):
     """Sequential residual fit: for each round, Forgy init from that round's residual rows,
     `iters` EM steps, then advance the residuals by one encoder round against the final
-    codebook. init_indices(r, N) -> row indices. Returns (cb [R, d/g, Nc', g], sse history)."""
+    codebook. init_indices(r, N) -> row indices. Returns (cb [R, d/g, Nc', g], sse history).
+    threads > 1 makes each step's assignments with the threaded encoder (the EM step's own
+    rule) and applies the update on them: the same codebooks bit for bit, and no SSE history
+    (None)."""
     res = _c(rows, np.float32).copy()
     N, d = res.shape
     rounds, hist = [], []
@@ -273,12 +339,16 @@ def fit_codebook(rows: np.ndarray, R: int, g: int, n_codes: int, iters: int, ini
         cb_r = forgy_init(res, init_indices(r, N), g)
         h = []
         for _ in range(iters):
-            cb_r, _, sse = em_step(res, cb_r)
-            h.append(sse)
+            if threads > 1:
+                codes, _ = encode(res, cb_r[None], threads=threads)
+                cb_r = em_update(res, cb_r, codes[:, 0])
+            else:
+                cb_r, _, sse = em_step(res, cb_r)
+                h.append(sse)
         hist.append(h)
         rounds.append(cb_r)
-        _, _, res = encode(res, cb_r[None], want_residual=True)
-    return np.stack(rounds).astype(np.float32), hist
+        _, _, res = encode(res, cb_r[None], want_residual=True, threads=threads)
+    return np.stack(rounds).astype(np.float32), (hist if threads <= 1 else None)
 
 
 def time_call(fn, *a, **kw):

@@ -39,8 +39,11 @@ def oracle_codebooks(w: synth.Workload):
     out = []
     for key in (True, False):
         rows = synth.fit_rows(w, key)
+        # the threaded face gives the single-threaded fit bit for bit (pinned in
+        # test_oracle_pins.py), in a fraction of the time
         cb, _ = O.fit_codebook(rows, w.R, w.g, w.n_codes, w.em_iters,
-                               lambda r, N, key=key: synth.forgy_indices(w, key, r, N))
+                               lambda r, N, key=key: synth.forgy_indices(w, key, r, N),
+                               threads=O.host_threads())
         out.append(cb)
     return tuple(out)
 
@@ -56,3 +59,40 @@ def to_torch_q(q_stored: np.ndarray, dtype: str, device):
     if dtype == "f16":
         return torch.from_numpy(q_stored).to(device)
     return torch.from_numpy(q_stored.astype(np.float32)).to(device)
+
+
+# Planted near ties for the encoder (the spec's rule: the two smallest fp32 distances d1 <= d2
+# of a decision form a near tie when d2 - d1 <= 1e-5 * d2). One 8-scalar group, residual 0, so
+# the distance of an entry is the fp32 fused sum of its squared coordinates; every coordinate
+# is an integer and every partial sum stays below 2^24, so each distance is exact:
+#   D2  = 1024^2                          = 1048576
+#   IN  = 1023^2 + 45^2 + 3^2 + 1 + 1 + 1 = 1048566   (d2 - d1 = 10 <= 10.4858: a near tie)
+#   OUT = 1023^2 + 45^2 + 3^2 + 1 + 1     = 1048565   (d2 - d1 = 11 >  10.4858: not one)
+#   MID = 1024^2 + 4^2                    = 1048592
+#   FAR = 2000^2                          = 4000000
+NEAR_TIE_ENTRIES = {
+    "D2": [1024, 0, 0, 0, 0, 0, 0, 0],
+    "IN": [1023, 45, 3, 1, 1, 1, 0, 0],
+    "OUT": [1023, 45, 3, 1, 1, 0, 0, 0],
+    "MID": [1024, 4, 0, 0, 0, 0, 0, 0],
+    "FAR": [2000, 0, 0, 0, 0, 0, 0, 0],
+}
+# (entry order in the sub-codebook, expected code, expected near-tie count). The second-best
+# distance appears before the best (it must be kept when the best is replaced), after it (it
+# must be picked up by the else branch), and is lowered after a farther second (it must be
+# replaced by the closer one).
+NEAR_TIE_CASES = [
+    (("D2", "IN"), 1, 1),
+    (("IN", "D2"), 0, 1),
+    (("D2", "OUT"), 1, 0),
+    (("OUT", "D2"), 0, 0),
+    (("IN", "FAR", "MID", "D2"), 0, 1),
+    (("FAR", "MID", "IN"), 2, 0),
+    (("MID", "D2", "IN"), 2, 1),
+]
+
+
+def near_tie_case(order):
+    """Codebook [1, 1, len(order), 8] float32 and one zero row [1, 8] for a planted case."""
+    cb = np.array([[[NEAR_TIE_ENTRIES[k] for k in order]]], dtype=np.float32)
+    return cb, np.zeros((1, 8), dtype=np.float32)

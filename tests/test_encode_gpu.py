@@ -73,19 +73,28 @@ def test_encode_1bit_layer_slice(api, gpu):
     _compare(api, cfg, x, kcb, gpu)
 
 
-def test_encode_full_workload_sampled_rows(api, gpu):
-    """The encode workload at full size (131072 x 8 rows of fp16 K): codes of a seeded
-    sample of rows are checked one by one against the oracle."""
+@pytest.mark.parametrize("key", [True, False])
+def test_encode_full_workload_with_its_own_codebooks(api, gpu, key):
+    """The encode workload at full size: all 131072 x 8 fp16 rows of K (outlier channels) or V,
+    encoded with the workload's own codebooks (the oracle's fit: 10 EM iterations per round on
+    65536 rows). The codes of 1000 seeded positions (8000 rows) plus the first and the last
+    position equal the oracle's bit for bit, and so do the near-tie count and the residuals of
+    those rows encoded on their own."""
     w = synth.WORKLOADS[4]
-    kcb, _ = oracle_codebooks(w.with_(em_rows=4096, em_iters=2))
+    kcb, vcb = oracle_codebooks(w)
+    cb = kcb if key else vcb
     cfg = _cfg(api, w)
-    x = synth.encode_rows(w, True, w.encode_tokens)
-    got, _, _ = _run(api, cfg, x, kcb, gpu)
-    rng = np.random.default_rng(123)
-    toks = np.sort(rng.choice(w.encode_tokens, 512, replace=False))
-    toks = np.concatenate([toks, [0, w.encode_tokens - 1]])
-    want, _ = O.encode(x[toks], kcb)
+    x = synth.encode_rows(w, key, w.encode_tokens)
+    got, _, _ = _run(api, cfg, x, cb, gpu)
+    rng = np.random.default_rng(124 + int(key))
+    toks = np.sort(rng.choice(np.arange(1, w.encode_tokens - 1), 1000, replace=False))
+    toks = np.concatenate([[0], toks, [w.encode_tokens - 1]])
+    want, want_ties, want_res = O.encode(x[toks], cb, want_residual=True, threads=O.host_threads())
     assert np.array_equal(got[toks], want)
+    sub_codes, sub_ties, sub_res = _run(api, cfg, np.ascontiguousarray(x[toks]), cb, gpu, residual=True)
+    assert np.array_equal(sub_codes, want)
+    assert sub_ties == want_ties
+    assert np.array_equal(sub_res.view(np.uint32), want_res.astype(np.float32).view(np.uint32))
 
 
 def test_encode_uint16_codes_and_multi_tile(api, gpu):
@@ -157,3 +166,41 @@ def test_warp_encoder_ties_and_tiny_codebooks(gpu):
     assert np.array_equal(codes.cpu().numpy().astype(np.int64), ref.astype(np.int64))
     assert int(nt.item()) == ties and ties >= 16
     assert (codes.cpu().numpy()[0, 0, 0] == 1).all()
+
+
+@pytest.mark.parametrize("rows", [1, 5000])
+def test_planted_near_ties(api, gpu, rows):
+    """The planted near ties of tests/helpers.py (gaps just inside and just outside 1e-5 * d2,
+    second-best distances before, after and lowered after the best) through the warp encoder
+    (1 row) and the block encoder (5000 rows, more than 4096 units): the planted code in every
+    row and exactly the planted count per row."""
+    from tests.helpers import NEAR_TIE_CASES, near_tie_case
+    for order, code, ties in NEAR_TIE_CASES:
+        cb, x = near_tie_case(order)
+        cfg = api.Config(d=8, g=8, R=1, n_codes=len(order), q_heads=1, kv_heads=1)
+        xs = np.ascontiguousarray(np.repeat(x.reshape(1, 1, 8), rows, axis=0))
+        got, n, _ = _run(api, cfg, xs, cb, gpu)
+        assert (got == code).all(), order
+        assert n == ties * rows, order
+
+
+@pytest.mark.parametrize("tokens", [1, 700])
+def test_encode_kv_equals_two_encodes(api, gpu, tokens):
+    """commvq_encode_kv (key and value rows in one launch; 1 token takes the warp encoder, 700 the
+    block encoder) gives the codes and near-tie count of the oracle on each tensor."""
+    w = synth.WORKLOADS[1]
+    kcb, vcb = oracle_codebooks(w)
+    cfg = _cfg(api, w)
+    kx = synth.kv_rows(w, True, tokens, sub=555, dtype="f16")
+    vx = synth.kv_rows(w, False, tokens, sub=555, dtype="f16")
+    kc = torch.empty((tokens, w.kv_heads, w.R, w.groups), dtype=torch.uint8, device=gpu)
+    vc = torch.empty_like(kc)
+    nt = torch.zeros(1, dtype=torch.int64, device=gpu)
+    api.encode_kv(cfg, torch.from_numpy(kx).to(gpu), torch.from_numpy(vx).to(gpu), torch.from_numpy(kcb).to(gpu),
+                  torch.from_numpy(vcb).to(gpu), kc, vc, near_ties=nt)
+    torch.cuda.synchronize()
+    ref_k, tk = O.encode(kx, kcb)
+    ref_v, tv = O.encode(vx, vcb)
+    assert np.array_equal(kc.cpu().numpy().astype(np.int64), ref_k)
+    assert np.array_equal(vc.cpu().numpy().astype(np.int64), ref_v)
+    assert int(nt.item()) == tk + tv

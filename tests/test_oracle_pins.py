@@ -584,3 +584,47 @@ def test_attend_binv_is_attention_on_decoded_values():
     ref, ref_lse = O.attend(q, O.decode(kc, kcb), vhat, offs, 1e4)
     assert np.abs(out - ref).max() <= 1e-12 * np.abs(ref).max()
     assert np.allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+def test_encoder_near_tie_threshold_and_second_best_tracking():
+    """Planted non-exact near ties (tests/helpers.py): a gap just inside and just outside
+    1e-5 * d2, with the second-best distance before, after and lowered after the best. Each
+    case must give the planted code and the exact count; the distances are exact integers, so
+    a dropped second-best update or a flipped comparison changes a count."""
+    from tests.helpers import NEAR_TIE_CASES, near_tie_case
+    for order, code, ties in NEAR_TIE_CASES:
+        cb, x = near_tie_case(order)
+        got, n = O.encode(x, cb)
+        assert int(got[0, 0, 0]) == code, order
+        assert n == ties, order
+    # the threshold itself, in fp32 as the spec evaluates it
+    lim = np.float32(1e-5) * np.float32(1048576)
+    assert np.float32(10) <= lim < np.float32(11)
+
+
+def test_threaded_oracle_calls_equal_single_threaded_ones():
+    """The oracle's threaded face (disjoint rows or KV heads per thread, the same C calls) must
+    give the single-threaded results bit for bit: encode (codes, near ties, residuals), the
+    codebook fit (assignments by the encoder's rule, then the EM update) and attention."""
+    w = synth.WORKLOADS[1].with_(seq_len=301, em_rows=700, em_iters=2)
+    rows = synth.fit_rows(w, True)
+    init = lambda r, N: synth.forgy_indices(w, True, r, N)
+    cb1, hist = O.fit_codebook(rows, 2, 8, 256, 2, init)
+    cb4, _ = O.fit_codebook(rows, 2, 8, 256, 2, init, threads=4)
+    assert np.array_equal(cb1.view(np.uint32), cb4.view(np.uint32))
+    assert len(hist) == 2 and hist[0][1] <= hist[0][0]
+    x = synth.kv_rows(w, True, T=301)
+    c1, t1, r1 = O.encode(x, cb1, want_residual=True)
+    c4, t4, r4 = O.encode(x, cb1, want_residual=True, threads=4)
+    assert np.array_equal(c1, c4) and t1 == t4 and np.array_equal(r1.view(np.uint32), r4.view(np.uint32))
+    vc, _ = O.encode(synth.kv_rows(w, False, T=301), cb1)
+    q = synth.as_f32(synth.queries(w), w.q_dtype).astype(np.float64)
+    offs = np.array([0, 301])
+    o1, l1 = O.attend_codes(q, c1, vc, offs, cb1, cb1, w.rope_base)
+    o4, l4 = O.attend_codes(q, c1, vc, offs, cb1, cb1, w.rope_base, threads=4)
+    assert np.array_equal(o1, o4) and np.array_equal(l1, l4)
+    # the update on the EM step's own assignments is the EM step
+    cb_r = cb1[0]
+    new_a, codes, _ = O.em_step(rows, cb_r)
+    new_b = O.em_update(rows, cb_r, codes)
+    assert np.array_equal(new_a.view(np.uint32), new_b.view(np.uint32))

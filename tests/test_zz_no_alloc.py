@@ -6,9 +6,11 @@ where a cudaMalloc (which may synchronise the device) is not allowed. It runs th
 attention as commvq_attend_decode with the library's fixed internal scratch (32 MiB per
 device) in place of a caller-provided workspace.
 
-These tests call it through the C ABI and compare it with commvq_attend_decode on the same
-inputs, on two calls in a row (the second call finds the first call's leftovers in the
-shared scratch). This file is named so that pytest collects it last.
+These tests call it through the C ABI and compare it with commvq_attend_decode and with the
+CPU oracle on the same inputs, on two calls in a row (the second call finds the first call's
+leftovers in the shared scratch). COMMVQ_ATTEND_PREPARED is refused: prepared state kept in
+the shared array could belong to another layer. This file is named so that pytest collects it
+last; each test stands on its own.
 """
 import numpy as np
 import pytest
@@ -76,21 +78,64 @@ def test_noalloc_rejects_requests_beyond_its_scratch(api, gpu):
     assert torch.count_nonzero(out).item() == 0
 
 
-@pytest.mark.parametrize("algo", [1, 2])
-def test_noalloc_reuses_its_prepared_state(api, gpu, algo):
-    """A call without the flag prepares the internal scratch; the next call on the same layer
-    passes COMMVQ_ATTEND_PREPARED and gives the same result."""
-    w = synth.WORKLOADS[1]
-    cfg, q, kc, vc, offs, max_T, kcb, vcb = _inputs(api, w, gpu)
-    outs = []
-    for prepared in (False, True):
-        out = torch.full((w.batch, w.q_heads, w.d), float("nan"), dtype=torch.float32, device=gpu)
-        lse = torch.full((w.batch, w.q_heads), float("nan"), dtype=torch.float32, device=gpu)
-        api.attend_decode_noalloc(cfg, q, kc, vc, offs, max_T, kcb, vcb, out, lse, algo=algo,
-                                  prepared=prepared)
+def test_noalloc_rejects_the_prepared_flag(api, gpu):
+    """Layer A, then layer B (other codebooks), both without the flag, then layer A with
+    COMMVQ_ATTEND_PREPARED: the shared array holds layer B's images by then, so the flagged call
+    must be refused (INVALID_ARG) and leave the caller's output untouched."""
+    w = synth.WORKLOADS[1].with_(seq_len=2048)
+    cfg, q, kc, vc, offs, max_T, kcb_a, vcb_a = _inputs(api, w, gpu)
+    wb = w.with_(seed=w.seed + 11)
+    kcb_b = torch.from_numpy(synth.normal_codebook(wb, True)).to(gpu)
+    vcb_b = torch.from_numpy(synth.normal_codebook(wb, False)).to(gpu)
+    out = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32, device=gpu)
+    for kcb, vcb in ((kcb_a, vcb_a), (kcb_b, vcb_b)):
+        api.attend_decode_noalloc(cfg, q, kc, vc, offs, max_T, kcb, vcb, out, algo=2)
+    sentinel = torch.full_like(out, 7.0)
+    out.copy_(sentinel)
+    with pytest.raises(api.CommVQError) as e:
+        api.attend_decode_noalloc(cfg, q, kc, vc, offs, max_T, kcb_a, vcb_a, out, algo=2, prepared=True)
+    assert e.value.status == 1
+    torch.cuda.synchronize()
+    assert torch.equal(out, sentinel)
+
+
+def test_noalloc_matches_the_oracle(api, gpu):
+    """The no-allocation call against the CPU oracle directly (not only against the workspace
+    call), on 3000 positions of the 2-bit layer's shape with uniform codes, twice in a row."""
+    from oracle import oracle as O
+    from tests.helpers import q_as_f64
+    w = synth.WORKLOADS[1].with_(seq_len=3000, codebook="normal")
+    cfg = api.Config(d=w.d, g=w.g, R=w.R, n_codes=w.n_codes, q_heads=w.q_heads,
+                     kv_heads=w.kv_heads, rope_base=w.rope_base)
+    offs = w.offsets()
+    kc = synth.uniform_codes(w, True, 3000)
+    vc = synth.uniform_codes(w, False, 3000)
+    kcb = synth.normal_codebook(w, True)
+    vcb = synth.normal_codebook(w, False)
+    q_np = synth.queries(w)
+    ref, ref_lse = O.attend_codes(q_as_f64(w, q_np), kc, vc, offs, kcb, vcb, w.rope_base)
+    args = (cfg, to_torch_q(q_np, w.q_dtype, gpu), torch.from_numpy(kc).to(gpu), torch.from_numpy(vc).to(gpu),
+            torch.from_numpy(offs).to(gpu), 3000, torch.from_numpy(kcb).to(gpu), torch.from_numpy(vcb).to(gpu))
+    for _ in range(2):
+        out = torch.full((1, w.q_heads, w.d), float("nan"), dtype=torch.float32, device=gpu)
+        lse = torch.full((1, w.q_heads), float("nan"), dtype=torch.float32, device=gpu)
+        api.attend_decode_noalloc(*args, out, lse)
         torch.cuda.synchronize()
-        outs.append((out, lse))
-    if algo == 2:   # no atomics on this path: the same bits
-        assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
-    else:           # histogram weights added with shared-memory atomics
-        assert rel_err(outs[1][0].cpu().numpy(), outs[0][0].cpu().numpy()) <= 1e-6
+        assert rel_err(out.cpu().numpy(), ref) <= tol_for(w)
+        assert np.allclose(lse.cpu().numpy(), ref_lse, rtol=1e-3, atol=5e-3)
+
+
+def test_noalloc_on_a_second_device(api):
+    """The array's address is looked up once per device, with that device current: a call with
+    cuda:1 current must use cuda:1's copy and match the workspace call there."""
+    if torch.cuda.device_count() < 2:
+        pytest.skip("one visible device")
+    dev = torch.device("cuda:1")
+    w = synth.WORKLOADS[1].with_(seq_len=2048)
+    with torch.cuda.device(dev):
+        cfg, q, kc, vc, offs, max_T, kcb, vcb = _inputs(api, w, dev)
+        ref, _ = api.attend_decode(cfg, q, kc, vc, offs, max_T, kcb, vcb)
+        out = torch.empty_like(ref)
+        api.attend_decode_noalloc(cfg, q, kc, vc, offs, max_T, kcb, vcb, out)
+        torch.cuda.synchronize(dev)
+        assert rel_err(out.cpu().numpy(), ref.cpu().numpy()) <= 1e-6
