@@ -52,7 +52,7 @@ def parse():
     ap.add_argument("--unprepared", action="store_true",
                     help="rebuild the codebook images and RoPE tables in every step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-heads", type=int, default=8, help="query heads in the oracle sample")
+    ap.add_argument("--cpu-heads", type=int, default=32, help="query heads in the oracle sample")
     return ap.parse_args()
 
 
@@ -349,7 +349,21 @@ def run_ours(args, w, rank, world, dev):
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
+    # spread: the same graph replayed again, each replay timed on its own (not part of `value`)
+    reps = []
+    with torch.cuda.stream(stream):
+        for _ in range(7):
+            r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            r0.record(stream)
+            graph.replay()
+            r1.record(stream)
+            reps.append((r0, r1))
+    torch.cuda.synchronize(dev)
     clk = clocks.stop()
+    rep_ms = np.array([a.elapsed_time(b) / K for a, b in reps])
+    spread = {"replays": len(reps), "ms_per_step_median": float(np.median(rep_ms)),
+              "ms_per_step_p10": float(np.percentile(rep_ms, 10)),
+              "ms_per_step_p90": float(np.percentile(rep_ms, 90))}
     ms = t0.elapsed_time(t1)
     ms_max = max_over_ranks(ms, world, dev)
     with torch.cuda.stream(stream):
@@ -420,7 +434,7 @@ def run_ours(args, w, rank, world, dev):
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": dtype_label(w, naive, args), "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
                    "d": w.d, "T": total_T, "R": w.R, "g": w.g, "n_codes": w.n_codes,
                    "q_dtype": w.q_dtype, "parallelism": f"replicas{world}",
@@ -441,13 +455,28 @@ def run_ours(args, w, rank, world, dev):
                      "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
                      "kernel": kname, "algorithmic_bytes_per_launch": alg_bytes,
                      "kernel_ms_mean": kern_ms,
-                     "traffic": recorded_traffic(kname, w.name)},
+                     "traffic": recorded_traffic(kname, w.name),
+                     "traffic_source": "dram__bytes_read.sum + dram__bytes_write.sum per launch from a committed "
+                                       "ncu capture (profiles/traffic.json: cold-cache replay of this exact kernel "
+                                       "source, not measured in this run; null when the source changed since)"},
+        "spread": spread,
         "e2e": e2e,
         "gpu_launches": launches_per_step * K,
         "clocks": clk,
     }
     result.update(extra)
     return result
+
+
+def dtype_label(w, naive, args):
+    """The operand and accumulation types of the timed path."""
+    if naive:
+        return f"{args.naive_dtype} dense rows and operands, fp32 accumulate"
+    if w.v_bits:
+        return "keys: fp16 codebook entries, bf16/fp16 two-term operands; values: int8 digit MMAs (exact int32); fp32 accumulate"
+    return ("fp16 codebook entries; keys rotated in fp32 and fed as two " +
+            ("bf16" if w.q_dtype == "bf16" else "fp16") +
+            " terms; softmax weights and values fp16; fp32 accumulate")
 
 
 def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, attend, stream, dev, torch, api,
@@ -536,8 +565,11 @@ def run_encode_fit(args, w, rank, world, dev):
     # kernels)
     fit_ms = {}
     cbs = []
-    warm = torch.from_numpy(synth.fit_rows(w.with_(em_rows=1024), True)).to(dev)
+    # warm-up at the full row count: loads the kernels and lets the caching allocator hold the
+    # fit's buffers, so neither timed fit pays for a first cudaMalloc
+    warm = torch.from_numpy(synth.fit_rows(w, True)).to(dev)
     fit.fit_codebook(warm, w.R, w.n_codes, 1, lambda r, N: synth.forgy_indices(w, True, r, N), g=w.g)
+    del warm
     for key in (True, False):
         rows = torch.from_numpy(synth.fit_rows(w, key)).to(dev)
         torch.cuda.synchronize(dev)
@@ -642,33 +674,46 @@ def oracle_sample(w, n_heads):
     return q, kc, vc, np.array([0, T]), kcb, vcb, n_heads, T
 
 
-def time_oracle_step(w, sample):
+def time_oracle_step(w, sample, threads=1):
     from oracle import oracle as O
     q, kc, vc, offs, kcb, vcb, n_heads, T = sample
     t0 = time.perf_counter()
     if w.v_bits:
         O.attend_binv(q, kc, vc, offs, kcb, vcb, w.rope_base)
     else:
-        O.attend_codes(q, kc, vc, offs, kcb, vcb, w.rope_base)
+        O.attend_codes(q, kc, vc, offs, kcb, vcb, w.rope_base, threads=threads)
     dt = time.perf_counter() - t0
     tokens = T * n_heads / w.q_heads        # context tokens of the full step this sample covers
     return dt, tokens
 
 
 def cpu_baseline(w, n_heads, min_seconds=10.0):
-    """The oracle on a bounded sample: n_heads query heads of sequence 0, repeated until at
-    least min_seconds of CPU time have been spent (about 10-30 s)."""
+    """The oracle on a bounded sample: n_heads query heads of sequence 0, repeated until at least
+    min_seconds of wall time have been spent, once single-threaded and once on every core this
+    process may use (the oracle's threaded face: one KV head's query group per thread, the same
+    single-threaded C calls). The multi-threaded figure is the line's baseline."""
+    from oracle import oracle as O
     sample = oracle_sample(w, n_heads)
-    total_dt, total_tok, reps = 0.0, 0.0, 0
-    while total_dt < min_seconds or reps == 0:
-        dt, tokens = time_oracle_step(w, sample)
-        total_dt += dt
-        total_tok += tokens
-        reps += 1
-    return {"value": total_tok / total_dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{sample[6]} of {w.q_heads} query heads of sequence 0 (T={sample[7]}), "
-                      f"single-threaded C oracle in fp64, {reps} repetitions, {total_dt:.1f} s",
-            "seconds": total_dt, "cpu": cpu_model()}
+
+    def timed(threads):
+        total_dt, total_tok, reps = 0.0, 0.0, 0
+        while total_dt < min_seconds or reps == 0:
+            dt, tokens = time_oracle_step(w, sample, threads)
+            total_dt += dt
+            total_tok += tokens
+            reps += 1
+        return total_tok / total_dt, total_dt, reps
+
+    cores = O.host_threads()
+    n_kv = sample[6] // (w.q_heads // w.kv_heads)
+    threads = max(1, min(cores, n_kv))
+    v1, dt1, r1 = timed(1)
+    vn, dtn, rn = timed(threads)
+    desc = f"{sample[6]} of {w.q_heads} query heads of sequence 0 (T={sample[7]}), C oracle in fp64"
+    return {"value": vn, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{desc}, {threads} threads (one KV head's query group each), {rn} repetitions, {dtn:.1f} s",
+            "seconds": dtn, "cpu": cpu_model(), "host_cores": cores,
+            "single_thread": {"value": v1, "unit": UNIT, "cores": 1, "repetitions": r1, "seconds": dt1}}
 
 
 def cpu_model():

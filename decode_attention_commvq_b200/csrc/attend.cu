@@ -259,6 +259,7 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
                                               const float* v_codebook, float* out, float* lse,
                                               void* workspace, size_t workspace_bytes,
                                               const commvq_attend_options* options, void* stream) {
+  const NvtxRange nvtx_range("commvq_attend_decode");
   const commvq_status cs = check_config(cfg);
   if (cs != COMMVQ_OK) return cs;
   if (B < 0 || max_T < 0) return COMMVQ_ERR_INVALID_ARG;
@@ -362,6 +363,7 @@ extern "C" commvq_status commvq_attend_prepare(const commvq_config* cfg, int32_t
                                                const float* k_codebook, const float* v_codebook,
                                                void* workspace, size_t workspace_bytes,
                                                const commvq_attend_options* options, void* stream) {
+  const NvtxRange nvtx_range("commvq_attend_prepare");
   const commvq_status cs = check_config(cfg);
   if (cs != COMMVQ_OK) return cs;
   if (B < 0 || max_T < 0) return COMMVQ_ERR_INVALID_ARG;
@@ -447,6 +449,7 @@ commvq_status launch_combine(const AttendArgs& a, int S, cudaStream_t st) {
 
 extern "C" commvq_status commvq_workspace_error(const void* workspace, int32_t* device_error,
                                                 void* stream) {
+  const NvtxRange nvtx_range("commvq_workspace_error");
   if (!workspace || !device_error) return COMMVQ_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t v = 0;

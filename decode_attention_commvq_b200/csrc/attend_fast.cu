@@ -2,7 +2,7 @@
 // with 2, 4 or 8 KV heads (up to 8 query heads each), R <= 2 rounds and Nc' <= 256 entries.
 //
 // The attention is the one of attend_mma.cu (and of the table form): each (position, KV head)
-// key is decoded once for its GQA group (sum over rounds of fp16 codebook entries), rotated by
+// key is decoded once for its GQA group (exact fp32 sum over rounds of fp16 codebook entries), rotated by
 // e^{i t theta_p} in fp32 -- the rotation moved onto the decoded key by the commuting-block
 // property of the review's "What carries the argument" (Property 1 / Eq. 7-8) -- and multiplied
 // with the query heads on the tensor cores as two 16-bit terms (value and rounding error). Values
@@ -55,6 +55,19 @@ __device__ __forceinline__ uint4 hadd4(uint4 a, uint4 b) {
   r.z = h2u(__hadd2(u2h(a.z), u2h(b.z)));
   r.w = h2u(__hadd2(u2h(a.w), u2h(b.w)));
   return r;
+}
+
+// f32(low or high fp16 half of w) + x, one instruction (sm_100 mixed precision): with x the other
+// round's entry widened to fp32, the sum of two fp16 entries is exact.
+__device__ __forceinline__ float add_lo(uint32_t w, float x) {
+  float d;
+  asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n add.rn.f32.f16 %0, l, %2;\n}" : "=f"(d) : "r"(w), "f"(x));
+  return d;
+}
+__device__ __forceinline__ float add_hi(uint32_t w, float x) {
+  float d;
+  asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n add.rn.f32.f16 %0, h, %2;\n}" : "=f"(d) : "r"(w), "f"(x));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int k) {
@@ -417,7 +430,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_keys_kernel(AttendArgs a, c
         float acc[4] = {0.f, 0.f, 0.f, 0.f}, accn[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int gs = 0; gs < 2; ++gs) {
-          uint4 e[2];   // rows g, g + 8: group i + 4 gs, rounds summed
+          uint4 e[2], e2[2];   // rows g, g + 8: group i + 4 gs, first and second round's entries
 #pragma unroll
           for (int rr = 0; rr < 2; ++rr) {
             const uint32_t w1 = gs ? cw[rr][0].y : cw[rr][0].x;
@@ -426,7 +439,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_keys_kernel(AttendArgs a, c
             if (R == 2) {
               const uint32_t w2 = gs ? cw[rr][1].y : cw[rr][1].x;
               const uint32_t a2 = kCheck ? img_addr_checked(w2, i, kc[gs][1], Nc, err) : img_addr(w2, kc[gs][1], sel);
-              e[rr] = hadd4(e[rr], ld16(smem, a2));
+              e2[rr] = ld16(smem, a2);
             }
           }
 #pragma unroll
@@ -435,8 +448,13 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_keys_kernel(AttendArgs a, c
             uint32_t hx[2], hy[2], nx[2], ny[2];
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
-              const float2 fA = __half22float2(u2h(word_of(e[rr], 2 * hp)));
-              const float2 fB = __half22float2(u2h(word_of(e[rr], 2 * hp + 1)));
+              float2 fA = __half22float2(u2h(word_of(e[rr], 2 * hp)));
+              float2 fB = __half22float2(u2h(word_of(e[rr], 2 * hp + 1)));
+              if (R == 2) {   // the rounds' sum in fp32 (exact): an fp16 sum would round the key
+                const uint32_t vA = word_of(e2[rr], 2 * hp), vB = word_of(e2[rr], 2 * hp + 1);
+                fA = make_float2(add_lo(vA, fA.x), add_hi(vA, fA.y));
+                fB = make_float2(add_lo(vB, fB.x), add_hi(vB, fB.y));
+              }
               const f32x2 X = pack2(fA.x, fB.x), Y = pack2(fA.y, fB.y);
               const f32x2 Xr = sub2(mul2(X, C[rr][u]), mul2(Y, Sn[rr][u]));
               const f32x2 Yr = fma2(X, Sn[rr][u], mul2(Y, C[rr][u]));

@@ -81,10 +81,29 @@ __device__ __forceinline__ float sub_h_f(__half h, float x) {
 // Each rotated pair leaves as two fp16 pairs: hi = (x, y) rounded (h0, h1) and the negated
 // rounding error nlo = hi - (x, y) rounded (n0, n1), so hi - nlo carries x and y to about
 // 2^-22 relative and a product with an fp16 query loses nothing to the fp16 operand type.
-__device__ __forceinline__ void rotate_two(uint32_t w0, uint32_t w1, f32x2 c, f32x2 s, uint32_t& h0,
-                                           uint32_t& h1, uint32_t& n0, uint32_t& n1) {
-  const float2 f0 = __half22float2(u32_as_h2(w0));
-  const float2 f1 = __half22float2(u32_as_h2(w1));
+// f32(low or high fp16 half of w) + x in one instruction (sm_100 mixed precision); the sum of two
+// fp16 entries is exact in fp32.
+__device__ __forceinline__ float addh_lo(uint32_t w, float x) {
+  float d;
+  asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n add.rn.f32.f16 %0, l, %2;\n}" : "=f"(d) : "r"(w), "f"(x));
+  return d;
+}
+__device__ __forceinline__ float addh_hi(uint32_t w, float x) {
+  float d;
+  asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n add.rn.f32.f16 %0, h, %2;\n}" : "=f"(d) : "r"(w), "f"(x));
+  return d;
+}
+
+// kSum: the stored pairs are the sum of w0/w1 (first round) and v0/v1 (second round), formed in fp32.
+template <bool kSum>
+__device__ __forceinline__ void rotate_two(uint32_t w0, uint32_t w1, uint32_t v0, uint32_t v1, f32x2 c, f32x2 s,
+                                           uint32_t& h0, uint32_t& h1, uint32_t& n0, uint32_t& n1) {
+  float2 f0 = __half22float2(u32_as_h2(w0));
+  float2 f1 = __half22float2(u32_as_h2(w1));
+  if (kSum) {
+    f0 = make_float2(addh_lo(v0, f0.x), addh_hi(v0, f0.y));
+    f1 = make_float2(addh_lo(v1, f1.x), addh_hi(v1, f1.y));
+  }
   float c0, c1, s0, s1;
   unpack2(c, c0, c1);
   unpack2(s, s0, s1);
@@ -413,19 +432,18 @@ attend_scores_kernel(AttendArgs a, const QT* __restrict__ q) {
         float accn[4] = {0.f, 0.f, 0.f, 0.f};   // q . nlo
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          uint4 e;
+          uint4 e, e2 = make_uint4(0u, 0u, 0u, 0u);
           int c0 = static_cast<int>(take_byte(word(cw[0], u), sel_i));
           if (kCheck) c0 = clamp_code(c0, Nc, err);
-          if (R == 2) {
+          e = lds128(smem, gF[u] + (c0 << 7));
+          if (R == 2) {   // the second round's entry, added in fp32 (an fp16 sum would round the key)
             int c1 = static_cast<int>(take_byte(word(cw[R - 1], u), sel_i));
             if (kCheck) c1 = clamp_code(c1, Nc, err);
-            e = hadd2x4(lds128(smem, gF[u] + (c0 << 7)), lds128(smem, gS[u] + (c1 << 7)));
-          } else {
-            e = lds128(smem, gF[u] + (c0 << 7));
+            e2 = lds128(smem, gS[u] + (c1 << 7));
           }
           uint32_t h0, h2, n0, n2, h0b, h2b, n0b, n2b;
-          rotate_two(e.x, e.y, pc[2 * u], ps[2 * u], h0, h2, n0, n2);
-          rotate_two(e.z, e.w, pc[2 * u + 1], ps[2 * u + 1], h0b, h2b, n0b, n2b);
+          rotate_two<R == 2>(e.x, e.y, e2.x, e2.y, pc[2 * u], ps[2 * u], h0, h2, n0, n2);
+          rotate_two<R == 2>(e.z, e.w, e2.z, e2.w, pc[2 * u + 1], ps[2 * u + 1], h0b, h2b, n0b, n2b);
           const uint2 b0 = qf[(kv * 8 + 2 * u) * 32 + lane];
           const uint2 b1 = qf[(kv * 8 + 2 * u + 1) * 32 + lane];
           mma16816(acc, h0, 0u, h2, 0u, b0.x, b0.y);

@@ -51,6 +51,7 @@ extern "C" commvq_status commvq_attend_decode_noalloc(
     const void* v_codes, const int64_t* seq_offsets, int32_t B, int64_t max_T,
     const float* k_codebook, const float* v_codebook, float* out, float* lse,
     const commvq_attend_options* options, void* stream) {
+  const NvtxRange nvtx_range("commvq_attend_decode_noalloc");
   // Prepared state would have to survive in the shared array from an earlier call, which any
   // other call on the device (another layer's codebooks, another rope base) may have
   // overwritten since: this entry point always rebuilds it.

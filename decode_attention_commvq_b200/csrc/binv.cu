@@ -631,6 +631,7 @@ extern "C" commvq_status commvq_attend_decode_binv(const commvq_config* cfg, con
                                                    const float* k_codebook, const float* v_codebook, float* out,
                                                    float* lse, void* workspace, size_t workspace_bytes,
                                                    int32_t flags, void* stream) {
+  const NvtxRange nvtx_range("commvq_attend_decode_binv");
   if (!cfg) return COMMVQ_ERR_INVALID_ARG;
   if (B < 0 || max_T < 0 || n_bits <= 0) return COMMVQ_ERR_INVALID_ARG;
   if (q_dtype != COMMVQ_F32 && q_dtype != COMMVQ_F16 && q_dtype != COMMVQ_BF16) return COMMVQ_ERR_INVALID_ARG;

@@ -347,6 +347,7 @@ commvq_status launch_em_hard(const commvq_config* cfg, const float* rows, int64_
 extern "C" commvq_status commvq_em_step(const commvq_config* cfg, const float* rows, int64_t N,
                                         float* codebook_round, void* codes_out, double* sse_out,
                                         void* workspace, size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx_range("commvq_em_step");
   const commvq_status cs = em_check(cfg, N);
   if (cs != COMMVQ_OK) return cs;
   if (!rows || !codebook_round || !workspace) return COMMVQ_ERR_INVALID_ARG;
@@ -368,6 +369,7 @@ extern "C" commvq_status commvq_em_step(const commvq_config* cfg, const float* r
 extern "C" commvq_status commvq_em_step_soft(const commvq_config* cfg, const float* rows, int64_t N,
                                              float* codebook_round, float tau, double* sse_out,
                                              void* workspace, size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx_range("commvq_em_step_soft");
   const commvq_status cs = em_check(cfg, N);
   if (cs != COMMVQ_OK) return cs;
   if (!(tau > 0.0f) || !isfinite(tau)) return COMMVQ_ERR_INVALID_ARG;

@@ -272,6 +272,7 @@ extern "C" commvq_status commvq_encode(const commvq_config* cfg, const void* x, 
                                        int64_t n_tokens, const float* codebook, void* codes,
                                        unsigned long long* near_ties, float* residual_out,
                                        void* stream) {
+  const NvtxRange nvtx_range("commvq_encode");
   const commvq_status cs = check_encode(cfg, x_dtype, n_tokens);
   if (cs != COMMVQ_OK) return cs;
   if (n_tokens == 0) return COMMVQ_OK;
@@ -289,6 +290,7 @@ extern "C" commvq_status commvq_encode_kv(const commvq_config* cfg, const void* 
                                           commvq_dtype x_dtype, int64_t n_tokens, const float* k_codebook,
                                           const float* v_codebook, void* k_codes, void* v_codes,
                                           unsigned long long* near_ties, void* stream) {
+  const NvtxRange nvtx_range("commvq_encode_kv");
   const commvq_status cs = check_encode(cfg, x_dtype, n_tokens);
   if (cs != COMMVQ_OK) return cs;
   if (n_tokens == 0) return COMMVQ_OK;

@@ -587,6 +587,7 @@ extern "C" commvq_status commvq_decompress(const commvq_config* cfg, const void*
                                            const float* k_codebook, const float* v_codebook,
                                            commvq_dtype out_dtype, void* k_out, void* v_out, void* workspace,
                                            size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx_range("commvq_decompress");
   const commvq_status cs = decomp_check(cfg);
   if (cs != COMMVQ_OK) return cs;
   if (B < 0 || max_T < 0) return COMMVQ_ERR_INVALID_ARG;
@@ -673,6 +674,7 @@ extern "C" commvq_status commvq_dense_decode(const commvq_config* cfg, const voi
                                              const int64_t* seq_offsets, int32_t B, int64_t max_T, float* out,
                                              float* lse, void* workspace, size_t workspace_bytes,
                                              const commvq_attend_options* options, void* stream) {
+  const NvtxRange nvtx_range("commvq_dense_decode");
   if (!cfg) return COMMVQ_ERR_INVALID_ARG;
   if (cfg->q_heads < 1 || cfg->kv_heads < 1 || cfg->q_heads % cfg->kv_heads || cfg->d <= 0)
     return COMMVQ_ERR_INVALID_ARG;

@@ -96,3 +96,23 @@ def near_tie_case(order):
     """Codebook [1, 1, len(order), 8] float32 and one zero row [1, 8] for a planted case."""
     cb = np.array([[[NEAR_TIE_ENTRIES[k] for k in order]]], dtype=np.float32)
     return cb, np.zeros((1, 8), dtype=np.float32)
+
+
+class Guarded:
+    """A device buffer with 256 canary bytes (0xA5) on each side: `t` is the caller's tensor (16-
+    and 256-byte alignment kept), `intact()` tells whether the kernels wrote only inside it."""
+    PAD = 256
+    CANARY = 0xA5
+
+    def __init__(self, shape, dtype, device):
+        import torch
+        n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        self.n = n
+        self.raw = torch.full((n + 2 * self.PAD,), self.CANARY, dtype=torch.uint8, device=device)
+        self.t = self.raw[self.PAD:self.PAD + n].view(dtype).view(shape)
+
+    def intact(self) -> bool:
+        import torch
+        r = self.raw
+        return bool(torch.all(r[:self.PAD] == self.CANARY).item() and
+                    torch.all(r[self.PAD + self.n:] == self.CANARY).item())

@@ -7,7 +7,7 @@ import torch
 
 from decode_attention_commvq_b200 import synth
 from oracle import oracle as O
-from tests.helpers import oracle_codebooks, q_as_f64, rel_err, to_torch_q, tol_for
+from tests.helpers import Guarded, oracle_codebooks, q_as_f64, rel_err, to_torch_q, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -30,14 +30,22 @@ def _codes_np_to_gpu(c, gpu):
 
 
 def _run(api, w, q_np, kc, vc, offs, kcb, vcb, gpu, algo=0, splits=0):
+    """One attention call with out, lse and the workspace inside canary guard bands, which must
+    be untouched afterwards."""
     cfg = _cfg(api, w)
     q = to_torch_q(q_np, w.q_dtype, gpu)
     offsets = torch.from_numpy(offs.astype(np.int64)).to(gpu)
     max_T = int(np.diff(offs).max()) if len(offs) > 1 else 0
+    B = len(offs) - 1
+    out_g = Guarded((B, w.q_heads, w.d), torch.float32, gpu)
+    lse_g = Guarded((B, w.q_heads), torch.float32, gpu)
+    ws_g = Guarded((api.attend_workspace_bytes(cfg, B, max_T, algo, splits),), torch.uint8, gpu)
     out, lse = api.attend_decode(cfg, q, _codes_np_to_gpu(kc, gpu), _codes_np_to_gpu(vc, gpu),
                                  offsets, max_T, torch.from_numpy(kcb).to(gpu),
-                                 torch.from_numpy(vcb).to(gpu), algo=algo, splits=splits)
+                                 torch.from_numpy(vcb).to(gpu), out=out_g.t, lse=lse_g.t, workspace=ws_g.t,
+                                 algo=algo, splits=splits)
     torch.cuda.synchronize()
+    assert out_g.intact() and lse_g.intact() and ws_g.intact(), "a kernel wrote outside its buffer"
     return out.cpu().numpy(), lse.cpu().numpy()
 
 

@@ -128,3 +128,27 @@ def test_soft_em_deterministic_and_small_codebooks(api, gpu):
     assert np.array_equal(a.view(np.uint32), b.view(np.uint32)) and sa == sb
     want, _ = O.em_soft_step(rows, cb, 2.0)
     assert np.abs(a - want).max() <= 2e-5 * np.abs(want).max()
+
+
+def test_checkpointed_fit_resumes_bit_for_bit(gpu, tmp_path):
+    """The GPU codebook fit (fit.py) saved after every EM step, interrupted part-way through round
+    1 and resumed from the file, ends with the uninterrupted fit's codebook bit for bit."""
+    from decode_attention_commvq_b200 import fit
+    w = synth.WORKLOADS[1].with_(em_rows=1024, em_iters=3)
+    rows = torch.from_numpy(synth.fit_rows(w, True)).to(gpu)
+    init = lambda r, N: synth.forgy_indices(w, True, r, N)
+    full = fit.fit_codebook(rows, w.R, w.n_codes, w.em_iters, init)
+    p = str(tmp_path / "k.bin")
+
+    class Stop(Exception):
+        pass
+
+    def stop(r, it):
+        if (r, it) == (1, 0):
+            raise Stop()
+
+    with pytest.raises(Stop):
+        fit.fit_codebook(rows, w.R, w.n_codes, w.em_iters, init, checkpoint=p, seed=1, on_step=stop)
+    resumed = fit.fit_codebook(rows, w.R, w.n_codes, w.em_iters, init, checkpoint=p, seed=1)
+    torch.cuda.synchronize()
+    assert torch.equal(full, resumed)

@@ -2,11 +2,12 @@
 numpy around oracle values, against the oracle's exact attention (CommVQ machine review, "What
 carries the argument": decoding is a sum of codewords; the bound is the bf16-input tolerance).
 
-Roundings emulated: key and value codebook entries to fp16 and their R-round sums in fp16, the
-rotation in fp64 (the kernel's fp32 rotation adds ~1e-7), and the rotated key either rounded to
-one fp16 operand or carried as two fp16 terms (the kernel's choice, exact to ~2^-22). The test
-pins the design decision: one fp16 operand leaves the worst head near the 5e-3 bound, the
-two-term operand keeps a clear margin."""
+Roundings emulated: key and value codebook entries to fp16; the keys' R-round sum exact (the
+kernels add the rounds in fp32) and the values' R-round sum in fp16; the rotation in fp64 (the
+kernel's fp32 rotation adds ~1e-7); and the rotated key either rounded to one fp16 operand or
+carried as two 16-bit terms (the kernels' choice, exact to ~2^-16 or better). The tests pin the
+design decisions: one fp16 operand, or an fp16 sum of the key rounds, leaves the worst head near
+or past the 5e-3 bound; the kernels' roundings keep a clear margin."""
 import numpy as np
 
 from decode_attention_commvq_b200 import synth
@@ -18,13 +19,14 @@ def _f16(x):
     return x.astype(np.float16).astype(np.float64)
 
 
-def _decode_f16(codes, cb16):
+def _decode_f16(codes, cb16, sum16=True):
+    """Sum of fp16 entries; each partial sum rounded to fp16 when sum16 (else exact)."""
     R, G, Nc, g = cb16.shape
     out = np.zeros(codes.shape[:2] + (G, g))
     for r in range(R):
         for j in range(G):
             e = cb16[r, j][codes[:, :, r, j]]
-            out[:, :, j] = _f16(out[:, :, j] + e) if r else e
+            out[:, :, j] = (_f16(out[:, :, j] + e) if sum16 else out[:, :, j] + e) if r else e
     return out.reshape(codes.shape[:2] + (G * g,))
 
 
@@ -36,7 +38,7 @@ def test_two_term_rotated_keys_keep_a_margin():
     offs = w.offsets()
     k_exact = O.rope_cache(O.decode(kc, kcb), offs, w.rope_base)
     v_exact = O.decode(vc, vcb)
-    k16 = O.rope_cache(_decode_f16(kc, _f16(kcb)), offs, w.rope_base)   # entries and sums in fp16
+    k16 = O.rope_cache(_decode_f16(kc, _f16(kcb), sum16=False), offs, w.rope_base)   # fp16 entries, exact sum
     v16 = _decode_f16(vc, _f16(vcb))
     one_term, two_term = 0.0, 0.0
     for seed in (1, 2, 3, 4):
@@ -48,6 +50,26 @@ def test_two_term_rotated_keys_keep_a_margin():
         two_term = max(two_term, rel_err(o2, ref))
     assert two_term <= 0.8 * TOL_BF16, two_term
     assert one_term > two_term
+
+
+def test_key_rounds_summed_exactly_at_full_length():
+    """All 32 heads over 32768 positions of the 2-bit layer with uniform codes (the full-size
+    parity workload): with the kernels' roundings the worst head stays well inside the bound;
+    summing the two key rounds in fp16 instead would take it past the bound."""
+    w = synth.WORKLOADS[1]
+    kcb, vcb = oracle_codebooks(w)
+    offs = w.offsets()
+    T = int(offs[-1])
+    kc = synth.uniform_codes(w, True, T)
+    vc = synth.uniform_codes(w, False, T)
+    q = q_as_f64(w, synth.queries(w))
+    ref, _ = O.attend_dense(q, O.rope_cache(O.decode(kc, kcb), offs, w.rope_base), O.decode(vc, vcb), offs)
+    v16 = _decode_f16(vc, _f16(vcb))
+    kernel_like, _ = O.attend_dense(q, O.rope_cache(_decode_f16(kc, _f16(kcb), sum16=False), offs, w.rope_base),
+                                    v16, offs)
+    fp16_key_sum, _ = O.attend_dense(q, O.rope_cache(_decode_f16(kc, _f16(kcb)), offs, w.rope_base), v16, offs)
+    assert rel_err(kernel_like, ref) <= 0.6 * TOL_BF16
+    assert rel_err(fp16_key_sum, ref) > TOL_BF16
 
 
 def test_binary_value_weights_in_three_digits_add_almost_nothing():
