@@ -2,12 +2,15 @@
 // with 2, 4 or 8 KV heads (up to 8 query heads each), R <= 2 rounds and Nc' <= 256 entries.
 //
 // The attention is the one of attend_mma.cu (and of the table form): each (position, KV head)
-// key is decoded once for its GQA group (exact fp32 sum over rounds of fp16 codebook entries), rotated by
-// e^{i t theta_p} in fp32 -- the rotation moved onto the decoded key by the commuting-block
-// property of the review's "What carries the argument" (Property 1 / Eq. 7-8) -- and multiplied
-// with the query heads on the tensor cores as two 16-bit terms (value and rounding error). Values
-// are decoded the same way and the softmax weights multiply them on the tensor cores ("If this is
-// right": weights meet the value codes before the codebook multiply).
+// key is decoded once for its GQA group (exact fp32 sum over rounds of fp16 codebook entries),
+// rotated by e^{i t theta_p} in fp32 -- the rotation moved onto the decoded key by the
+// commuting-block property of the review's "What carries the argument" (Property 1 / Eq. 7-8) --
+// and multiplied with the query heads on the tensor cores as one fp16 operand. (With the rounds
+// summed exactly, one fp16 rounding of the rotated key keeps the worst head of every parity
+// workload at <= 4.2e-3 against the 5e-3 bound; the two-term operand of attend_mma.cu cost a
+// fifth of this kernel's instructions.) Values are decoded the same way and the softmax weights
+// multiply them on the tensor cores ("If this is right": weights meet the value codes before
+// the codebook multiply).
 //
 // What differs from attend_mma.cu is the work split, chosen to spend fewer instructions per
 // (position, KV head):
@@ -70,6 +73,14 @@ __device__ __forceinline__ float add_hi(uint32_t w, float x) {
   return d;
 }
 
+// 2^x for x <= 0 (a softmax weight relative to a maximum), the hardware approximation (relative
+// error ~2^-22, far below the fp16 rounding the weight then takes).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int k) {
   return k == 0 ? v.x : (k == 1 ? v.y : (k == 2 ? v.z : v.w));
 }
@@ -109,61 +120,21 @@ __device__ __forceinline__ uint32_t img_addr_checked(uint32_t code_word, int b, 
   return cst | (c << 8);
 }
 
-// 16-bit mma operand types: the key terms take the query's type (bf16 queries stay exact).
-template <typename KT>
-struct Op16;
-template <>
-struct Op16<__half> {
-  __device__ static __forceinline__ uint32_t pack(float lo, float hi) { return h2u(__floats2half2_rn(lo, hi)); }
-  // f32(low or high half of w) - x in one instruction (sm_100 mixed precision)
-  __device__ static __forceinline__ float sub_lo(uint32_t w, float x) {
-    float d;
-    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n sub.rn.f32.f16 %0, l, %2;\n}" : "=f"(d) : "r"(w), "f"(x));
-    return d;
-  }
-  __device__ static __forceinline__ float sub_hi(uint32_t w, float x) {
-    float d;
-    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n sub.rn.f32.f16 %0, h, %2;\n}" : "=f"(d) : "r"(w), "f"(x));
-    return d;
-  }
-  __device__ static __forceinline__ void mma(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                             uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};\n"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-  }
-};
-template <>
-struct Op16<__nv_bfloat16> {
-  __device__ static __forceinline__ uint32_t pack(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-  }
-  __device__ static __forceinline__ float sub_lo(uint32_t w, float x) {
-    float d;
-    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n sub.rn.f32.bf16 %0, l, %2;\n}" : "=f"(d) : "r"(w), "f"(x));
-    return d;
-  }
-  __device__ static __forceinline__ float sub_hi(uint32_t w, float x) {
-    float d;
-    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n sub.rn.f32.bf16 %0, h, %2;\n}" : "=f"(d) : "r"(w), "f"(x));
-    return d;
-  }
-  __device__ static __forceinline__ void mma(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                             uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};\n"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-  }
-};
+// Two fp32 values to fp16x2 (low half = lo), rounded to nearest, finite values saturating at
+// +-65504 (a query component outside the fp16 range cannot become inf).
+__device__ __forceinline__ uint32_t pack_f16_sat(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
 
 __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                         uint32_t b0, uint32_t b1) {
-  Op16<__half>::mma(c, a0, a1, a2, a3, b0, b1);
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 template <typename QT>
@@ -251,14 +222,13 @@ __global__ void fast_prep_kernel(AttendArgs a, int R) {
 // finalises the first half of its KV heads, the warp of half 1 the rest: it adds the partner's
 // partial scores (shared memory, in the order half 0 + half 1), scales them to the exp2 domain,
 // stores them in the score buffer and keeps their maxima.
-template <int R, int KV, typename KT, typename QT, bool kCheck>
+template <int R, int KV, typename QT, bool kCheck>
 __global__ void __launch_bounds__(kFThreads, 1) fast_keys_kernel(AttendArgs a, const QT* __restrict__ q) {
   constexpr int MK = KV / 2;                  // KV heads per warp
   constexpr int kFin = MK > 1 ? MK / 2 : 1;   // KV heads each warp of a pair finalises (KV = 2: half 0 only)
   constexpr int kRec = KV * R * 16;
   constexpr int kRowStride = kRec + 16;
   constexpr int kStageBytes = kFStage * kRowStride;
-  using Op = Op16<KT>;
   extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* stages = smem + kFImg;                                          // [2][64 rows][kRowStride]
   uint2* qf = reinterpret_cast<uint2*>(stages + 2 * kStageBytes);                 // [KV][2 hf][4 u][32 lanes]
@@ -298,8 +268,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_keys_kernel(AttendArgs a, c
     if (col < G) {
       const QT* qh = q + (static_cast<int64_t>(b) * a.q_heads + kv * G + col) * kD;
       const int pA = 4 * (8 * hf2 + ii + 4 * (u >> 1)) + 2 * (u & 1), pB = pA + 1;
-      v.x = Op::pack(qget(qh, 2 * pA), qget(qh, 2 * pB));
-      v.y = Op::pack(qget(qh, 2 * pA + 1), qget(qh, 2 * pB + 1));
+      v.x = pack_f16_sat(qget(qh, 2 * pA), qget(qh, 2 * pB));
+      v.y = pack_f16_sat(qget(qh, 2 * pA + 1), qget(qh, 2 * pB + 1));
     }
     qf[e] = v;
   }
@@ -427,7 +397,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_keys_kernel(AttendArgs a, c
           if (!valid1) { cw[1][0] = make_uint2(0u, 0u); cw[1][1] = make_uint2(0u, 0u); }
         }
         const uint2* qk = qf + ((kv * 2 + hf) * 4) * 32 + lane;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f}, accn[4] = {0.f, 0.f, 0.f, 0.f};
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int gs = 0; gs < 2; ++gs) {
           uint4 e[2], e2[2];   // rows g, g + 8: group i + 4 gs, first and second round's entries
@@ -445,7 +415,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_keys_kernel(AttendArgs a, c
 #pragma unroll
           for (int hp = 0; hp < 2; ++hp) {
             const int u = 2 * gs + hp;
-            uint32_t hx[2], hy[2], nx[2], ny[2];
+            uint32_t hx[2], hy[2];
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
               float2 fA = __half22float2(u2h(word_of(e[rr], 2 * hp)));
@@ -461,19 +431,14 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_keys_kernel(AttendArgs a, c
               float xA, xB, yA, yB;
               unpack2(Xr, xA, xB);
               unpack2(Yr, yA, yB);
-              hx[rr] = Op::pack(xA, xB);
-              hy[rr] = Op::pack(yA, yB);
-              nx[rr] = Op::pack(Op::sub_lo(hx[rr], xA), Op::sub_hi(hx[rr], xB));
-              ny[rr] = Op::pack(Op::sub_lo(hy[rr], yA), Op::sub_hi(hy[rr], yB));
+              hx[rr] = h2u(__floats2half2_rn(xA, xB));
+              hy[rr] = h2u(__floats2half2_rn(yA, yB));
             }
             const uint2 qb = qk[u * 32];
-            Op::mma(acc, hx[0], hx[1], hy[0], hy[1], qb.x, qb.y);
-            Op::mma(accn, nx[0], nx[1], ny[0], ny[1], qb.x, qb.y);
+            mma_f16(acc, hx[0], hx[1], hy[0], hy[1], qb.x, qb.y);
           }
         }
-        float d[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) d[k] = acc[k] - accn[k];
+        const float* d = acc;
         // d: (row g, col 2i), (row g, col 2i + 1), (row g + 8, col 2i), (row g + 8, col 2i + 1)
         // the first kFin KV heads are finalised by the half-0 warp, the rest by the half-1 warp
         // (compile-time slots: no local memory)
@@ -681,7 +646,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_values_kernel(AttendArgs a)
         const float sk[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          if (tau[k] < rem) p[k] = exp2f(sk[k] - m_h);
+          if (tau[k] < rem) p[k] = ex2(sk[k] - m_h);
           lsum += p[k];
         }
       }
@@ -774,9 +739,9 @@ commvq_status launch_fast_rkc(const AttendArgs& a, const void* q, commvq_dtype q
   const size_t smem_v = fast_values_smem_bytes(R, KV, a.q_heads);
   dim3 grid(S, a.B);
   if (a.main_start && record_event(a.main_start, st) != cudaSuccess) return COMMVQ_ERR_CUDA;
-#define COMMVQ_FAST_KEYS(KT, QT)                                                                      \
+#define COMMVQ_FAST_KEYS(QT)                                                                          \
   {                                                                                                   \
-    auto k = fast_keys_kernel<R, KV, KT, QT, kCheck>;                                                 \
+    auto k = fast_keys_kernel<R, KV, QT, kCheck>;                                                     \
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_k) != cudaSuccess) \
       return COMMVQ_ERR_CUDA;                                                                         \
     const QT* qq = static_cast<const QT*>(q);                                                         \
@@ -787,9 +752,9 @@ commvq_status launch_fast_rkc(const AttendArgs& a, const void* q, commvq_dtype q
     }                                                                                                 \
   }
   switch (qt) {
-    case COMMVQ_F32: COMMVQ_FAST_KEYS(__half, float) break;
-    case COMMVQ_F16: COMMVQ_FAST_KEYS(__half, __half) break;
-    case COMMVQ_BF16: COMMVQ_FAST_KEYS(__nv_bfloat16, __nv_bfloat16) break;
+    case COMMVQ_F32: COMMVQ_FAST_KEYS(float) break;
+    case COMMVQ_F16: COMMVQ_FAST_KEYS(__half) break;
+    case COMMVQ_BF16: COMMVQ_FAST_KEYS(__nv_bfloat16) break;
     default: return COMMVQ_ERR_UNSUPPORTED;
   }
 #undef COMMVQ_FAST_KEYS

@@ -4,10 +4,10 @@ carries the argument": decoding is a sum of codewords; the bound is the bf16-inp
 
 Roundings emulated: key and value codebook entries to fp16; the keys' R-round sum exact (the
 kernels add the rounds in fp32) and the values' R-round sum in fp16; the rotation in fp64 (the
-kernel's fp32 rotation adds ~1e-7); and the rotated key either rounded to one fp16 operand or
-carried as two 16-bit terms (the kernels' choice, exact to ~2^-16 or better). The tests pin the
-design decisions: one fp16 operand, or an fp16 sum of the key rounds, leaves the worst head near
-or past the 5e-3 bound; the kernels' roundings keep a clear margin."""
+kernel's fp32 rotation adds ~1e-7); and the rotated key rounded to one fp16 operand (the fast
+kernels, attend_fast.cu) or carried as two fp16 terms (attend_mma.cu, exact to ~2^-22). The tests
+pin the design decisions: with the key rounds summed exactly, one fp16 operand keeps the worst
+head clear of the 5e-3 bound; an fp16 sum of the key rounds would take it past the bound."""
 import numpy as np
 
 from decode_attention_commvq_b200 import synth
@@ -30,7 +30,7 @@ def _decode_f16(codes, cb16, sum16=True):
     return out.reshape(codes.shape[:2] + (G * g,))
 
 
-def test_two_term_rotated_keys_keep_a_margin():
+def test_rotated_key_operand_keeps_a_margin():
     w = synth.WORKLOADS[1].with_(seq_len=3000)
     kcb, vcb = oracle_codebooks(synth.WORKLOADS[1])
     kc, _ = O.encode(synth.kv_cache_rows(w, True), kcb)
@@ -48,7 +48,8 @@ def test_two_term_rotated_keys_keep_a_margin():
         o2, _ = O.attend_dense(q, k16, v16, offs)
         one_term = max(one_term, rel_err(o1, ref))
         two_term = max(two_term, rel_err(o2, ref))
-    assert two_term <= 0.8 * TOL_BF16, two_term
+    assert one_term <= 0.85 * TOL_BF16, one_term    # the fast kernels
+    assert two_term <= 0.6 * TOL_BF16, two_term     # attend_mma.cu
     assert one_term > two_term
 
 
@@ -65,10 +66,10 @@ def test_key_rounds_summed_exactly_at_full_length():
     q = q_as_f64(w, synth.queries(w))
     ref, _ = O.attend_dense(q, O.rope_cache(O.decode(kc, kcb), offs, w.rope_base), O.decode(vc, vcb), offs)
     v16 = _decode_f16(vc, _f16(vcb))
-    kernel_like, _ = O.attend_dense(q, O.rope_cache(_decode_f16(kc, _f16(kcb), sum16=False), offs, w.rope_base),
-                                    v16, offs)
+    kernel_like, _ = O.attend_dense(q, _f16(O.rope_cache(_decode_f16(kc, _f16(kcb), sum16=False), offs,
+                                                         w.rope_base)), v16, offs)   # one fp16 operand
     fp16_key_sum, _ = O.attend_dense(q, O.rope_cache(_decode_f16(kc, _f16(kcb)), offs, w.rope_base), v16, offs)
-    assert rel_err(kernel_like, ref) <= 0.6 * TOL_BF16
+    assert rel_err(kernel_like, ref) <= 0.8 * TOL_BF16
     assert rel_err(fp16_key_sum, ref) > TOL_BF16
 
 
