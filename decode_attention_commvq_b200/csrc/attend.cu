@@ -285,9 +285,7 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
   if (di.device < 0) return COMMVQ_ERR_CUDA;
   const bool fast = run == COMMVQ_ATTN_DECODE_MMA && use_fast(cfg);
   if (fast) {
-    if (fast_keys_smem_bytes(cfg->R, cfg->kv_heads) > di.smem_optin ||
-        fast_values_smem_bytes(cfg->R, cfg->kv_heads, cfg->q_heads) > di.smem_optin)
-      return COMMVQ_ERR_UNSUPPORTED;
+    if (fast_smem_bytes(cfg->R, cfg->kv_heads, cfg->q_heads) > di.smem_optin) return COMMVQ_ERR_UNSUPPORTED;
   } else if (run == COMMVQ_ATTN_DECODE_MMA) {
     if (mma_scores_smem_bytes(cfg->R, cfg->kv_heads, cfg->n_codes) > di.smem_optin ||
         mma_values_smem_bytes(cfg->R, cfg->kv_heads, cfg->q_heads, cfg->n_codes) > di.smem_optin)
@@ -333,7 +331,7 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
       rc = launch_fast_prep(a, st);   // also clears the error words
       if (rc != COMMVQ_OK) return rc;
     }   // else: the previous call's merge left the running error word clear
-    // the keys kernel copies the prepared state before its dependency wait: launch it as a
+    // the attention kernel copies the prepared state before its dependency wait: launch it as a
     // programmatic dependent only when the kernel before it is not the one writing that state
     rc = launch_attend_fast(a, q, q_dtype, S, st, prepared);
   } else if (run == COMMVQ_ATTN_DECODE_MMA) {

@@ -75,8 +75,9 @@ commvq_status launch_combine(const AttendArgs& a, int splits, cudaStream_t st);
 bool fast_supported(int g, int R, int q_heads, int kv_heads, int n_codes);
 size_t fast_keys_smem_bytes(int R, int KV);
 size_t fast_values_smem_bytes(int R, int KV, int q_heads);
+size_t fast_smem_bytes(int R, int KV, int q_heads);   // the fused kernel's dynamic shared memory
 commvq_status launch_fast_prep(const AttendArgs& a, cudaStream_t st);
-// dependent: launch the keys kernel as a programmatic dependent of the previous kernel (only when
+// dependent: launch the attention kernel as a programmatic dependent of the previous kernel (only when
 // that kernel does not write the prepared state).
 commvq_status launch_attend_fast(const AttendArgs& a, const void* q, commvq_dtype qt, int splits, cudaStream_t st,
                                  bool dependent);

@@ -1,5 +1,5 @@
-// Decode attention on CommVQ codes, decode-and-rotate form: the fast pair of kernels for layers
-// with 2, 4 or 8 KV heads (up to 8 query heads each), R <= 2 rounds and Nc' <= 256 entries.
+// Decode attention on CommVQ codes, decode-and-rotate form: the fast kernel for layers with 2, 4
+// or 8 KV heads (up to 8 query heads each), R <= 2 rounds and Nc' <= 256 entries.
 //
 // The attention is the one of attend_mma.cu (and of the table form): each (position, KV head)
 // key is decoded once for its GQA group (exact fp32 sum over rounds of fp16 codebook entries),
@@ -22,8 +22,9 @@
 //   values : a thread owns 16 value dims (two groups) and four positions of a 16-position tile;
 //            the round sum is one fp16x2 add per word, the transpose into mma fragments one byte
 //            permute per register.
-// Both kernels keep their codebook image (128 KB, fp16) in shared memory, one 512-thread CTA per
-// SM, and stream 64-position stages of code records with 16-byte asynchronous copies.
+// One 512-thread CTA per SM runs both phases over its split of positions: the keys phase with the
+// key codebook image (128 KB, fp16) in shared memory, then the values phase with the value image
+// loaded over it, each streaming stages of code records with 16-byte asynchronous copies.
 //
 // Codebook image layout (per codebook, 128 KB): half h = j / 8 of the 16 groups at h * 64 KB;
 // entry (v, j, c) -- v the round, or for one round a copy index -- at byte
@@ -223,13 +224,14 @@ __global__ void fast_prep_kernel(AttendArgs a, int R) {
 // partial scores (shared memory, in the order half 0 + half 1), scales them to the exp2 domain,
 // stores them in the score buffer and keeps their maxima.
 template <int R, int KV, typename QT, bool kCheck>
-__global__ void __launch_bounds__(kFThreads, 1) fast_keys_kernel(AttendArgs a, const QT* __restrict__ q) {
+__device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __restrict__ q, unsigned char* smem,
+                                           int64_t row0, int64_t t_begin, int64_t t_end, Partial* part,
+                                           float* msplit) {
   constexpr int MK = KV / 2;                  // KV heads per warp
   constexpr int kFin = MK > 1 ? MK / 2 : 1;   // KV heads each warp of a pair finalises (KV = 2: half 0 only)
   constexpr int kRec = KV * R * 16;
   constexpr int kRowStride = kRec + 16;
   constexpr int kStageBytes = kFStage * kRowStride;
-  extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* stages = smem + kFImg;                                          // [2][64 rows][kRowStride]
   uint2* qf = reinterpret_cast<uint2*>(stages + 2 * kStageBytes);                 // [KV][2 hf][4 u][32 lanes]
   float* xbuf = reinterpret_cast<float*>(qf + KV * 2 * 4 * 32);                  // [2][4 rt][KV][16][8]
@@ -239,17 +241,14 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_keys_kernel(AttendArgs a, c
 
   const int Nc = kCheck ? a.n_codes : 256;
   const int G = a.q_heads / KV;
-  const int s = blockIdx.x, b = blockIdx.y, S = gridDim.x;
+  const int b = blockIdx.y, S = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, i = lane & 3;
   const int rt = warp >> 2, hf = (warp >> 1) & 1, kg = warp & 1;
-  int64_t row0, t_begin, t_end;
-  fast_split(a, b, s, S, row0, t_begin, t_end);
-  Partial* part = a.partials + static_cast<int64_t>(b) * a.q_heads * S + s;
 
   // Prepared state (codebook image, advance phasors) and the queries are not written by the
   // kernel this one may follow as a programmatic dependent: copy and form them before the wait.
-  if (t_begin < t_end) {
+  {
     const uint4* src = a.k_img;
     uint4* dst = reinterpret_cast<uint4*>(smem);
     const int n16 = (kFImgHalf / 16);
@@ -281,12 +280,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_keys_kernel(AttendArgs a, c
     advt[tid] = make_float4(cA.x, cB.x, cA.y, cB.y);
   }
   pdl_wait();
-  if (t_begin >= t_end) {
-    for (int h = tid; h < a.q_heads; h += kFThreads) part[static_cast<int64_t>(h) * S].m = -INFINITY;
-    cp_async_wait<0>();
-    return;
-  }
-  pdl_trigger();   // the values kernel may take SMs as this grid's CTAs finish
+  pdl_trigger();   // the merge kernel may be scheduled; it waits for this grid
 
   fast_issue_stage<kRec>(stages, a.k_codes, row0, t_begin, t_end);
   cp_async_commit();
@@ -517,6 +511,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_keys_kernel(AttendArgs a, c
 #pragma unroll
     for (int r2 = 0; r2 < kFStageTiles; ++r2) m = fmaxf(m, mred[r2 * KV * 8 + e]);
     part[static_cast<int64_t>(kv * G + col) * S].m = m;
+    msplit[kv * G + col] = m;
   }
   if (kCheck) {
     err = __syncthreads_or(err);
@@ -533,39 +528,24 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_keys_kernel(AttendArgs a, c
 // ((i >> 1) ^ (n >> 1)) & 1, so the lanes of a quarter-warp read eight different (round, group)
 // slots; lanes with odd i swap the two group sums back.
 template <int R, int KV, bool kCheck>
-__global__ void __launch_bounds__(kFThreads, 1) fast_values_kernel(AttendArgs a) {
+__device__ __forceinline__ void values_phase(const AttendArgs& a, unsigned char* smem, int64_t row0, int64_t t_begin,
+                                             int64_t t_end, Partial* part, const float* msplit) {
   constexpr int WPK = kFWarps / KV;
   constexpr int kTiles = WPK > kFStageTiles ? WPK : kFStageTiles;
   constexpr int kStageT = kFTile * kTiles;
   constexpr int kRec = KV * R * 16;
   constexpr int kRowStride = kRec + 16;
   constexpr int kStageBytes = kStageT * kRowStride;
-  extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* stages = smem + kFImg;                       // [2][kStageT][kRowStride]
   unsigned char* sstage = stages + 2 * kStageBytes;            // [2][kTiles][Hq][16] floats
 
   const int Nc = kCheck ? a.n_codes : 256;
   const int G = a.q_heads / KV;
-  const int s = blockIdx.x, b = blockIdx.y, S = gridDim.x;
+  const int b = blockIdx.y, S = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, i = lane & 3;
   const int kv = warp / WPK, sub = warp % WPK;
   const int score_stage_bytes = kTiles * a.q_heads * kFTile * 4;
-  int64_t row0, t_begin, t_end;
-  fast_split(a, b, s, S, row0, t_begin, t_end);
-  Partial* part = a.partials + static_cast<int64_t>(b) * a.q_heads * S + s;
-
-  if (t_begin >= t_end) {
-    pdl_wait();
-    for (int e = tid; e < a.q_heads * (kD + 1); e += kFThreads) {
-      const int h = e / (kD + 1), d = e % (kD + 1);
-      if (d < kD)
-        part[static_cast<int64_t>(h) * S].o[d] = 0.0f;
-      else
-        part[static_cast<int64_t>(h) * S].l = 0.0f;
-    }
-    return;
-  }
   const int64_t n_tiles = (a.max_T + kFTile - 1) / kFTile;
   auto issue_codes = [&](unsigned char* dst, int64_t t0) {
     constexpr int kPieces = kRec / 16;
@@ -585,8 +565,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_values_kernel(AttendArgs a)
     for (int p = tid; p < pieces; p += kFThreads) cp_async16(dst + p * 16, src + p * 16);
   };
 
-  pdl_trigger();   // the merge may be scheduled as SMs free up; it waits for this grid
-  {   // prepared image and the first code stage: not written by the scores kernel
+  {   // the value image replaces the key image (the keys phase is done with it)
     const uint4* src = a.v_img;
     uint4* dst = reinterpret_cast<uint4*>(smem);
     const int n16 = (kFImgHalf / 16);
@@ -596,11 +575,10 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_values_kernel(AttendArgs a)
     }
   }
   issue_codes(stages, t_begin);
-  pdl_wait();   // the scores kernel's maxima and score buffer are complete from here on
-  issue_scores(sstage, t_begin);
+  issue_scores(sstage, t_begin);   // written by this CTA's keys phase (fenced before the barrier)
   cp_async_commit();
 
-  const float m_h = (g < G) ? part[static_cast<int64_t>(kv * G + g) * S].m : 0.0f;
+  const float m_h = (g < G) ? msplit[kv * G + g] : 0.0f;
   float O[8][4];
 #pragma unroll
   for (int m = 0; m < 8; ++m) O[m][0] = O[m][1] = O[m][2] = O[m][3] = 0.0f;
@@ -732,38 +710,67 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_values_kernel(AttendArgs a)
   }
 }
 
+// One CTA per (split, sequence): the keys phase (scores of the split into the L2-resident score
+// buffer, the split's maxima), then, in the same shared memory, the values phase with the split's
+// own maxima -- no grid-wide dependency between the two. msplit_off: byte offset of the split
+// maxima in shared memory (past both phases' buffers).
+template <int R, int KV, typename QT, bool kCheck>
+__global__ void __launch_bounds__(kFThreads, 1) fast_attend_kernel(AttendArgs a, const QT* __restrict__ q,
+                                                                    int msplit_off) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  float* msplit = reinterpret_cast<float*>(smem + msplit_off);
+  const int s = blockIdx.x, b = blockIdx.y, S = gridDim.x;
+  int64_t row0, t_begin, t_end;
+  fast_split(a, b, s, S, row0, t_begin, t_end);
+  Partial* part = a.partials + static_cast<int64_t>(b) * a.q_heads * S + s;
+  if (t_begin >= t_end) {   // an empty split: m = -inf, o = 0, l = 0
+    pdl_wait();
+    pdl_trigger();
+    for (int e = threadIdx.x; e < a.q_heads * (kD + 2); e += kFThreads) {
+      const int h = e / (kD + 2), d = e % (kD + 2);
+      Partial* ph = part + static_cast<int64_t>(h) * S;
+      if (d < kD)
+        ph->o[d] = 0.0f;
+      else if (d == kD)
+        ph->l = 0.0f;
+      else
+        ph->m = -INFINITY;
+    }
+    return;
+  }
+  keys_phase<R, KV, QT, kCheck>(a, q, smem, row0, t_begin, t_end, part, msplit);
+  __threadfence();   // the score buffer rows written above are read back by asynchronous copies
+  __syncthreads();
+  values_phase<R, KV, kCheck>(a, smem, row0, t_begin, t_end, part, msplit);
+}
+
 template <int R, int KV, bool kCheck>
 commvq_status launch_fast_rkc(const AttendArgs& a, const void* q, commvq_dtype qt, int S, cudaStream_t st,
                               bool dependent) {
-  const size_t smem_k = fast_keys_smem_bytes(R, KV);
-  const size_t smem_v = fast_values_smem_bytes(R, KV, a.q_heads);
+  const size_t smem = fast_smem_bytes(R, KV, a.q_heads);
+  const size_t smem_main = smem - 64 * sizeof(float);   // the split maxima sit past both phases' buffers
   dim3 grid(S, a.B);
   if (a.main_start && record_event(a.main_start, st) != cudaSuccess) return COMMVQ_ERR_CUDA;
-#define COMMVQ_FAST_KEYS(QT)                                                                          \
+#define COMMVQ_FAST(QT)                                                                               \
   {                                                                                                   \
-    auto k = fast_keys_kernel<R, KV, QT, kCheck>;                                                     \
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_k) != cudaSuccess) \
+    auto k = fast_attend_kernel<R, KV, QT, kCheck>;                                                   \
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)   \
       return COMMVQ_ERR_CUDA;                                                                         \
     const QT* qq = static_cast<const QT*>(q);                                                         \
+    const int off = static_cast<int>(smem_main);                                                      \
     if (dependent) {                                                                                  \
-      if (launch_dependent(k, grid, dim3(kFThreads), smem_k, st, a, qq) != cudaSuccess) return COMMVQ_ERR_CUDA; \
+      if (launch_dependent(k, grid, dim3(kFThreads), smem, st, a, qq, off) != cudaSuccess) return COMMVQ_ERR_CUDA; \
     } else {                                                                                          \
-      k<<<grid, kFThreads, smem_k, st>>>(a, qq);                                                      \
+      k<<<grid, kFThreads, smem, st>>>(a, qq, off);                                                   \
     }                                                                                                 \
   }
   switch (qt) {
-    case COMMVQ_F32: COMMVQ_FAST_KEYS(float) break;
-    case COMMVQ_F16: COMMVQ_FAST_KEYS(__half) break;
-    case COMMVQ_BF16: COMMVQ_FAST_KEYS(__nv_bfloat16) break;
+    case COMMVQ_F32: COMMVQ_FAST(float) break;
+    case COMMVQ_F16: COMMVQ_FAST(__half) break;
+    case COMMVQ_BF16: COMMVQ_FAST(__nv_bfloat16) break;
     default: return COMMVQ_ERR_UNSUPPORTED;
   }
-#undef COMMVQ_FAST_KEYS
-  {
-    auto k = fast_values_kernel<R, KV, kCheck>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_v) != cudaSuccess)
-      return COMMVQ_ERR_CUDA;
-    if (launch_dependent(k, grid, dim3(kFThreads), smem_v, st, a) != cudaSuccess) return COMMVQ_ERR_CUDA;
-  }
+#undef COMMVQ_FAST
   if (a.main_stop && record_event(a.main_stop, st) != cudaSuccess) return COMMVQ_ERR_CUDA;
   return launch_status();
 }
@@ -803,6 +810,11 @@ size_t fast_values_smem_bytes(int R, int KV, int q_heads) {
   const size_t xred = static_cast<size_t>(kFWarps) * 32 * 33 * 4;
   if (stages < xred) stages = xred;   // the per-warp sums reuse the code stages after the loop
   return kFImg + stages + static_cast<size_t>(2) * tiles * q_heads * kFTile * 4;
+}
+
+size_t fast_smem_bytes(int R, int KV, int q_heads) {
+  const size_t k = fast_keys_smem_bytes(R, KV), v = fast_values_smem_bytes(R, KV, q_heads);
+  return (k > v ? k : v) + 64 * sizeof(float);
 }
 
 bool fast_supported(int g, int R, int q_heads, int kv_heads, int n_codes) {
