@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--unprepared", action="store_true",
                     help="rebuild the codebook images and RoPE tables in every step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-transfer", default="kernel", choices=["kernel", "copy"],
+                    help="how the end-to-end step moves its inputs and output across the host link")
     ap.add_argument("--cpu-heads", type=int, default=32, help="query heads in the oracle sample")
     return ap.parse_args()
 
@@ -502,26 +504,39 @@ def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, attend, stre
         stage_h[int(o):int(o) + n] = torch.from_numpy(np.ascontiguousarray(x).view(np.uint8).reshape(-1))
     stage_d = torch.empty_like(stage_h, device=dev)
 
+    out_h = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32).pin_memory()
+    out_d = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32, device=dev)
+    # kernel: one commvq_copy_async kernel brings the step's inputs from the pinned host buffer
+    # across the host link, and the merge kernel writes the output straight into the pinned host
+    # output (both mapped at their host addresses under unified addressing); copy: copy-engine
+    # transfers around the kernels
+    mapped = (args.e2e_transfer == "kernel" and not binv and api.host_mapped(stage_h) and api.host_mapped(out_h))
+    src = stage_d
+
     def view(k, dtype, shape):
-        return stage_d[int(offsets[k]):int(offsets[k]) + sizes[k]].view(dtype).view(shape)
+        return src[int(offsets[k]):int(offsets[k]) + sizes[k]].view(dtype).view(shape)
 
     q_d = view(0, torch.bfloat16 if w.q_dtype == "bf16" else torch.float32, q_np.shape)
     kv_d = view(1, torch.float16, kv_new.shape)
     bits_d = view(2, torch.uint8, (1, w.v_bits // 8)) if binv else None
-    out_h = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32).pin_memory()
-    out_d = torch.empty((w.batch, w.q_heads, w.d), dtype=torch.float32, device=dev)
     last = int(w.offsets()[1]) - 1
 
     def step(i):
         kc, vc = kcs[i % n_copies], vcs[i % n_copies]
-        stage_d.copy_(stage_h, non_blocking=True)
+        if mapped:
+            api.copy_async(stage_d, stage_h, stream=stream)
+        else:
+            stage_d.copy_(stage_h, non_blocking=True)
         if binv:   # the value encoder is a learned network: its bits arrive from the host
             vc[last:last + 1].copy_(bits_d, non_blocking=True)
             api.encode(cfg, kv_d[0], kcb, codes=kc[last:last + 1], stream=stream)
         else:      # the new key and value rows in one launch
             api.encode_kv(cfg, kv_d[0], kv_d[1], kcb, vcb, kc[last:last + 1], vc[last:last + 1], stream=stream)
-        attend(kc, vc, q_d, out_d, None, i=i)
-        out_h.copy_(out_d, non_blocking=True)
+        if mapped:
+            attend(kc, vc, q_d, out_h, None, i=i)
+        else:
+            attend(kc, vc, q_d, out_d, None, i=i)
+            out_h.copy_(out_d, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for i in range(W):
@@ -547,8 +562,12 @@ def run_e2e(args, w, cfg, kcb, vcb, kcs, vcs, offs, max_T, total_T, attend, stre
             "h2d_bytes_per_step": int(stage_h.numel()),
             "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()),
             "ms_per_step": ms / K,
-            "note": "one copy of q + the new position's K/V rows (+ value bits) in, encode (K and V rows in one "
-                    "launch) + attend, output out; one CUDA graph of K steps"}
+            "transfer": "kernel" if mapped else "copy",
+            "note": ("q and the new position's K/V rows brought in from pinned host memory by one copy kernel "
+                     "(commvq_copy_async, loads across the host link), the output written by the merge kernel "
+                     "straight into pinned host memory" if mapped else
+                     "one copy of q + the new position's K/V rows (+ value bits) in, output out (copy engine)") +
+                    "; encode (K and V rows in one launch) + attend; one CUDA graph of K steps"}
 
 
 # ---------------------------------------------------------------------------------------

@@ -27,7 +27,7 @@ EXPORTS = ("commvq_encode", "commvq_encode_kv", "commvq_attend_workspace_bytes",
            "commvq_em_step_soft", "commvq_decompress_workspace_bytes", "commvq_decompress",
            "commvq_dense_decode_workspace_bytes", "commvq_dense_decode",
            "commvq_attend_binv_workspace_bytes", "commvq_attend_decode_binv",
-           "commvq_workspace_error", "commvq_status_string", "commvq_abi_version")
+           "commvq_copy_async", "commvq_workspace_error", "commvq_status_string", "commvq_abi_version")
 
 
 class CConfig(ctypes.Structure):
@@ -87,6 +87,8 @@ def _load():
     lib.commvq_attend_binv_workspace_bytes.restype = SZ
     lib.commvq_attend_decode_binv.argtypes = [CP, P, I32, P, P, I32, P, I32, I64, P, P, P, P, P, SZ, I32, P]
     lib.commvq_attend_decode_binv.restype = I32
+    lib.commvq_copy_async.argtypes = [P, P, SZ, P]
+    lib.commvq_copy_async.restype = I32
     lib.commvq_workspace_error.argtypes = [P, ctypes.POINTER(I32), P]
     lib.commvq_workspace_error.restype = I32
     lib.commvq_status_string.argtypes = [I32]
@@ -385,6 +387,29 @@ def attend_decode_binv(cfg: Config, q: torch.Tensor, k_codes: torch.Tensor, v_bi
                                          ATTEND_PREPARED if prepared else 0, _stream(stream)),
            "commvq_attend_decode_binv")
     return out, lse
+
+
+def copy_async(dst: torch.Tensor, src: torch.Tensor, stream=None):
+    """commvq_copy_async: src's bytes into dst by one kernel; either tensor may be device memory or
+    pinned host memory that the device maps at its host address (see host_mapped)."""
+    n = src.numel() * src.element_size()
+    if dst.numel() * dst.element_size() < n:
+        raise ValueError("dst is smaller than src")
+    _check(LIB.commvq_copy_async(_ptr(dst), _ptr(src), n, _stream(stream)), "commvq_copy_async")
+    return dst
+
+
+def host_mapped(t: torch.Tensor) -> bool:
+    """Whether pinned host tensor t is device-accessible at its host address (mapped pinned memory
+    under unified addressing), as the CUDA runtime reports it."""
+    if t.is_cuda or not t.is_pinned():
+        return False
+    try:
+        from cuda.bindings import runtime as rt
+    except Exception:
+        return False
+    err, dptr = rt.cudaHostGetDevicePointer(t.data_ptr(), 0)
+    return err == rt.cudaError_t.cudaSuccess and int(dptr) == t.data_ptr()
 
 
 def workspace_error(workspace: torch.Tensor, stream=None) -> int:

@@ -35,8 +35,9 @@ constexpr size_t kHeaderBytes = 256;   // device error word + padding
 // Grid: (sequence x head, 4 quarters of the 128 output dims), 256 threads = 32 groups of 8
 // lanes. Lane gl of group grp owns float4 gl of the quarter's 32 dims and the splits grp,
 // grp + 32, ...; it issues the loads of (m, l, its float4 of o) for 8 splits at a time before
-// any arithmetic, folds them in with a running maximum, and the 32 groups are merged in a
-// fixed order through shared memory, so one call's result does not depend on timing.
+// any arithmetic, folds them in with a running maximum, and the 32 groups are merged in parallel
+// in a fixed order (shuffles, then the 8 warps' sums), so one call's result does not depend on
+// timing.
 constexpr int kCombineThreads = 256;
 constexpr int kCombineQuarters = 4;
 constexpr int kCombineGroups = kCombineThreads / 8;
@@ -100,22 +101,42 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(AttendArgs a, 
     ml_s[grp][1] = L;
   }
   __syncthreads();
-  if (tid < 8) {
-    float Mg = -INFINITY;
+  // Merge of the 32 groups in parallel, in a fixed order: thread (grp, gl) weights float4 gl of
+  // group grp by 2^(M_grp - Mg); lanes with equal gl add the warp's four groups (xor 8, then 16),
+  // and 8 threads add the 8 warps' sums in warp order.
+  static_assert(kCombineGroups == 32 && kCombineThreads == 256, "one max per lane, 8 warps");
+  __shared__ float4 wsum[kCombineThreads / 32][8];
+  __shared__ float lsum_w[kCombineThreads / 32];
+  const int lane = tid & 31, wid = tid >> 5;
+  float Mg = ml_s[lane][0];
 #pragma unroll
-    for (int g2 = 0; g2 < kCombineGroups; ++g2) Mg = fmaxf(Mg, ml_s[g2][0]);
-    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-    float Lt = 0.0f;
-    if (Mg != -INFINITY) {
-      for (int g2 = 0; g2 < kCombineGroups; ++g2) {
-        const float w = exp2f(ml_s[g2][0] - Mg);
-        const float4 u = acc_s[g2][tid];
-        t.x = fmaf(w, u.x, t.x);
-        t.y = fmaf(w, u.y, t.y);
-        t.z = fmaf(w, u.z, t.z);
-        t.w = fmaf(w, u.w, t.w);
-        Lt = fmaf(w, ml_s[g2][1], Lt);
-      }
+  for (int o = 16; o > 0; o >>= 1) Mg = fmaxf(Mg, __shfl_xor_sync(0xffffffffu, Mg, o));
+  const float w = Mg == -INFINITY ? 0.0f : exp2f(ml_s[grp][0] - Mg);
+  float4 v = acc_s[grp][gl];
+  v = make_float4(w * v.x, w * v.y, w * v.z, w * v.w);
+  float lv = gl == 0 ? w * ml_s[grp][1] : 0.0f;
+#pragma unroll
+  for (int o = 8; o < 32; o <<= 1) {
+    v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
+    v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
+    v.z += __shfl_xor_sync(0xffffffffu, v.z, o);
+    v.w += __shfl_xor_sync(0xffffffffu, v.w, o);
+    lv += __shfl_xor_sync(0xffffffffu, lv, o);
+  }
+  if (lane < 8) wsum[wid][lane] = v;
+  if (lane == 0) lsum_w[wid] = lv;
+  __syncthreads();
+  if (tid < 8) {
+    float4 t = wsum[0][tid];
+    float Lt = lsum_w[0];
+#pragma unroll
+    for (int w2 = 1; w2 < kCombineThreads / 32; ++w2) {
+      const float4 u = wsum[w2][tid];
+      t.x += u.x;
+      t.y += u.y;
+      t.z += u.z;
+      t.w += u.w;
+      Lt += lsum_w[w2];
     }
     const float inv = Lt > 0.0f ? 1.0f / Lt : 0.0f;
     reinterpret_cast<float4*>(a.out + static_cast<int64_t>(bh) * kD)[quarter * 8 + tid] =

@@ -34,6 +34,8 @@
 // lanes of each quarter-warp gather eight different (round, group) slots, whatever the codes.
 #include <math.h>
 
+#include <type_traits>
+
 #include "attend.cuh"
 
 namespace commvq {
@@ -225,8 +227,7 @@ __global__ void fast_prep_kernel(AttendArgs a, int R) {
 // stores them in the score buffer and keeps their maxima.
 template <int R, int KV, typename QT, bool kCheck>
 __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __restrict__ q, unsigned char* smem,
-                                           int64_t row0, int64_t t_begin, int64_t t_end, Partial* part,
-                                           float* msplit) {
+                                           int64_t row0, int64_t t_begin, int64_t t_end, float* msplit) {
   constexpr int MK = KV / 2;                  // KV heads per warp
   constexpr int kFin = MK > 1 ? MK / 2 : 1;   // KV heads each warp of a pair finalises (KV = 2: half 0 only)
   constexpr int kRec = KV * R * 16;
@@ -241,7 +242,7 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
 
   const int Nc = kCheck ? a.n_codes : 256;
   const int G = a.q_heads / KV;
-  const int b = blockIdx.y, S = gridDim.x;
+  const int b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, i = lane & 3;
   const int rt = warp >> 2, hf = (warp >> 1) & 1, kg = warp & 1;
@@ -338,38 +339,30 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
 
   const float scale = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
   const int64_t n_tiles = (a.max_T + kFTile - 1) / kFTile;
+  // Score buffer of sequence b: [tile][Hq][16 slots] floats; tile position g sits in slot
+  // 4 (g / 2) + g % 2, position g + 8 two slots later. A thread finalises head columns 2i, 2i + 1
+  // (those below G) of rows g, g + 8: per finalised KV head f its slots start at fo[f].
+  const int tile_floats = a.q_heads * kFTile;
+  float* const sc_seq = a.scores + static_cast<int64_t>(b) * n_tiles * tile_floats;
+  const bool col0 = 2 * i < G, col1 = 2 * i + 1 < G;
   float mrun[kFin][2];
 #pragma unroll
   for (int f = 0; f < kFin; ++f) mrun[f][0] = mrun[f][1] = -INFINITY;
   int err = 0;
   const int fin0 = hf * kFin;            // first m this warp finalises (MK == 2 kFin, or KV = 2)
   const bool fins = (MK > 1) || hf == 0;  // KV = 2: only half 0 finalises
-
-  int stage = 0, it = 0;
-  for (int64_t t0 = t_begin; t0 < t_end; t0 += kFStage, stage ^= 1, ++it) {
-    cp_async_wait<0>();
-    __syncthreads();   // this stage's codes (and, the first time, the image) are in shared memory,
-                       // and every warp is done with the previous stage's buffer
-    if (t0 + kFStage < t_end) fast_issue_stage<kRec>(stages + (stage ^ 1) * kStageBytes, a.k_codes, row0, t0 + kFStage, t_end);
-    cp_async_commit();
-    if (it > 0) {
-      if (it % kFRefresh == 0) {
-        refresh(t0);
-      } else {
+  int fo[kFin];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 d = advt[(hf * 4 + i) * 4 + u];
-          const f32x2 dc = pack2(d.x, d.y), ds = pack2(d.z, d.w);
-#pragma unroll
-          for (int rr = 0; rr < 2; ++rr) cmul2(C[rr][u], Sn[rr][u], dc, ds);
-        }
-      }
-    }
+  for (int f = 0; f < kFin; ++f) fo[f] = ((kg + 2 * (fin0 + f)) * G + 2 * i) * kFTile + (g >> 1) * 4 + (g & 1);
 
+  // One stage; kFull: all its positions lie before t_end, so no row needs a check.
+  auto stage_body = [&](auto full_tag, int64_t t0, int stage) {
+    constexpr bool kFull = decltype(full_tag)::value;
     const int64_t tile_t0 = t0 + kFTile * rt;
-    const bool tile_live = tile_t0 < t_end;
-    const int rows_valid = tile_live ? static_cast<int>(min(static_cast<int64_t>(kFTile), t_end - tile_t0)) : 0;
-    const bool valid0 = g < rows_valid, valid1 = g + 8 < rows_valid;
+    const int rows_valid =
+        kFull ? kFTile : static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(kFTile), t_end - tile_t0)));
+    const bool tile_live = kFull || rows_valid > 0;
+    const bool valid0 = kFull || g < rows_valid, valid1 = kFull || g + 8 < rows_valid;
     const unsigned char* sb = stages + stage * kStageBytes;
     float* xb = xbuf + ((stage * kFStageTiles + rt) * KV) * 16 * 8;
     float fin[kFin][4];
@@ -386,7 +379,7 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
           cw[0][1] = ld8(sb, rowoff0 + cwoff2 + mo);
           cw[1][1] = ld8(sb, rowoff1 + cwoff2 + mo);
         }
-        if (kCheck) {   // rows past the end may hold stale bytes: read them as code 0
+        if (kCheck && !kFull) {   // rows past the end may hold stale bytes: read them as code 0
           if (!valid0) { cw[0][0] = make_uint2(0u, 0u); cw[0][1] = make_uint2(0u, 0u); }
           if (!valid1) { cw[1][0] = make_uint2(0u, 0u); cw[1][1] = make_uint2(0u, 0u); }
         }
@@ -432,25 +425,24 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
             mma_f16(acc, hx[0], hx[1], hy[0], hy[1], qb.x, qb.y);
           }
         }
-        const float* d = acc;
-        // d: (row g, col 2i), (row g, col 2i + 1), (row g + 8, col 2i), (row g + 8, col 2i + 1)
+        // acc: (row g, col 2i), (row g, col 2i + 1), (row g + 8, col 2i), (row g + 8, col 2i + 1);
         // the first kFin KV heads are finalised by the half-0 warp, the rest by the half-1 warp
         // (compile-time slots: no local memory)
         const bool mine = fins && ((m < kFin) == (hf == 0));
         if (mine) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) fin[m < kFin ? m : m - kFin][k] = d[k];
+          for (int k = 0; k < 4; ++k) fin[m < kFin ? m : m - kFin][k] = acc[k];
         } else {
           float* xr = xb + kv * 16 * 8;
-          *reinterpret_cast<float2*>(xr + g * 8 + 2 * i) = make_float2(d[0], d[1]);
-          *reinterpret_cast<float2*>(xr + (g + 8) * 8 + 2 * i) = make_float2(d[2], d[3]);
+          *reinterpret_cast<float2*>(xr + g * 8 + 2 * i) = make_float2(acc[0], acc[1]);
+          *reinterpret_cast<float2*>(xr + (g + 8) * 8 + 2 * i) = make_float2(acc[2], acc[3]);
         }
       }
     }
     // the two warps of a (tile, KV group) pair meet: named barrier 1 + (rt * 2 + kg)
     asm volatile("bar.sync %0, 64;\n" ::"r"(1 + rt * 2 + kg) : "memory");
     if (tile_live && fins) {
-      const int64_t tau = tile_t0 / kFTile;   // the tile's index within the sequence
+      float* dst = sc_seq + (tile_t0 >> 4) * tile_floats;
 #pragma unroll
       for (int f = 0; f < kFin; ++f) {
         const int kv = kg + 2 * (fin0 + f);
@@ -462,25 +454,48 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
         const float s01 = (hf == 0 ? fin[f][1] + p0.y : p0.y + fin[f][1]) * scale;
         const float s10 = (hf == 0 ? fin[f][2] + p1.x : p1.x + fin[f][2]) * scale;
         const float s11 = (hf == 0 ? fin[f][3] + p1.y : p1.y + fin[f][3]) * scale;
-        // score slots of positions g and g + 8 of the tile for head columns 2i, 2i + 1
-        const int slot0 = ((g & 7) >> 1) * 4 + (g & 1);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int col = 2 * i + c;
-          if (col >= G) continue;
-          float* dst = a.scores + ((static_cast<int64_t>(b) * n_tiles + tau) * a.q_heads + kv * G + col) * kFTile;
-          const float va = c ? s01 : s00, vb = c ? s11 : s10;
-          if (valid0) {
-            dst[slot0] = va;
-            mrun[f][c] = fmaxf(mrun[f][c], va);
-          }
-          if (valid1) {
-            dst[slot0 + 2] = vb;
-            mrun[f][c] = fmaxf(mrun[f][c], vb);
-          }
+        float* d = dst + fo[f];   // column 2i at d, column 2i + 1 one slot row later
+        // maxima over every column (past G: zero scores, never read back)
+        if (valid0) {
+          if (col0) d[0] = s00;
+          if (col1) d[kFTile] = s01;
+          mrun[f][0] = fmaxf(mrun[f][0], s00);
+          mrun[f][1] = fmaxf(mrun[f][1], s01);
+        }
+        if (valid1) {
+          if (col0) d[2] = s10;
+          if (col1) d[kFTile + 2] = s11;
+          mrun[f][0] = fmaxf(mrun[f][0], s10);
+          mrun[f][1] = fmaxf(mrun[f][1], s11);
         }
       }
     }
+  };
+
+  int stage = 0, it = 0;
+  for (int64_t t0 = t_begin; t0 < t_end; t0 += kFStage, stage ^= 1, ++it) {
+    cp_async_wait<0>();
+    __syncthreads();   // this stage's codes (and, the first time, the image) are in shared memory,
+                       // and every warp is done with the previous stage's buffer
+    if (t0 + kFStage < t_end) fast_issue_stage<kRec>(stages + (stage ^ 1) * kStageBytes, a.k_codes, row0, t0 + kFStage, t_end);
+    cp_async_commit();
+    if (it > 0) {
+      if (it % kFRefresh == 0) {
+        refresh(t0);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 d = advt[(hf * 4 + i) * 4 + u];
+          const f32x2 dc = pack2(d.x, d.y), ds = pack2(d.z, d.w);
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) cmul2(C[rr][u], Sn[rr][u], dc, ds);
+        }
+      }
+    }
+    if (t0 + kFStage <= t_end)
+      stage_body(std::true_type{}, t0, stage);
+    else
+      stage_body(std::false_type{}, t0, stage);
   }
   cp_async_wait<0>();
 
@@ -504,14 +519,12 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
     }
   }
   __syncthreads();
+  // [KV][8] (columns past G: the max of their zero scores)
   for (int e = tid; e < KV * 8; e += kFThreads) {
-    const int kv = e >> 3, col = e & 7;
-    if (col >= G) continue;
     float m = -INFINITY;
 #pragma unroll
     for (int r2 = 0; r2 < kFStageTiles; ++r2) m = fmaxf(m, mred[r2 * KV * 8 + e]);
-    part[static_cast<int64_t>(kv * G + col) * S].m = m;
-    msplit[kv * G + col] = m;
+    msplit[e] = m;
   }
   if (kCheck) {
     err = __syncthreads_or(err);
@@ -545,8 +558,9 @@ __device__ __forceinline__ void values_phase(const AttendArgs& a, unsigned char*
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, i = lane & 3;
   const int kv = warp / WPK, sub = warp % WPK;
-  const int score_stage_bytes = kTiles * a.q_heads * kFTile * 4;
   const int64_t n_tiles = (a.max_T + kFTile - 1) / kFTile;
+  const int tile_floats = a.q_heads * kFTile;                  // one tile of the score buffer
+  const int score_stage_bytes = kTiles * tile_floats * 4;
   auto issue_codes = [&](unsigned char* dst, int64_t t0) {
     constexpr int kPieces = kRec / 16;
     const int n = static_cast<int>(min(static_cast<int64_t>(kStageT), t_end - t0));
@@ -559,10 +573,9 @@ __device__ __forceinline__ void values_phase(const AttendArgs& a, unsigned char*
   auto issue_scores = [&](unsigned char* dst, int64_t t0) {   // whole tiles, contiguous
     const int64_t tau0 = t0 / kFTile;
     const int64_t tau1 = (min(t_end, t0 + kStageT) + kFTile - 1) / kFTile;
-    const int pieces = static_cast<int>((tau1 - tau0) * a.q_heads * 4);
-    const unsigned char* src =
-        reinterpret_cast<const unsigned char*>(a.scores + (static_cast<int64_t>(b) * n_tiles + tau0) * a.q_heads * kFTile);
-    for (int p = tid; p < pieces; p += kFThreads) cp_async16(dst + p * 16, src + p * 16);
+    const int pieces = static_cast<int>(tau1 - tau0) * (tile_floats / 4);
+    const float* src = a.scores + (static_cast<int64_t>(b) * n_tiles + tau0) * tile_floats;
+    for (int p = tid; p < pieces; p += kFThreads) cp_async16_ca(dst + p * 16, src + 4 * p);
   };
 
   {   // the value image replaces the key image (the keys phase is done with it)
@@ -575,10 +588,14 @@ __device__ __forceinline__ void values_phase(const AttendArgs& a, unsigned char*
     }
   }
   issue_codes(stages, t_begin);
-  issue_scores(sstage, t_begin);   // written by this CTA's keys phase (fenced before the barrier)
+  issue_scores(sstage, t_begin);   // written by this CTA's keys phase before the barrier
   cp_async_commit();
 
-  const float m_h = (g < G) ? msplit[kv * G + g] : 0.0f;
+  // head column g of this warp's KV head; a column past G reads column G - 1 (finite weights in an
+  // mma column that is never written out)
+  const int gc = min(g, G - 1);
+  const float m_h = msplit[kv * 8 + gc];
+  const int sc_off = (kv * G + gc) * kFTile + 4 * i;   // the thread's 4 slots in a score tile
   float O[8][4];
 #pragma unroll
   for (int m = 0; m < 8; ++m) O[m][0] = O[m][1] = O[m][2] = O[m][3] = 0.0f;
@@ -601,6 +618,52 @@ __device__ __forceinline__ void values_phase(const AttendArgs& a, unsigned char*
   const uint32_t cwo1 = static_cast<uint32_t>(2 * i * kRowStride + (kv * R + (rfirst ^ 1)) * 16 + (g >> 1) * 4);
   constexpr int kTauOff[4] = {0, 1, 8, 9};
 
+  // One 16-position tile; kFull: all 16 positions lie before t_end (rem is then 16).
+  auto tile_body = [&](auto full_tag, int tile, const unsigned char* sb, const float* ssc, int rem) {
+    constexpr bool kFull = decltype(full_tag)::value;
+    const float4 sv = *reinterpret_cast<const float4*>(ssc + tile * tile_floats + sc_off);
+    float p[4] = {ex2(sv.x - m_h), ex2(sv.y - m_h), ex2(sv.z - m_h), ex2(sv.w - m_h)};
+    if (!kFull) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (2 * i + kTauOff[k] >= rem) p[k] = 0.0f;   // past the end: stale slots
+    }
+    lsum += (p[0] + p[1]) + (p[2] + p[3]);
+    const uint32_t b0 = h2u(__floats2half2_rn(p[0], p[1]));
+    const uint32_t b1 = h2u(__floats2half2_rn(p[2], p[3]));
+    const uint32_t tb = static_cast<uint32_t>(tile * kFTile * kRowStride);
+    uint4 E[4][2];   // [position k][group 2g, 2g + 1]
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t w0 = ld4(sb, tb + cwo0 + kTauOff[k] * kRowStride);
+      uint32_t w1 = (R == 2) ? ld4(sb, tb + cwo1 + kTauOff[k] * kRowStride) : 0u;
+      if (kCheck && !kFull && 2 * i + kTauOff[k] >= rem) w0 = w1 = 0u;   // stale bytes read as code 0
+      uint4 sA, sB;
+      // gathers n = 0, 1 use the first round's word, n = 2, 3 the second's
+      const uint32_t a0 = kCheck ? img_addr_checked(w0, (2 * g + (i & 1)) & 3, vc[0], Nc, err) : img_addr(w0, vc[0], vs0);
+      const uint32_t a1 = kCheck ? img_addr_checked(w0, (2 * g + ((i ^ 1) & 1)) & 3, vc[1], Nc, err) : img_addr(w0, vc[1], vs1);
+      sA = ld16(smem, a0);
+      sB = ld16(smem, a1);
+      if (R == 2) {
+        const uint32_t a2 = kCheck ? img_addr_checked(w1, (2 * g + (i & 1)) & 3, vc[2], Nc, err) : img_addr(w1, vc[2], vs0);
+        const uint32_t a3 = kCheck ? img_addr_checked(w1, (2 * g + ((i ^ 1) & 1)) & 3, vc[3], Nc, err) : img_addr(w1, vc[3], vs1);
+        sA = hadd4(sA, ld16(smem, a2));
+        sB = hadd4(sB, ld16(smem, a3));
+      }
+      E[k][0] = odd ? sB : sA;
+      E[k][1] = odd ? sA : sB;
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const uint32_t sl = (m & 1) ? 0x7632u : 0x5410u;
+      const uint32_t A0 = __byte_perm(word_of(E[0][0], m >> 1), word_of(E[1][0], m >> 1), sl);
+      const uint32_t A1 = __byte_perm(word_of(E[0][1], m >> 1), word_of(E[1][1], m >> 1), sl);
+      const uint32_t A2 = __byte_perm(word_of(E[2][0], m >> 1), word_of(E[3][0], m >> 1), sl);
+      const uint32_t A3 = __byte_perm(word_of(E[2][1], m >> 1), word_of(E[3][1], m >> 1), sl);
+      mma_f16(O[m], A0, A1, A2, A3, b0, b1);
+    }
+  };
+
   int stage = 0;
   for (int64_t t0 = t_begin; t0 < t_end; t0 += kStageT, stage ^= 1) {
     cp_async_wait<0>();
@@ -612,97 +675,67 @@ __device__ __forceinline__ void values_phase(const AttendArgs& a, unsigned char*
     cp_async_commit();
     const unsigned char* sb = stages + stage * kStageBytes;
     const float* ssc = reinterpret_cast<const float*>(sstage + stage * score_stage_bytes);
-
-    for (int tile = sub; tile < kTiles; tile += WPK) {
-      const int64_t tt0 = t0 + tile * kFTile;
-      if (tt0 >= t_end) break;
-      const int rem = static_cast<int>(min(static_cast<int64_t>(kFTile), t_end - tt0));
-      const int tau[4] = {2 * i, 2 * i + 1, 2 * i + 8, 2 * i + 9};
-      float p[4] = {0.f, 0.f, 0.f, 0.f};
-      if (g < G) {
-        const float4 sv = *reinterpret_cast<const float4*>(ssc + ((tile * a.q_heads + kv * G + g) * kFTile) + 4 * i);
-        const float sk[4] = {sv.x, sv.y, sv.z, sv.w};
+    if (t0 + kStageT <= t_end) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (tau[k] < rem) p[k] = ex2(sk[k] - m_h);
-          lsum += p[k];
-        }
-      }
-      const uint32_t b0 = h2u(__floats2half2_rn(p[0], p[1]));
-      const uint32_t b1 = h2u(__floats2half2_rn(p[2], p[3]));
-      const uint32_t tb = static_cast<uint32_t>(tile * kFTile * kRowStride);
-      uint4 E[4][2];   // [position k][group 2g, 2g + 1]
+      for (int ti = 0; ti < kTiles / WPK; ++ti) tile_body(std::true_type{}, sub + ti * WPK, sb, ssc, kFTile);
+    } else {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint32_t w0 = ld4(sb, tb + cwo0 + kTauOff[k] * kRowStride);
-        uint32_t w1 = (R == 2) ? ld4(sb, tb + cwo1 + kTauOff[k] * kRowStride) : 0u;
-        if (kCheck && tau[k] >= rem) w0 = w1 = 0u;   // stale bytes past the end read as code 0
-        uint4 sA, sB;
-        // gathers n = 0, 1 use the first round's word, n = 2, 3 the second's
-        const uint32_t a0 = kCheck ? img_addr_checked(w0, (2 * g + (i & 1)) & 3, vc[0], Nc, err) : img_addr(w0, vc[0], vs0);
-        const uint32_t a1 = kCheck ? img_addr_checked(w0, (2 * g + ((i ^ 1) & 1)) & 3, vc[1], Nc, err) : img_addr(w0, vc[1], vs1);
-        sA = ld16(smem, a0);
-        sB = ld16(smem, a1);
-        if (R == 2) {
-          const uint32_t a2 = kCheck ? img_addr_checked(w1, (2 * g + (i & 1)) & 3, vc[2], Nc, err) : img_addr(w1, vc[2], vs0);
-          const uint32_t a3 = kCheck ? img_addr_checked(w1, (2 * g + ((i ^ 1) & 1)) & 3, vc[3], Nc, err) : img_addr(w1, vc[3], vs1);
-          sA = hadd4(sA, ld16(smem, a2));
-          sB = hadd4(sB, ld16(smem, a3));
-        }
-        E[k][0] = odd ? sB : sA;
-        E[k][1] = odd ? sA : sB;
-      }
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const uint32_t sl = (m & 1) ? 0x7632u : 0x5410u;
-        const uint32_t A0 = __byte_perm(word_of(E[0][0], m >> 1), word_of(E[1][0], m >> 1), sl);
-        const uint32_t A1 = __byte_perm(word_of(E[0][1], m >> 1), word_of(E[1][1], m >> 1), sl);
-        const uint32_t A2 = __byte_perm(word_of(E[2][0], m >> 1), word_of(E[3][0], m >> 1), sl);
-        const uint32_t A3 = __byte_perm(word_of(E[2][1], m >> 1), word_of(E[3][1], m >> 1), sl);
-        mma_f16(O[m], A0, A1, A2, A3, b0, b1);
+      for (int ti = 0; ti < kTiles / WPK; ++ti) {
+        const int tile = sub + ti * WPK;
+        const int64_t tt0 = t0 + tile * kFTile;
+        if (tt0 >= t_end) break;
+        tile_body(std::false_type{}, tile, sb, ssc, static_cast<int>(min(static_cast<int64_t>(kFTile), t_end - tt0)));
       }
     }
   }
   cp_async_wait<0>();
-  __syncthreads();   // the code stages are reused below
+  __syncthreads();   // every warp is done with the image: its space holds the warps' sums below
 
   // l: sum over the quad (lanes with equal g hold the same head column)
   lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
   lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-  // warps of one KV head add their accumulators in a fixed order through shared memory
-  float* xred = reinterpret_cast<float*>(stages);   // [16 warps][32 lanes][33]
-  if (WPK > 1) {
-    float* mine = xred + (warp * 32 + lane) * 33;
+  // Each warp's O^T (8 head columns x 128 dims) goes to shared memory, [warp][col][dim'] with
+  // dim' = dim + 4 (dim / 16) and a column stride of 164 floats (16-byte stores of a quarter-warp
+  // hit distinct banks); then the warps of a KV head are added in a fixed order and the split's
+  // partials are written with coalesced 16-byte stores.
+  constexpr int kColStride = 164, kWarpStride = 8 * kColStride;
+  float* obuf = reinterpret_cast<float*>(smem);
+  float* lbuf = obuf + kFWarps * kWarpStride;   // [warp][8]
+  {
+    float* mine = obuf + warp * kWarpStride + 20 * g;
 #pragma unroll
-    for (int m = 0; m < 8; ++m)
+    for (int c = 0; c < 2; ++c)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) mine[m * 4 + c] = O[m][c];
-    mine[32] = lsum;
-    __syncthreads();
-    if (sub == 0) {
-      for (int w = 1; w < WPK; ++w) {
-        const float* other = xred + ((warp + w) * 32 + lane) * 33;
+      for (int h8 = 0; h8 < 2; ++h8)
 #pragma unroll
-        for (int m = 0; m < 8; ++m)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) O[m][c] += other[m * 4 + c];
-        lsum += other[32];
-      }
-    }
+        for (int q4 = 0; q4 < 2; ++q4)
+          *reinterpret_cast<float4*>(mine + (2 * i + c) * kColStride + 8 * h8 + 4 * q4) =
+              make_float4(O[4 * q4][2 * h8 + c], O[4 * q4 + 1][2 * h8 + c], O[4 * q4 + 2][2 * h8 + c],
+                          O[4 * q4 + 3][2 * h8 + c]);
+    if (i == 0) lbuf[warp * 8 + g] = lsum;
   }
-  if (sub == 0) {
+  __syncthreads();
+  for (int e = tid; e < a.q_heads * (kD / 4); e += kFThreads) {
+    const int h = e >> 5, d4 = e & 31;   // head kv * G + col, dims 4 d4 .. 4 d4 + 3
+    const int hk = h / G, col = h - hk * G;
+    const float* src = obuf + (hk * WPK) * kWarpStride + col * kColStride + 20 * (d4 >> 2) + 4 * (d4 & 3);
+    float4 acc = *reinterpret_cast<const float4*>(src);
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int col = 2 * i + c;
-      if (col >= G) continue;
-      Partial* ph = part + static_cast<int64_t>(kv * G + col) * S;
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        ph->o[16 * g + m] = O[m][c];
-        ph->o[16 * g + 8 + m] = O[m][2 + c];
-      }
+    for (int w = 1; w < WPK; ++w) {
+      const float4 o = *reinterpret_cast<const float4*>(src + w * kWarpStride);
+      acc.x += o.x;
+      acc.y += o.y;
+      acc.z += o.z;
+      acc.w += o.w;
     }
-    if (i == 0 && g < G) part[static_cast<int64_t>(kv * G + g) * S].l = lsum;
+    reinterpret_cast<float4*>(part[static_cast<int64_t>(h) * S].o)[d4] = acc;
+  }
+  for (int h = tid; h < a.q_heads; h += kFThreads) {
+    const int hk = h / G, col = h - hk * G;
+    float l = lbuf[(hk * WPK) * 8 + col];
+#pragma unroll
+    for (int w = 1; w < WPK; ++w) l += lbuf[(hk * WPK + w) * 8 + col];
+    *reinterpret_cast<float2*>(&part[static_cast<int64_t>(h) * S].m) = make_float2(msplit[hk * 8 + col], l);
   }
   if (kCheck) {
     err = __syncthreads_or(err);
@@ -738,8 +771,9 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_attend_kernel(AttendArgs a,
     }
     return;
   }
-  keys_phase<R, KV, QT, kCheck>(a, q, smem, row0, t_begin, t_end, part, msplit);
-  __threadfence();   // the score buffer rows written above are read back by asynchronous copies
+  keys_phase<R, KV, QT, kCheck>(a, q, smem, row0, t_begin, t_end, msplit);
+  // the score buffer rows written above are read back by this CTA's own (L1) copies: the
+  // barrier makes them visible
   __syncthreads();
   values_phase<R, KV, kCheck>(a, smem, row0, t_begin, t_end, part, msplit);
 }
@@ -806,9 +840,9 @@ size_t fast_values_smem_bytes(int R, int KV, int q_heads) {
   const int wpk = kFWarps / KV;
   const int tiles = wpk > kFStageTiles ? wpk : kFStageTiles;
   const size_t row = static_cast<size_t>(KV) * R * 16 + 16;
-  size_t stages = static_cast<size_t>(2) * kFTile * tiles * row;
-  const size_t xred = static_cast<size_t>(kFWarps) * 32 * 33 * 4;
-  if (stages < xred) stages = xred;   // the per-warp sums reuse the code stages after the loop
+  const size_t stages = static_cast<size_t>(2) * kFTile * tiles * row;
+  // the warps' sums after the loop (16 x 8 x 164 floats + 16 x 8) reuse the image's space
+  static_assert(kFWarps * 8 * 164 * 4 + kFWarps * 8 * 4 <= kFImg, "epilogue buffer exceeds the image");
   return kFImg + stages + static_cast<size_t>(2) * tiles * q_heads * kFTile * 4;
 }
 

@@ -208,6 +208,12 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
   const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem_src) : "memory");
 }
+// The same copy through L1 (.ca): used for data this CTA wrote to global memory before a
+// barrier, which the barrier makes visible to the CTA's own reads.
+__device__ __forceinline__ void cp_async16_ca(void* smem_dst, const void* gmem_src) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem_src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
@@ -250,6 +256,51 @@ __device__ __forceinline__ void cmul2(f32x2& c, f32x2& s, f32x2 cc, f32x2 ss) {
 __device__ __forceinline__ void load_phasor(float4 v, f32x2& c, f32x2& s) {
   c = pack2(v.x, v.y);
   s = pack2(v.z, v.w);
+}
+
+// Nearest-entry update with a distance already computed by the encoder's fp32 rule (the
+// comparison half of nearest_step).
+template <bool kTrack>
+__device__ __forceinline__ void nearest_take(Nearest& n, float dist, int c) {
+  if (dist < n.best) {
+    if (kTrack) n.second = n.best;
+    n.best = dist;
+    n.idx = c;
+  } else if (kTrack && dist < n.second) {
+    n.second = dist;
+  }
+}
+
+// g = 8 sub-codebook tile for the packed scan: entries 2p and 2p + 1 side by side, so that one
+// packed fp32x2 instruction takes the same step of both distances. Pair p occupies float4s
+// 4p .. 4p + 3; float4 kk holds (e_2p[2kk], e_2p+1[2kk], e_2p[2kk+1], e_2p+1[2kk+1]). An odd last
+// entry is paired with itself (its second lane is never compared). src: n entries of 8 floats.
+__device__ __forceinline__ void stage_pairs8(float4* tile, const float* src, int n) {
+  const int pairs = (n + 1) >> 1;
+  for (int e = threadIdx.x; e < pairs * 4; e += blockDim.x) {
+    const int p = e >> 2, kk = e & 3;
+    const int c1 = min(2 * p + 1, n - 1);
+    const float2 lo = __ldg(reinterpret_cast<const float2*>(src + static_cast<int64_t>(2 * p) * kG) + kk);
+    const float2 hi = __ldg(reinterpret_cast<const float2*>(src + static_cast<int64_t>(c1) * kG) + kk);
+    tile[e] = make_float4(lo.x, hi.x, lo.y, hi.y);
+  }
+}
+
+// Distances of one row to entries 2p and 2p + 1 of a pair tile; res2[k] holds the row's residual
+// k in both lanes. Each lane follows the encoder's fp32 rule exactly (k = 0..7 in order: subtract,
+// then a fused multiply-add onto the running sum from +0), so the distances -- and the codes they
+// decide -- are bit-identical to the scalar scan.
+__device__ __forceinline__ f32x2 pair_dist8(const f32x2 (&res2)[kG], const float4* pair) {
+  f32x2 acc = 0ull;   // +0.0f in both lanes
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    const float4 v = pair[kk];
+    f32x2 t = sub2(res2[2 * kk], pack2(v.x, v.y));
+    acc = fma2(t, t, acc);
+    t = sub2(res2[2 * kk + 1], pack2(v.z, v.w));
+    acc = fma2(t, t, acc);
+  }
+  return acc;
 }
 
 // Phasor e^{i phi} of RoPE pair p into a packed row: float4 p/2 holds (cos p, cos p+1, sin p,

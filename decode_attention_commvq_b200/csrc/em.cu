@@ -84,16 +84,50 @@ em_assign_kernel(const float* __restrict__ rows, int64_t N, int d, int Nc,
         for (int k = 0; k < kG; ++k) res[i][q * kG + k] = v[k];
       }
     }
-    for (int c0 = 0; c0 < Nc; c0 += kTileE) {
-      const int n = min(kTileE, Nc - c0);
-      __syncthreads();
-      for (int e = threadIdx.x; e < n * (GG / 4); e += kThreads)
-        tile[e] = __ldg(reinterpret_cast<const float4*>(sub_cb + static_cast<int64_t>(c0) * GG) + e);
-      __syncthreads();
-#pragma unroll 2
-      for (int c = 0; c < n; ++c) {
+    if constexpr (GG == kG) {
+      // packed scan (the encoder's): two entries per fp32x2 instruction, each lane the scalar rule
+      f32x2 res2[kRows][kG];
 #pragma unroll
-        for (int i = 0; i < kRows; ++i) nearest_step_g<GG, false>(best[i], res[i], tile + c * (GG / 4), c0 + c);
+      for (int i = 0; i < kRows; ++i)
+#pragma unroll
+        for (int k = 0; k < kG; ++k) res2[i][k] = pack2(res[i][k], res[i][k]);
+      for (int c0 = 0; c0 < Nc; c0 += kTileE) {
+        const int n = min(kTileE, Nc - c0);
+        __syncthreads();
+        stage_pairs8(tile, sub_cb + static_cast<int64_t>(c0) * GG, n);
+        __syncthreads();
+        const int pairs = n >> 1;
+#pragma unroll 2
+        for (int p = 0; p < pairs; ++p) {
+#pragma unroll
+          for (int i = 0; i < kRows; ++i) {
+            float d0, d1;
+            unpack2(pair_dist8(res2[i], tile + 4 * p), d0, d1);
+            nearest_take<false>(best[i], d0, c0 + 2 * p);
+            nearest_take<false>(best[i], d1, c0 + 2 * p + 1);
+          }
+        }
+        if (n & 1) {
+#pragma unroll
+          for (int i = 0; i < kRows; ++i) {
+            float d0, d1;
+            unpack2(pair_dist8(res2[i], tile + 4 * pairs), d0, d1);
+            nearest_take<false>(best[i], d0, c0 + n - 1);
+          }
+        }
+      }
+    } else {
+      for (int c0 = 0; c0 < Nc; c0 += kTileE) {
+        const int n = min(kTileE, Nc - c0);
+        __syncthreads();
+        for (int e = threadIdx.x; e < n * (GG / 4); e += kThreads)
+          tile[e] = __ldg(reinterpret_cast<const float4*>(sub_cb + static_cast<int64_t>(c0) * GG) + e);
+        __syncthreads();
+#pragma unroll 2
+        for (int c = 0; c < n; ++c) {
+#pragma unroll
+          for (int i = 0; i < kRows; ++i) nearest_step_g<GG, false>(best[i], res[i], tile + c * (GG / 4), c0 + c);
+        }
       }
     }
 #pragma unroll

@@ -9,7 +9,8 @@
 // Grid: x = blocks of kThreads rows (2 kThreads for g = 8), y = group j. The block stages a
 // tile of its group's sub-codebook in shared memory; every thread reads the same entry at the
 // same time (a broadcast), so the scan issues g/4 shared loads per entry for 1 (g = 8: 2)
-// rows of arithmetic. g = 8 is the library's attention layout; 16, 32 and 64 cover the
+// rows of arithmetic. For g = 8 the tile holds entries in pairs and the scan runs on sm_100's
+// packed fp32x2 instructions, two entries per instruction with each lane the scalar rule. g = 8 is the library's attention layout; 16, 32 and 64 cover the
 // pages' own setting (g = 64, Nc' = 64, R = 21 or 11).
 #include "common.cuh"
 
@@ -75,16 +76,50 @@ encode_kernel(EncodeJobs<XT> jobs, int64_t n_rows, int d, int R, int n_codes, in
 #pragma unroll
     for (int i = 0; i < kRows; ++i) nearest_init(best[i]);
 
-    for (int c0 = 0; c0 < n_codes; c0 += kTile) {
-      const int n = min(kTile, n_codes - c0);
-      __syncthreads();
-      for (int e = threadIdx.x; e < n * (GG / 4); e += kThreads)
-        tile[e] = __ldg(reinterpret_cast<const float4*>(sub + static_cast<int64_t>(c0) * GG) + e);
-      __syncthreads();
-#pragma unroll 2
-      for (int c = 0; c < n; ++c) {
+    if constexpr (GG == kG) {
+      // packed scan: two entries per fp32x2 instruction, each lane the scalar rule
+      f32x2 res2[kRows][kG];
 #pragma unroll
-        for (int i = 0; i < kRows; ++i) nearest_step_g<GG, kTrack>(best[i], res[i], tile + c * (GG / 4), c0 + c);
+      for (int i = 0; i < kRows; ++i)
+#pragma unroll
+        for (int k = 0; k < kG; ++k) res2[i][k] = pack2(res[i][k], res[i][k]);
+      for (int c0 = 0; c0 < n_codes; c0 += kTile) {
+        const int n = min(kTile, n_codes - c0);
+        __syncthreads();
+        stage_pairs8(tile, sub + static_cast<int64_t>(c0) * GG, n);
+        __syncthreads();
+        const int pairs = n >> 1;
+#pragma unroll 2
+        for (int p = 0; p < pairs; ++p) {
+#pragma unroll
+          for (int i = 0; i < kRows; ++i) {
+            float d0, d1;
+            unpack2(pair_dist8(res2[i], tile + 4 * p), d0, d1);
+            nearest_take<kTrack>(best[i], d0, c0 + 2 * p);
+            nearest_take<kTrack>(best[i], d1, c0 + 2 * p + 1);
+          }
+        }
+        if (n & 1) {
+#pragma unroll
+          for (int i = 0; i < kRows; ++i) {
+            float d0, d1;
+            unpack2(pair_dist8(res2[i], tile + 4 * pairs), d0, d1);
+            nearest_take<kTrack>(best[i], d0, c0 + n - 1);
+          }
+        }
+      }
+    } else {
+      for (int c0 = 0; c0 < n_codes; c0 += kTile) {
+        const int n = min(kTile, n_codes - c0);
+        __syncthreads();
+        for (int e = threadIdx.x; e < n * (GG / 4); e += kThreads)
+          tile[e] = __ldg(reinterpret_cast<const float4*>(sub + static_cast<int64_t>(c0) * GG) + e);
+        __syncthreads();
+#pragma unroll 2
+        for (int c = 0; c < n; ++c) {
+#pragma unroll
+          for (int i = 0; i < kRows; ++i) nearest_step_g<GG, kTrack>(best[i], res[i], tile + c * (GG / 4), c0 + c);
+        }
       }
     }
 

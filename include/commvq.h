@@ -383,6 +383,17 @@ commvq_status commvq_dense_decode(const commvq_config* cfg, const void* q, commv
  * clamped). Returns COMMVQ_ERR_DEVICE_CHECK when the word is non-zero. */
 commvq_status commvq_workspace_error(const void* workspace, int32_t* device_error, void* stream);
 
+/* Copies `bytes` bytes from src to dst with one kernel on `stream` (asynchronous, like
+ * cudaMemcpyAsync). Either pointer may be device memory or mapped pinned host memory (memory
+ * from cudaHostAlloc / cudaMallocHost, whose host address the device can use under unified
+ * addressing): the kernel's loads or stores then cross the host link. Meant for the few-KB
+ * per-step transfers of a decode loop (the query and the new position's K/V rows in, the output
+ * out), where a copy-engine transfer inside a CUDA graph costs more in scheduling than the bytes.
+ * Both pointers 16-byte aligned, ranges not overlapping (else COMMVQ_ERR_INVALID_ARG); bytes = 0
+ * is a no-op. The caller owns both buffers. Not part of the method: plumbing for the end-to-end
+ * step of a decode loop. */
+commvq_status commvq_copy_async(void* dst, const void* src, size_t bytes, void* stream);
+
 /* Static description of a status code. */
 const char* commvq_status_string(commvq_status status);
 

@@ -256,3 +256,14 @@ def test_binary_value_code_workspace_holds_the_key_side_and_the_sums(api):
     for n_bits in (1024, 2048, 8192):
         assert api.attend_binv_workspace_bytes(cfg, n_bits, 1, 32768) >= base + 32 * n_bits * 4
     assert api.attend_binv_workspace_bytes(cfg, 2048, -1, 10) == 0
+
+
+def test_copy_rejects_bad_arguments(api):
+    f = api.LIB.commvq_copy_async
+    P = ctypes.c_void_p
+    assert f(P(FAKE), P(FAKE + 4096), 0, None) == 0            # nothing to copy
+    assert f(None, P(FAKE), 64, None) == 1                     # null destination
+    assert f(P(FAKE), None, 64, None) == 1                     # null source
+    assert f(P(FAKE + 8), P(FAKE + 4096), 64, None) == 1       # misaligned destination
+    assert f(P(FAKE), P(FAKE + 4104), 64, None) == 1           # misaligned source
+    assert f(P(FAKE), P(FAKE + 32), 64, None) == 1             # overlapping ranges
