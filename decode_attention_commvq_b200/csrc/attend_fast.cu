@@ -50,6 +50,7 @@ constexpr int kFImgHalf = 65536;
 constexpr int kFImg = 2 * kFImgHalf;
 constexpr int kFRefresh = 16;               // stages between exact phasor refreshes
 constexpr int kFPhaseRows = kFStage;        // rows of the offset phasor table
+constexpr uint32_t kImgWaitPolls = 1u << 20;   // bound on the image copies' mbarrier wait
 
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
@@ -216,6 +217,26 @@ __global__ void fast_prep_kernel(AttendArgs a, int R) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// The codebook image (the Nc' used rows of each 64 KB half) into shared memory by two bulk copies
+// of the tensor memory accelerator, completing on `bar` (issued by thread 0). Then every thread
+// waits for the phase of `parity`; a wait that runs out sets the wait bit of the error word and
+// waits once more (bounded), so that no copy is left in flight when the CTA goes on.
+__device__ __forceinline__ void image_copy_issue(unsigned char* smem, const uint4* img, int Nc, uint64_t* bar) {
+  if (threadIdx.x == 0) {
+    const uint32_t half = static_cast<uint32_t>(Nc) * 256u;
+    mbar_arrive_expect_tx(bar, 2 * half);
+    bulk_copy_g2s(smem, img, half, bar);
+    bulk_copy_g2s(smem + kFImgHalf, reinterpret_cast<const unsigned char*>(img) + kFImgHalf, half, bar);
+  }
+}
+__device__ __forceinline__ void image_copy_wait(const AttendArgs& a, uint64_t* bar, uint32_t parity) {
+  if (!mbar_wait_bounded(bar, parity, kImgWaitPolls)) {
+    atomicOr(running_error(a.error_word), kErrWaitLimit);
+    mbar_wait_bounded(bar, parity, kImgWaitPolls);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // Keys. Warp w: row tile rt = w / 4 of each 64-position stage, half hf = (w / 2) % 2 of the head
 // dimension (groups 8 hf .. 8 hf + 7), KV heads kg + 2m (kg = w % 2, m < KV / 2). Thread (g, i):
 // rows g and g + 8 of the tile; local groups i and i + 4 of its half. mma k-step u (0..3) covers
@@ -227,7 +248,8 @@ __global__ void fast_prep_kernel(AttendArgs a, int R) {
 // stores them in the score buffer and keeps their maxima.
 template <int R, int KV, typename QT, bool kCheck>
 __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __restrict__ q, unsigned char* smem,
-                                           int64_t row0, int64_t t_begin, int64_t t_end, float* msplit) {
+                                           int64_t row0, int64_t t_begin, int64_t t_end, float* msplit,
+                                           uint64_t* ibar) {
   constexpr int MK = KV / 2;                  // KV heads per warp
   constexpr int kFin = MK > 1 ? MK / 2 : 1;   // KV heads each warp of a pair finalises (KV = 2: half 0 only)
   constexpr int kRec = KV * R * 16;
@@ -249,16 +271,12 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
 
   // Prepared state (codebook image, advance phasors) and the queries are not written by the
   // kernel this one may follow as a programmatic dependent: copy and form them before the wait.
-  {
-    const uint4* src = a.k_img;
-    uint4* dst = reinterpret_cast<uint4*>(smem);
-    const int n16 = (kFImgHalf / 16);
-    for (int p = tid; p < 2 * n16; p += kFThreads) {
-      const int hh = p / n16, off = p - hh * n16;
-      if (off < Nc * 16) cp_async16(dst + p, src + p);   // codes >= Nc' are never read
-    }
+  if (tid == 0) {
+    mbar_init(ibar, 1);
+    fence_mbar_init();
   }
-  cp_async_commit();
+  __syncthreads();
+  image_copy_issue(smem, a.k_img, Nc, ibar);   // rows of codes >= Nc' are never read
   // query fragments: entry (kv, hf2, u, ln) = (x of pair A, x of pair B), (y of A, y of B) of head
   // column ln / 4 (zero past G) in the key operand type
   for (int e = tid; e < KV * 2 * 4 * 32; e += kFThreads) {
@@ -336,6 +354,7 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
     __syncwarp();
   };
   refresh(t_begin);
+  image_copy_wait(a, ibar, 0);
 
   const float scale = 1.4426950408889634f / sqrtf(static_cast<float>(kD));
   const int64_t n_tiles = (a.max_T + kFTile - 1) / kFTile;
@@ -542,7 +561,7 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
 // slots; lanes with odd i swap the two group sums back.
 template <int R, int KV, bool kCheck>
 __device__ __forceinline__ void values_phase(const AttendArgs& a, unsigned char* smem, int64_t row0, int64_t t_begin,
-                                             int64_t t_end, Partial* part, const float* msplit) {
+                                             int64_t t_end, Partial* part, const float* msplit, uint64_t* ibar) {
   constexpr int WPK = kFWarps / KV;
   constexpr int kTiles = WPK > kFStageTiles ? WPK : kFStageTiles;
   constexpr int kStageT = kFTile * kTiles;
@@ -578,15 +597,10 @@ __device__ __forceinline__ void values_phase(const AttendArgs& a, unsigned char*
     for (int p = tid; p < pieces; p += kFThreads) cp_async16_ca(dst + p * 16, src + 4 * p);
   };
 
-  {   // the value image replaces the key image (the keys phase is done with it)
-    const uint4* src = a.v_img;
-    uint4* dst = reinterpret_cast<uint4*>(smem);
-    const int n16 = (kFImgHalf / 16);
-    for (int p = tid; p < 2 * n16; p += kFThreads) {
-      const int hh = p / n16, off = p - hh * n16;
-      if (off < Nc * 16) cp_async16(dst + p, src + p);
-    }
-  }
+  // the value image replaces the key image: every read of it is before the caller's barrier, and
+  // the proxy fence orders those reads before the bulk copies' writes
+  if (tid == 0) fence_async_smem();
+  image_copy_issue(smem, a.v_img, Nc, ibar);
   issue_codes(stages, t_begin);
   issue_scores(sstage, t_begin);   // written by this CTA's keys phase before the barrier
   cp_async_commit();
@@ -664,6 +678,7 @@ __device__ __forceinline__ void values_phase(const AttendArgs& a, unsigned char*
     }
   };
 
+  image_copy_wait(a, ibar, 1);
   int stage = 0;
   for (int64_t t0 = t_begin; t0 < t_end; t0 += kStageT, stage ^= 1) {
     cp_async_wait<0>();
@@ -751,7 +766,8 @@ template <int R, int KV, typename QT, bool kCheck>
 __global__ void __launch_bounds__(kFThreads, 1) fast_attend_kernel(AttendArgs a, const QT* __restrict__ q,
                                                                     int msplit_off) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  float* msplit = reinterpret_cast<float*>(smem + msplit_off);
+  float* msplit = reinterpret_cast<float*>(smem + msplit_off);            // [KV][8]
+  uint64_t* ibar = reinterpret_cast<uint64_t*>(smem + msplit_off + 64 * sizeof(float));   // image copies
   const int s = blockIdx.x, b = blockIdx.y, S = gridDim.x;
   int64_t row0, t_begin, t_end;
   fast_split(a, b, s, S, row0, t_begin, t_end);
@@ -771,18 +787,18 @@ __global__ void __launch_bounds__(kFThreads, 1) fast_attend_kernel(AttendArgs a,
     }
     return;
   }
-  keys_phase<R, KV, QT, kCheck>(a, q, smem, row0, t_begin, t_end, msplit);
+  keys_phase<R, KV, QT, kCheck>(a, q, smem, row0, t_begin, t_end, msplit, ibar);
   // the score buffer rows written above are read back by this CTA's own (L1) copies: the
   // barrier makes them visible
   __syncthreads();
-  values_phase<R, KV, kCheck>(a, smem, row0, t_begin, t_end, part, msplit);
+  values_phase<R, KV, kCheck>(a, smem, row0, t_begin, t_end, part, msplit, ibar);
 }
 
 template <int R, int KV, bool kCheck>
 commvq_status launch_fast_rkc(const AttendArgs& a, const void* q, commvq_dtype qt, int S, cudaStream_t st,
                               bool dependent) {
   const size_t smem = fast_smem_bytes(R, KV, a.q_heads);
-  const size_t smem_main = smem - 64 * sizeof(float);   // the split maxima sit past both phases' buffers
+  const size_t smem_main = smem - 64 * sizeof(float) - 16;   // split maxima and mbarrier past both phases' buffers
   dim3 grid(S, a.B);
   if (a.main_start && record_event(a.main_start, st) != cudaSuccess) return COMMVQ_ERR_CUDA;
 #define COMMVQ_FAST(QT)                                                                               \
@@ -848,7 +864,7 @@ size_t fast_values_smem_bytes(int R, int KV, int q_heads) {
 
 size_t fast_smem_bytes(int R, int KV, int q_heads) {
   const size_t k = fast_keys_smem_bytes(R, KV), v = fast_values_smem_bytes(R, KV, q_heads);
-  return (k > v ? k : v) + 64 * sizeof(float);
+  return (k > v ? k : v) + 64 * sizeof(float) + 16;
 }
 
 bool fast_supported(int g, int R, int q_heads, int kv_heads, int n_codes) {
