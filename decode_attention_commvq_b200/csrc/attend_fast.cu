@@ -257,8 +257,10 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
   constexpr int kStageBytes = kFStage * kRowStride;
   unsigned char* stages = smem + kFImg;                                          // [2][64 rows][kRowStride]
   uint2* qf = reinterpret_cast<uint2*>(stages + 2 * kStageBytes);                 // [KV][2 hf][4 u][32 lanes]
-  float* xbuf = reinterpret_cast<float*>(qf + KV * 2 * 4 * 32);                  // [2][4 rt][KV][16][8]
-  float4* advt = reinterpret_cast<float4*>(xbuf + 2 * kFStageTiles * KV * 16 * 8);   // [2 hf][4 i][4 u]
+  // partial scores of the non-finalising warps, [4 rt][KV][16][8]: written and read between the
+  // barrier at the top of a stage and the next one, so one buffer serves every stage
+  float* xbuf = reinterpret_cast<float*>(qf + KV * 2 * 4 * 32);
+  float4* advt = reinterpret_cast<float4*>(xbuf + kFStageTiles * KV * 16 * 8);   // [2 hf][4 i][4 u]
   float2* basep = reinterpret_cast<float2*>(advt + 32);                          // [16 warps][32]
   float* mred = reinterpret_cast<float*>(basep + kFWarps * 32);                  // [4 rt][KV][8]
 
@@ -383,7 +385,7 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
     const bool tile_live = kFull || rows_valid > 0;
     const bool valid0 = kFull || g < rows_valid, valid1 = kFull || g + 8 < rows_valid;
     const unsigned char* sb = stages + stage * kStageBytes;
-    float* xb = xbuf + ((stage * kFStageTiles + rt) * KV) * 16 * 8;
+    float* xb = xbuf + (rt * KV) * 16 * 8;
     float fin[kFin][4];
     if (tile_live) {
 #pragma unroll
@@ -848,7 +850,7 @@ commvq_status launch_fast_r(const AttendArgs& a, const void* q, commvq_dtype qt,
 size_t fast_keys_smem_bytes(int R, int KV) {
   const size_t row = static_cast<size_t>(KV) * R * 16 + 16;
   return kFImg + 2 * kFStage * row + static_cast<size_t>(KV) * 2 * 4 * 32 * 8 +
-         static_cast<size_t>(2) * kFStageTiles * KV * 16 * 8 * 4 + 32 * 16 + kFWarps * 32 * 8 +
+         static_cast<size_t>(kFStageTiles) * KV * 16 * 8 * 4 + 32 * 16 + kFWarps * 32 * 8 +
          static_cast<size_t>(kFStageTiles) * KV * 8 * 4;
 }
 
