@@ -2,7 +2,8 @@
 // Eq. 20 -- hard assignment, closed-form centroid update). The hard step takes g = 8, 16, 32
 // or 64 scalars per group (g = 64 is the pages' own setting); the soft step takes g = 8.
 //
-// Kernel 1 (grid: row chunks x groups): assigns every row of the chunk to its nearest
+// Kernel 1 (grid: row chunks x groups; 512-row chunks, 256 when that leaves fewer than two CTAs
+// per SM, e.g. a 4096-row fit): assigns every row of the chunk to its nearest
 // entry with the encoder's exact fp32 rule, then sums the assigned sub-vectors per entry
 // in fp64. Each entry's sum is taken by one thread over the chunk's rows in row order, so
 // the partial is independent of scheduling. Kernel 2 (grid: entries) adds the chunk
@@ -16,7 +17,8 @@
 namespace commvq {
 namespace {
 
-constexpr int kChunkRows = 512;                   // rows per CTA (4096 rows fill 128 CTAs)
+constexpr int kChunkRows = 512;                   // rows per CTA of the hard step, at most
+constexpr int64_t kFillCtas = 2 * 148;            // CTAs below which chunks halve (two per B200 SM)
 constexpr int kTile = 1024;                       // codebook entries staged per pass (g = 8)
 constexpr int kTileFloats = kTile * kG;           // 32 KB of entries per pass, any g
 constexpr int kMaxCodes = 4096;
@@ -27,6 +29,7 @@ constexpr int kSoftChunkRows = 256;               // rows per CTA of the soft st
 // entry) fp64 sums of g scalars, then 8 bytes (int32 counts of the hard step or fp64 weight
 // sums of the soft step), then per (chunk, group) fp64 SSE partials.
 struct EmLayout {
+  int chunk_rows;         // hard-step rows per chunk: 512, or 256 when 512 would leave SMs idle
   int64_t chunks;        // hard-step chunks
   int64_t soft_chunks;   // soft-step chunks
   size_t sums_off, counts_off, sse_off, total;
@@ -34,7 +37,8 @@ struct EmLayout {
 
 EmLayout em_layout(int64_t N, int G, int Nc, int g) {
   EmLayout L;
-  L.chunks = (N + kChunkRows - 1) / kChunkRows;
+  L.chunk_rows = ((N + kChunkRows - 1) / kChunkRows) * G >= kFillCtas ? kChunkRows : kChunkRows / 2;
+  L.chunks = (N + L.chunk_rows - 1) / L.chunk_rows;
   L.soft_chunks = (N + kSoftChunkRows - 1) / kSoftChunkRows;
   const int64_t cap = L.soft_chunks > L.chunks ? L.soft_chunks : L.chunks;
   L.sums_off = 0;
@@ -49,7 +53,8 @@ template <int GG>
 __global__ void __launch_bounds__(kThreads)
 em_assign_kernel(const float* __restrict__ rows, int64_t N, int d, int Nc,
                  const float* __restrict__ cb, void* __restrict__ codes_out, int code_bytes,
-                 double* __restrict__ psum, int32_t* __restrict__ pcnt, double* __restrict__ psse) {
+                 double* __restrict__ psum, int32_t* __restrict__ pcnt, double* __restrict__ psse,
+                 int chunk_rows) {
   constexpr int kRows = GG == 8 ? 2 : 1;
   constexpr int kSub = kThreads * kRows;          // rows assigned per pass
   constexpr int kTileE = kTileFloats / GG;        // entries staged per pass
@@ -60,8 +65,8 @@ em_assign_kernel(const float* __restrict__ rows, int64_t N, int d, int Nc,
   const int G = d / GG;
   const int j = blockIdx.y;
   const int64_t chunk = blockIdx.x;
-  const int64_t base = chunk * kChunkRows;
-  const int rows_here = static_cast<int>(min(static_cast<int64_t>(kChunkRows), N - base));
+  const int64_t base = chunk * chunk_rows;
+  const int rows_here = static_cast<int>(min(static_cast<int64_t>(chunk_rows), N - base));
   const float* sub_cb = cb + static_cast<int64_t>(j) * Nc * GG;
 
   for (int s0 = 0; s0 < rows_here; s0 += kSub) {
@@ -191,13 +196,28 @@ em_update_kernel(int64_t chunks, int G, int Nc, float* __restrict__ cb, const do
 #pragma unroll
       for (int k = 0; k < kG; ++k) acc[k] = 0.0;
       int64_t cnt = 0;
-      for (int64_t ch = 0; ch < chunks; ++ch) {
-        const int64_t at = ch * G * Nc + e;
-        const int32_t m = pcnt[at];
-        if (m == 0) continue;
-        cnt += m;
+      // four chunks' counts and sums loaded before any is used (the loads do not wait on one
+      // another), then added in chunk order, skipping chunks where no row chose the entry
+      for (int64_t ch0 = 0; ch0 < chunks; ch0 += 4) {
+        int32_t m[4];
+        double v[4][kG];
 #pragma unroll
-        for (int k = 0; k < kG; ++k) acc[k] += psum[at * GG + q * kG + k];
+        for (int u = 0; u < 4; ++u) {
+          m[u] = 0;
+          if (ch0 + u < chunks) {
+            const int64_t at = (ch0 + u) * G * Nc + e;
+            m[u] = pcnt[at];
+#pragma unroll
+            for (int k = 0; k < kG; ++k) v[u][k] = psum[at * GG + q * kG + k];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (m[u] == 0) continue;
+          cnt += m[u];
+#pragma unroll
+          for (int k = 0; k < kG; ++k) acc[k] += v[u][k];
+        }
       }
       if (cnt > 0) {
 #pragma unroll
@@ -369,7 +389,7 @@ commvq_status launch_em_hard(const commvq_config* cfg, const float* rows, int64_
   int32_t* pcnt = reinterpret_cast<int32_t*>(ws + L.counts_off);
   double* psse = reinterpret_cast<double*>(ws + L.sse_off);
   em_assign_kernel<GG><<<dim3(static_cast<unsigned>(L.chunks), G), kThreads, 0, st>>>(
-      rows, N, cfg->d, Nc, cb, codes_out, cfg->code_bytes, psum, pcnt, psse);
+      rows, N, cfg->d, Nc, cb, codes_out, cfg->code_bytes, psum, pcnt, psse, L.chunk_rows);
   const commvq_status rc = launch_status();
   if (rc != COMMVQ_OK) return rc;
   const unsigned g2 = static_cast<unsigned>((static_cast<int64_t>(G) * Nc + kThreads - 1) / kThreads);

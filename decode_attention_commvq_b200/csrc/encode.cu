@@ -33,6 +33,12 @@ struct EncodeJobs {
   EncodeJob<XT> job[2];
 };
 
+// Rows per thread: g = 8 takes two (independent distance chains for the packed scan, and one
+// shared-memory read of an entry pair serves both; four rows need ~160 registers and run slower),
+// larger groups one.
+template <int GG>
+constexpr int kEncodeRows = GG == 8 ? 2 : 1;
+
 // GG: scalars per group (8, 16, 32 or 64). Each thread encodes kRows rows of one group.
 template <typename XT, bool kTrack, int GG>
 __global__ void __launch_bounds__(kThreads)
@@ -42,7 +48,7 @@ encode_kernel(EncodeJobs<XT> jobs, int64_t n_rows, int d, int R, int n_codes, in
   const float* __restrict__ cb = jobs.job[blockIdx.z].cb;
   void* __restrict__ codes = jobs.job[blockIdx.z].codes;
   float* __restrict__ residual_out = jobs.job[blockIdx.z].residual_out;
-  constexpr int kRows = GG == 8 ? 2 : 1;
+  constexpr int kRows = kEncodeRows<GG>;
   constexpr int kTile = kTileFloats / GG;   // entries per pass
   __shared__ float4 tile[kTileFloats / 4];
   const int G = d / GG;
@@ -247,7 +253,7 @@ void launch_encode_g(const EncodeJobs<XT>& jobs, int n_jobs, int64_t n_rows, int
                                                                                  code_bytes, nullptr);
     return;
   }
-  const int64_t per_block = kThreads * (GG == 8 ? 2 : 1);
+  const int64_t per_block = kThreads * kEncodeRows<GG>;
   dim3 grid(static_cast<unsigned>((n_rows + per_block - 1) / per_block), d / GG, n_jobs);
   if (near_ties)
     encode_kernel<XT, true, GG><<<grid, kThreads, 0, s>>>(jobs, n_rows, d, R, n_codes, code_bytes, near_ties);

@@ -179,7 +179,12 @@ size_t commvq_attend_workspace_bytes(const commvq_config* cfg, int32_t B, int64_
  *             status leaves the workspace's prepared state unspecified: prepare it again.
  * options     nullable (defaults: AUTO algorithm, library-chosen splits, no flags). With
  *             COMMVQ_ATTEND_PREPARED the workspace's prepared state (see commvq_attend_prepare)
- *             is used as it stands; otherwise the call writes it first.
+ *             is used as it stands; otherwise the call writes it first. A prepared
+ *             decode-and-rotate call launches its attention kernel as a programmatic dependent
+ *             of the kernel before it on the stream, and that kernel reads q (and the prepared
+ *             state) before it waits: q must not be written by the immediately preceding
+ *             kernel on the stream (an event record or a copy in between, or a call without
+ *             the flag, orders it fully).
  * Shapes: d = 128, q_heads % kv_heads == 0, B >= 0 (B = 0 is a no-op), and per algorithm
  *   DECODE_MMA  g = 8, R <= 2, Nc' <= 256, kv_heads in {1, 2, 4, 8}, q_heads / kv_heads <= 8;
  *   TABLE       g = 8, R <= 4, Nc' <= 256;

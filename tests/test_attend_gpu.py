@@ -297,6 +297,31 @@ def test_prepared_workspace_is_identical(api, gpu, algo):
     assert api.workspace_error(ws) == 0
 
 
+def test_prepared_state_survives_a_longer_context(api, gpu, algo=2):
+    """The prepared state sits at fixed workspace offsets: prepared once at a short context,
+    it serves PREPARED decode steps at that length and at a longer one, where the split count,
+    and so the size of the per-split buffers, differ (1000 positions: 63 splits; 3000: 148)."""
+    w, kc, vc, kcb, vcb = _encoded_inputs(synth.WORKLOADS[1], T=3000)
+    cfg = _cfg(api, w)
+    kcg, vcg = _codes_np_to_gpu(kc, gpu), _codes_np_to_gpu(vc, gpu)
+    kcbt, vcbt = torch.from_numpy(kcb).to(gpu), torch.from_numpy(vcb).to(gpu)
+    ws = api.attend_workspace(cfg, 1, 3000, gpu, algo)
+    api.attend_prepare(cfg, 1, 1000, kcbt, vcbt, ws, algo=algo)
+    q_np = synth.queries(w)
+    q = to_torch_q(q_np, w.q_dtype, gpu)
+    for T in (1000, 3000, 1000):
+        offs = np.array([0, T], dtype=np.int64)
+        offsets = torch.from_numpy(offs).to(gpu)
+        out_p, _ = api.attend_decode(cfg, q, kcg[:T], vcg[:T], offsets, T, kcbt, vcbt, workspace=ws,
+                                     algo=algo, prepared=True)
+        out_u, _ = api.attend_decode(cfg, q, kcg[:T], vcg[:T], offsets, T, kcbt, vcbt, algo=algo)
+        torch.cuda.synchronize()
+        assert torch.equal(out_p, out_u), T
+        ref, _ = O.attend_codes(q_as_f64(w, q_np), kc[:T], vc[:T], offs, kcb, vcb, w.rope_base)
+        assert rel_err(out_p.cpu().numpy(), ref) <= tol_for(w)
+    assert api.workspace_error(ws) == 0
+
+
 def test_many_queries_within_bound(api, gpu):
     """The bf16 bound on 6 seeded queries x 32 heads (192 heads) over 3000 encoded positions of
     the 2-bit layer, decode-and-rotate path: the tail of the error distribution, not one
