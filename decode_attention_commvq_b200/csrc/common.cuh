@@ -298,14 +298,18 @@ __device__ __forceinline__ void load_phasor(float4 v, f32x2& c, f32x2& s) {
 }
 
 // Nearest-entry update with a distance already computed by the encoder's fp32 rule (the
-// comparison half of nearest_step).
+// comparison half of nearest_step). A distance is a sum of squares from +0, so it is >= +0 (or
+// NaN for non-finite input); on such values the fp32 order is the unsigned order of the bit
+// patterns, with NaN above +inf (never taken, as in the fp32 comparison). The comparisons run
+// as integer instructions, leaving the fp32 pipe to the distance arithmetic.
 template <bool kTrack>
 __device__ __forceinline__ void nearest_take(Nearest& n, float dist, int c) {
-  if (dist < n.best) {
+  const uint32_t d = __float_as_uint(dist);
+  if (d < __float_as_uint(n.best)) {
     if (kTrack) n.second = n.best;
     n.best = dist;
     n.idx = c;
-  } else if (kTrack && dist < n.second) {
+  } else if (kTrack && d < __float_as_uint(n.second)) {
     n.second = dist;
   }
 }
