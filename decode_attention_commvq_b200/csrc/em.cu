@@ -48,14 +48,15 @@ EmLayout em_layout(int64_t N, int G, int Nc, int g) {
   return L;
 }
 
-// GG: scalars per group (8, 16, 32 or 64); 2 rows per thread and pass for GG = 8, else 1.
-template <int GG>
+// GG: scalars per group (8, 16, 32 or 64); kRowsT rows per thread and pass (2 for GG = 8 with
+// 512-row chunks, else 1, so that a 256-row chunk keeps every thread busy).
+template <int GG, int kRowsT>
 __global__ void __launch_bounds__(kThreads)
 em_assign_kernel(const float* __restrict__ rows, int64_t N, int d, int Nc,
                  const float* __restrict__ cb, void* __restrict__ codes_out, int code_bytes,
                  double* __restrict__ psum, int32_t* __restrict__ pcnt, double* __restrict__ psse,
                  int chunk_rows) {
-  constexpr int kRows = GG == 8 ? 2 : 1;
+  constexpr int kRows = kRowsT;
   constexpr int kSub = kThreads * kRows;          // rows assigned per pass
   constexpr int kTileE = kTileFloats / GG;        // entries staged per pass
   __shared__ float4 tile[kTileFloats / 4];
@@ -396,8 +397,13 @@ commvq_status launch_em_hard(const commvq_config* cfg, const float* rows, int64_
   double* psum = reinterpret_cast<double*>(ws + L.sums_off);
   int32_t* pcnt = reinterpret_cast<int32_t*>(ws + L.counts_off);
   double* psse = reinterpret_cast<double*>(ws + L.sse_off);
-  em_assign_kernel<GG><<<dim3(static_cast<unsigned>(L.chunks), G), kThreads, 0, st>>>(
-      rows, N, cfg->d, Nc, cb, codes_out, cfg->code_bytes, psum, pcnt, psse, L.chunk_rows);
+  const dim3 grid(static_cast<unsigned>(L.chunks), G);
+  if (GG == kG && L.chunk_rows == kChunkRows)
+    em_assign_kernel<GG, 2><<<grid, kThreads, 0, st>>>(rows, N, cfg->d, Nc, cb, codes_out, cfg->code_bytes, psum,
+                                                        pcnt, psse, L.chunk_rows);
+  else
+    em_assign_kernel<GG, 1><<<grid, kThreads, 0, st>>>(rows, N, cfg->d, Nc, cb, codes_out, cfg->code_bytes, psum,
+                                                        pcnt, psse, L.chunk_rows);
   const commvq_status rc = launch_status();
   if (rc != COMMVQ_OK) return rc;
   const unsigned g2 = static_cast<unsigned>((static_cast<int64_t>(G) * Nc + kThreads - 1) / kThreads);
