@@ -162,15 +162,15 @@ __device__ __forceinline__ void fast_split(const AttendArgs& a, int b, int s, in
   t_end = min(Tb, t_begin + per);
 }
 
-// Copy the code records of positions t0 .. t0 + kFStage - 1 (those before t_end) into a stage whose
-// rows are kRec + 16 bytes apart (consecutive rows start in different bank groups).
+// The rows t0 .. t0 + 15 (those before t_end) of one 16-position row tile, copied by that tile's
+// 128 threads (lt: the thread's index among them) into the tile's place of a stage.
 template <int kRec>
-__device__ __forceinline__ void fast_issue_stage(unsigned char* dst, const uint8_t* codes, int64_t row0, int64_t t0,
-                                                 int64_t t_end) {
+__device__ __forceinline__ void fast_issue_tile(unsigned char* dst, const uint8_t* codes, int64_t row0, int64_t t0,
+                                                int64_t t_end, int lt) {
   constexpr int kPieces = kRec / 16;
-  const int n = static_cast<int>(min(static_cast<int64_t>(kFStage), t_end - t0));
+  const int n = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(kFTile), t_end - t0)));
   const uint8_t* src = codes + (row0 + t0) * kRec;
-  for (int p = threadIdx.x; p < n * kPieces; p += kFThreads) {
+  for (int p = lt; p < n * kPieces; p += 4 * 32) {
     const int row = p / kPieces, piece = p - row * kPieces;
     cp_async16(dst + row * (kRec + 16) + piece * 16, src + p * 16);
   }
@@ -303,7 +303,8 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
   pdl_wait();
   pdl_trigger();   // the merge kernel may be scheduled; it waits for this grid
 
-  fast_issue_stage<kRec>(stages, a.k_codes, row0, t_begin, t_end);
+  // each row tile's four warps copy and wait for their own rows (a named barrier per tile)
+  fast_issue_tile<kRec>(stages + kFTile * rt * kRowStride, a.k_codes, row0, t_begin + kFTile * rt, t_end, tid & 127);
   cp_async_commit();
 
   // Per-thread constants. Rows of the thread in a stage, code-word offsets (round order by row
@@ -493,12 +494,16 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
     }
   };
 
+  __syncthreads();   // the query fragments and phasor tables of the prologue are in place
   int stage = 0, it = 0;
   for (int64_t t0 = t_begin; t0 < t_end; t0 += kFStage, stage ^= 1, ++it) {
     cp_async_wait<0>();
-    __syncthreads();   // this stage's codes (and, the first time, the image) are in shared memory,
-                       // and every warp is done with the previous stage's buffer
-    if (t0 + kFStage < t_end) fast_issue_stage<kRec>(stages + (stage ^ 1) * kStageBytes, a.k_codes, row0, t0 + kFStage, t_end);
+    // this stage's rows of the row tile are in shared memory, and the tile's four warps are done
+    // with its previous buffer (named barrier 9 + rt, 128 threads; the warps of other tiles run on)
+    asm volatile("bar.sync %0, 128;\n" ::"r"(9 + rt) : "memory");
+    if (t0 + kFStage < t_end)
+      fast_issue_tile<kRec>(stages + (stage ^ 1) * kStageBytes + kFTile * rt * kRowStride, a.k_codes, row0,
+                            t0 + kFStage + kFTile * rt, t_end, tid & 127);
     cp_async_commit();
     if (it > 0) {
       if (it % kFRefresh == 0) {
