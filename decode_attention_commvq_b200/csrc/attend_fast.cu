@@ -587,29 +587,35 @@ __device__ __forceinline__ void values_phase(const AttendArgs& a, unsigned char*
   const int64_t n_tiles = (a.max_T + kFTile - 1) / kFTile;
   const int tile_floats = a.q_heads * kFTile;                  // one tile of the score buffer
   const int score_stage_bytes = kTiles * tile_floats * 4;
-  auto issue_codes = [&](unsigned char* dst, int64_t t0) {
-    constexpr int kPieces = kRec / 16;
-    const int n = static_cast<int>(min(static_cast<int64_t>(kStageT), t_end - t0));
-    const uint8_t* src = a.v_codes + (row0 + t0) * kRec;
-    for (int p = tid; p < n * kPieces; p += kFThreads) {
-      const int row = p / kPieces, piece = p - row * kPieces;
-      cp_async16(dst + row * kRowStride + piece * 16, src + p * 16);
-    }
-  };
-  auto issue_scores = [&](unsigned char* dst, int64_t t0) {   // whole tiles, contiguous
-    const int64_t tau0 = t0 / kFTile;
-    const int64_t tau1 = (min(t_end, t0 + kStageT) + kFTile - 1) / kFTile;
-    const int pieces = static_cast<int>(tau1 - tau0) * (tile_floats / 4);
-    const float* src = a.scores + (static_cast<int64_t>(b) * n_tiles + tau0) * tile_floats;
-    for (int p = tid; p < pieces; p += kFThreads) cp_async16_ca(dst + p * 16, src + 4 * p);
-  };
-
   // the value image replaces the key image: every read of it is before the caller's barrier, and
   // the proxy fence orders those reads before the bulk copies' writes
   if (tid == 0) fence_async_smem();
   image_copy_issue(smem, a.v_img, Nc, ibar);
-  issue_codes(stages, t_begin);
-  issue_scores(sstage, t_begin);   // written by this CTA's keys phase before the barrier
+  // The warps with the same sub (one per KV head) share their tiles' rows and score tiles: they
+  // copy and wait for those alone (named barrier 1 + sub), so the WPK groups run independently.
+  constexpr int kGroupThreads = KV * 32;
+  const int lt = kv * 32 + lane;   // the thread's index in its group
+  auto issue_group = [&](unsigned char* cdst, unsigned char* sdst, int64_t t0) {
+    constexpr int kPieces = kRec / 16;
+#pragma unroll
+    for (int ti = 0; ti < kTiles / WPK; ++ti) {
+      const int tile = sub + ti * WPK;
+      const int64_t tt0 = t0 + tile * kFTile;
+      const int n = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(kFTile), t_end - tt0)));
+      const uint8_t* src = a.v_codes + (row0 + tt0) * kRec;
+      unsigned char* d = cdst + tile * kFTile * kRowStride;
+      for (int q = lt; q < n * kPieces; q += kGroupThreads) {
+        const int row = q / kPieces, piece = q - row * kPieces;
+        cp_async16(d + row * kRowStride + piece * 16, src + q * 16);
+      }
+      if (n > 0) {   // the tile's scores, written by this CTA's keys phase before the barrier
+        const float* ss = a.scores + (static_cast<int64_t>(b) * n_tiles + tt0 / kFTile) * tile_floats;
+        unsigned char* sd = sdst + tile * tile_floats * 4;
+        for (int q = lt; q < tile_floats / 4; q += kGroupThreads) cp_async16_ca(sd + q * 16, ss + 4 * q);
+      }
+    }
+  };
+  issue_group(stages, sstage, t_begin);
   cp_async_commit();
 
   // head column g of this warp's KV head; a column past G reads column G - 1 (finite weights in an
@@ -689,11 +695,10 @@ __device__ __forceinline__ void values_phase(const AttendArgs& a, unsigned char*
   int stage = 0;
   for (int64_t t0 = t_begin; t0 < t_end; t0 += kStageT, stage ^= 1) {
     cp_async_wait<0>();
-    __syncthreads();   // this stage's codes and scores are in; the other buffers are free
-    if (t0 + kStageT < t_end) {
-      issue_codes(stages + (stage ^ 1) * kStageBytes, t0 + kStageT);
-      issue_scores(sstage + (stage ^ 1) * score_stage_bytes, t0 + kStageT);
-    }
+    // the group's codes and scores of this stage are in; its warps are done with the other buffers
+    asm volatile("bar.sync %0, %1;\n" ::"r"(1 + sub), "r"(kGroupThreads) : "memory");
+    if (t0 + kStageT < t_end)
+      issue_group(stages + (stage ^ 1) * kStageBytes, sstage + (stage ^ 1) * score_stage_bytes, t0 + kStageT);
     cp_async_commit();
     const unsigned char* sb = stages + stage * kStageBytes;
     const float* ssc = reinterpret_cast<const float*>(sstage + stage * score_stage_bytes);
