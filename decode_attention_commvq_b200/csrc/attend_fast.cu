@@ -545,6 +545,11 @@ __device__ __forceinline__ void keys_phase(const AttendArgs& a, const QT* __rest
     }
   }
   __syncthreads();
+  // every warp is done with the key image: the value image's bulk copies start now, under the
+  // rest of this phase and the values phase's set-up (the proxy fence orders the image reads
+  // before the copies' writes)
+  if (tid == 0) fence_async_smem();
+  image_copy_issue(smem, a.v_img, Nc, ibar);
   // [KV][8] (columns past G: the max of their zero scores)
   for (int e = tid; e < KV * 8; e += kFThreads) {
     float m = -INFINITY;
@@ -587,10 +592,7 @@ __device__ __forceinline__ void values_phase(const AttendArgs& a, unsigned char*
   const int64_t n_tiles = (a.max_T + kFTile - 1) / kFTile;
   const int tile_floats = a.q_heads * kFTile;                  // one tile of the score buffer
   const int score_stage_bytes = kTiles * tile_floats * 4;
-  // the value image replaces the key image: every read of it is before the caller's barrier, and
-  // the proxy fence orders those reads before the bulk copies' writes
-  if (tid == 0) fence_async_smem();
-  image_copy_issue(smem, a.v_img, Nc, ibar);
+  // the value image's bulk copies were issued at the end of the keys phase
   // The warps with the same sub (one per KV head) share their tiles' rows and score tiles: they
   // copy and wait for those alone (named barrier 1 + sub), so the WPK groups run independently.
   constexpr int kGroupThreads = KV * 32;
