@@ -375,7 +375,7 @@ extern "C" commvq_status commvq_attend_decode(const commvq_config* cfg, const vo
       return COMMVQ_ERR_CUDA;
   }
   if (rc != COMMVQ_OK) return rc;
-  return launch_combine(a, partial_slots(cfg, run, S), st);
+  return launch_combine(a, partial_slots(cfg, run, S), st, fast && static_cast<int64_t>(S) * B >= di.sms);
 }
 
 extern "C" commvq_status commvq_attend_prepare(const commvq_config* cfg, int32_t B, int64_t max_T,
@@ -458,8 +458,23 @@ int attend_mma_setup(const commvq_config* cfg, int B, int64_t max_T, unsigned ch
 }  // namespace commvq
 
 namespace commvq {
-commvq_status launch_combine(const AttendArgs& a, int S, cudaStream_t st) {
-  if (launch_dependent(combine_kernel, dim3(a.B * a.q_heads, kCombineQuarters), dim3(kCombineThreads), 0, st, a,
+// one_per_sm: the kernel before has one CTA on every SM and lets this grid launch early. Its CTAs
+// then take SMs as that kernel's CTAs leave; left alone, the scheduler stacks up to eight of them
+// on each of the first SMs to free up, where they share one SM's load path for every split's
+// partials. A dynamic shared-memory request of over half an SM's capacity (unused by the kernel)
+// leaves room for one merge CTA per SM, so they spread out. When the kernel before leaves SMs
+// idle, the CTAs go there at once and stacking them costs less than waiting for SMs.
+commvq_status launch_combine(const AttendArgs& a, int S, cudaStream_t st, bool one_per_sm) {
+  size_t dyn = 0;
+  if (one_per_sm) {
+    const DeviceInfo di = current_device_info();
+    if (di.device < 0) return COMMVQ_ERR_CUDA;
+    dyn = di.smem_optin / 2 + 4096;
+    if (cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn)) !=
+        cudaSuccess)
+      return COMMVQ_ERR_CUDA;
+  }
+  if (launch_dependent(combine_kernel, dim3(a.B * a.q_heads, kCombineQuarters), dim3(kCombineThreads), dyn, st, a,
                        S) != cudaSuccess)
     return COMMVQ_ERR_CUDA;
   return launch_status();

@@ -68,7 +68,7 @@ __host__ __device__ inline int64_t score_slot(int64_t b, int64_t t, int kv, int 
 }
 commvq_status launch_attend_table(const AttendArgs& a, const void* q, commvq_dtype qt, int splits,
                                   cudaStream_t st);
-commvq_status launch_combine(const AttendArgs& a, int splits, cudaStream_t st);
+commvq_status launch_combine(const AttendArgs& a, int splits, cudaStream_t st, bool one_per_sm = false);
 // The fast decode-and-rotate kernels (attend_fast.cu): KV heads in {2, 4, 8}, up to 8 query heads
 // per KV head, R <= 2, Nc' <= 256, g = 8. Their prepared state is 128 KB per codebook image, RoPE
 // tables theta [64] fp64, offset rows [64][64] (cos, sin) and the 64-position advance [64].
