@@ -459,9 +459,9 @@ int attend_mma_setup(const commvq_config* cfg, int B, int64_t max_T, unsigned ch
 
 namespace commvq {
 // one_per_sm: the kernel before has one CTA on every SM and lets this grid launch early. Its CTAs
-// then take SMs as that kernel's CTAs leave; left alone, the scheduler may stack several of them
-// (up to eight by thread count) on each of the first SMs to free up, where they share one SM's
-// load path for every split's partials (a 32K context's merge ran 0.9 us faster spread out). A dynamic shared-memory request of over half an SM's capacity (unused by the kernel)
+// then take SMs as that kernel's CTAs leave; left alone, the scheduler stacks them on the first
+// SMs to free up (at a 32K context: 128 CTAs on 46 SMs, three on most), where they share those
+// SMs' load paths for every split's partials (spread out, that merge ran 0.9 us faster). A dynamic shared-memory request of over half an SM's capacity (unused by the kernel)
 // leaves room for one merge CTA per SM, so they spread out. When the kernel before leaves SMs
 // idle, the CTAs go there at once and stacking them costs less than waiting for SMs.
 commvq_status launch_combine(const AttendArgs& a, int S, cudaStream_t st, bool one_per_sm) {
