@@ -175,8 +175,11 @@ template <typename XT, bool kTrack, int GG>
 __global__ void __launch_bounds__(32 * kWarpUnitsPerBlock)
 encode_warp_kernel(EncodeJobs<XT> jobs, int64_t n_rows, int d, int R, int n_codes, int code_bytes,
                    unsigned long long* __restrict__ near_ties) {
-  // a following kernel launched as a programmatic dependent (a decode step's attention) may start
-  // its own set-up now; it waits for this grid before it reads the codes
+  // launched as a programmatic dependent: the launch overlaps the kernel before, and the wait
+  // gives it that kernel's writes (the rows, a step's input copy) before anything is read or
+  // written. Then a following dependent (a decode step's attention) may start its own set-up; it
+  // waits for this grid before it reads the codes.
+  pdl_wait();
   pdl_trigger();
   const XT* __restrict__ x = jobs.job[blockIdx.z].x;
   const float* __restrict__ cb = jobs.job[blockIdx.z].cb;
@@ -246,11 +249,11 @@ void launch_encode_g(const EncodeJobs<XT>& jobs, int n_jobs, int64_t n_rows, int
     const unsigned blocks = static_cast<unsigned>((units + kWarpUnitsPerBlock - 1) / kWarpUnitsPerBlock);
     const dim3 grid(blocks, 1, n_jobs);
     if (near_ties)
-      encode_warp_kernel<XT, true, GG><<<grid, 32 * kWarpUnitsPerBlock, 0, s>>>(jobs, n_rows, d, R, n_codes,
-                                                                                code_bytes, near_ties);
+      (void)launch_dependent(encode_warp_kernel<XT, true, GG>, grid, dim3(32 * kWarpUnitsPerBlock), 0, s, jobs,
+                             n_rows, d, R, n_codes, code_bytes, near_ties);
     else
-      encode_warp_kernel<XT, false, GG><<<grid, 32 * kWarpUnitsPerBlock, 0, s>>>(jobs, n_rows, d, R, n_codes,
-                                                                                 code_bytes, nullptr);
+      (void)launch_dependent(encode_warp_kernel<XT, false, GG>, grid, dim3(32 * kWarpUnitsPerBlock), 0, s, jobs,
+                             n_rows, d, R, n_codes, code_bytes, static_cast<unsigned long long*>(nullptr));
     return;
   }
   const int64_t per_block = kThreads * kEncodeRows<GG>;

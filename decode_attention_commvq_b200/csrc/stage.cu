@@ -15,7 +15,11 @@ constexpr int kCopyMaxBlocks = 148;
 __global__ void __launch_bounds__(kCopyThreads) copy_kernel(uint4* __restrict__ dst, const uint4* __restrict__ src,
                                                             int64_t n16, uint8_t* __restrict__ dst_tail,
                                                             const uint8_t* __restrict__ src_tail, int tail) {
-  pdl_trigger();   // a dependent kernel may start its own set-up; it waits for this grid
+  // launched as a programmatic dependent: the launch overlaps the kernel before, and the wait
+  // gives it that kernel's writes (ordinary stream order) before any load or store; the kernel
+  // after it may then start its own set-up
+  pdl_wait();
+  pdl_trigger();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kCopyThreads;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * kCopyThreads + threadIdx.x; i < n16; i += stride)
     dst[i] = src[i];
@@ -40,8 +44,10 @@ extern "C" commvq_status commvq_copy_async(void* dst, const void* src, size_t by
   int64_t blocks = (n16 + kCopyThreads - 1) / kCopyThreads;
   if (blocks < 1) blocks = 1;
   if (blocks > kCopyMaxBlocks) blocks = kCopyMaxBlocks;
-  copy_kernel<<<static_cast<unsigned>(blocks), kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint4*>(dst), static_cast<const uint4*>(src), n16, static_cast<uint8_t*>(dst) + n16 * 16,
-      static_cast<const uint8_t*>(src) + n16 * 16, tail);
+  if (launch_dependent(copy_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kCopyThreads), 0,
+                       static_cast<cudaStream_t>(stream), static_cast<uint4*>(dst), static_cast<const uint4*>(src),
+                       n16, static_cast<uint8_t*>(dst) + n16 * 16, static_cast<const uint8_t*>(src) + n16 * 16,
+                       tail) != cudaSuccess)
+    return COMMVQ_ERR_CUDA;
   return launch_status();
 }

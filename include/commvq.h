@@ -131,9 +131,12 @@ commvq_status commvq_encode(const commvq_config* cfg, const void* x, commvq_dtyp
  * k_codebook, v_codebook  [R, d/g, Nc', g] float32, 16-byte aligned.
  * k_codes, v_codes  [n_tokens, kv_heads, R, d/g] out, code_bytes per element.
  * near_ties         nullable device counter; both tensors' near-tie decisions are ADDED to it.
- * When the next kernel on the stream is launched as a programmatic dependent (the attention of a
- * decode step with COMMVQ_ATTEND_PREPARED), it may start its set-up while this encode runs; it
- * reads the codes only after the encode has finished. Limits and errors as commvq_encode. */
+ * A small encode (up to 4096 rows x groups, e.g. a decode step's new position) is launched as a
+ * programmatic dependent of the kernel before it on the stream, so that its launch overlaps that
+ * kernel, and waits for that kernel's completion before it reads or writes anything: ordinary
+ * stream order. Only then may a following programmatic dependent (the attention of a decode step
+ * with COMMVQ_ATTEND_PREPARED) start its set-up; that kernel reads the codes only after the
+ * encode has finished. Limits and errors as commvq_encode. */
 commvq_status commvq_encode_kv(const commvq_config* cfg, const void* k_x, const void* v_x,
                                commvq_dtype x_dtype, int64_t n_tokens, const float* k_codebook,
                                const float* v_codebook, void* k_codes, void* v_codes,
@@ -395,8 +398,11 @@ commvq_status commvq_workspace_error(const void* workspace, int32_t* device_erro
  * per-step transfers of a decode loop (the query and the new position's K/V rows in, the output
  * out), where a copy-engine transfer inside a CUDA graph costs more in scheduling than the bytes.
  * Both pointers 16-byte aligned, ranges not overlapping (else COMMVQ_ERR_INVALID_ARG); bytes = 0
- * is a no-op. The caller owns both buffers. Not part of the method: plumbing for the end-to-end
- * step of a decode loop. */
+ * is a no-op. The caller owns both buffers. The kernel is launched as a programmatic dependent of
+ * the kernel before it on the stream (its launch overlaps that kernel) and waits for that
+ * kernel's completion before its first load or store, so it is ordered like any stream operation;
+ * a following programmatic dependent may start its set-up once every block has passed that wait.
+ * Not part of the method: plumbing for the end-to-end step of a decode loop. */
 commvq_status commvq_copy_async(void* dst, const void* src, size_t bytes, void* stream);
 
 /* Static description of a status code. */
