@@ -164,15 +164,28 @@ encode_kernel(EncodeJobs<XT> jobs, int64_t n_rows, int d, int R, int n_codes, in
   }
 }
 
-// Few rows (a decode step's new position): one warp per (row, group). Lane l scans entries
-// l, l+32, ... with the same fp32 distance rule (entries read through L1/L2); the warp then
-// merges (best, index, second best) by shuffles: the smallest distance wins, ties go to the
-// lowest entry, and the second best is the second smallest distance overall -- exactly what the
-// in-order scan of encode_kernel produces, so codes and near-tie counts are the same.
-constexpr int kWarpUnitsPerBlock = 8;
+// Few rows (a decode step's new position): kWarpsPerUnit warps per (row, group), so that each lane
+// scans only a few entries and a round costs one round trip of entry loads. Warp p of a unit takes
+// entries p*32 + lane, p*32 + lane + 128, ... in increasing order with the same fp32 distance rule
+// (entries read through L1/L2); each warp merges (best, index, second best) over its lanes by
+// shuffles, and the unit's warps then merge their four results through shared memory. The merge
+// is exact in any order (the smallest distance wins, ties go to the lowest entry, the second best
+// is the second smallest distance overall): what the in-order scan of encode_kernel produces, so
+// codes and near-tie counts are the same.
+constexpr int kWarpsPerUnit = 4;
+constexpr int kWarpUnitsPerBlock = 2;   // 8 warps per block
+
+__device__ __forceinline__ void nearest_merge(Nearest& n, float ob, int oi, float os) {
+  const float hi = fmaxf(n.best, ob);
+  if (ob < n.best || (ob == n.best && oi < n.idx)) {
+    n.best = ob;
+    n.idx = oi;
+  }
+  n.second = fminf(hi, fminf(n.second, os));
+}
 
 template <typename XT, bool kTrack, int GG>
-__global__ void __launch_bounds__(32 * kWarpUnitsPerBlock)
+__global__ void __launch_bounds__(32 * kWarpsPerUnit * kWarpUnitsPerBlock)
 encode_warp_kernel(EncodeJobs<XT> jobs, int64_t n_rows, int d, int R, int n_codes, int code_bytes,
                    unsigned long long* __restrict__ near_ties) {
   // launched as a programmatic dependent: the launch overlaps the kernel before, and the wait
@@ -181,21 +194,31 @@ encode_warp_kernel(EncodeJobs<XT> jobs, int64_t n_rows, int d, int R, int n_code
   // waits for this grid before it reads the codes.
   pdl_wait();
   pdl_trigger();
+  __shared__ float m_best[kWarpUnitsPerBlock][kWarpsPerUnit];
+  __shared__ float m_second[kWarpUnitsPerBlock][kWarpsPerUnit];
+  __shared__ int m_idx[kWarpUnitsPerBlock][kWarpsPerUnit];
   const XT* __restrict__ x = jobs.job[blockIdx.z].x;
   const float* __restrict__ cb = jobs.job[blockIdx.z].cb;
   void* __restrict__ codes = jobs.job[blockIdx.z].codes;
   float* __restrict__ residual_out = jobs.job[blockIdx.z].residual_out;
   const int G = d / GG;
-  const int lane = threadIdx.x & 31;
-  const int64_t unit = static_cast<int64_t>(blockIdx.x) * kWarpUnitsPerBlock + (threadIdx.x >> 5);
-  if (unit >= n_rows * G) return;   // the whole warp leaves together
-  const int64_t n = unit / G;
-  const int j = static_cast<int>(unit - n * G);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ul = warp / kWarpsPerUnit, part = warp % kWarpsPerUnit;
+  const int64_t unit = static_cast<int64_t>(blockIdx.x) * kWarpUnitsPerBlock + ul;
+  const bool valid = unit < n_rows * G;   // every warp stays for the block barriers
+  const int64_t n = valid ? unit / G : 0;
+  const int j = valid ? static_cast<int>(unit - n * G) : 0;
+  const bool leader = valid && part == 0 && lane == 0;
   float res[GG];
 #pragma unroll
   for (int q = 0; q < GG / kG; ++q) {
     float v[kG];
-    load_row8(x + n * d + j * GG + q * kG, v);
+    if (valid) {
+      load_row8(x + n * d + j * GG + q * kG, v);
+    } else {
+#pragma unroll
+      for (int k = 0; k < kG; ++k) v[k] = 0.0f;
+    }
 #pragma unroll
     for (int k = 0; k < kG; ++k) res[q * kG + k] = v[k];
   }
@@ -204,38 +227,49 @@ encode_warp_kernel(EncodeJobs<XT> jobs, int64_t n_rows, int d, int R, int n_code
     const float* sub = cb + (static_cast<int64_t>(r) * G + j) * n_codes * GG;
     Nearest best;
     nearest_init(best);
-    for (int c = lane; c < n_codes; c += 32)
-      nearest_step_g<GG, kTrack>(best, res, reinterpret_cast<const float4*>(sub + static_cast<int64_t>(c) * GG), c);
+    if (valid)
+      for (int c = part * 32 + lane; c < n_codes; c += 32 * kWarpsPerUnit)
+        nearest_step_g<GG, kTrack>(best, res, reinterpret_cast<const float4*>(sub + static_cast<int64_t>(c) * GG), c);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float ob = __shfl_xor_sync(0xffffffffu, best.best, o);
       const int oi = __shfl_xor_sync(0xffffffffu, best.idx, o);
       const float os = __shfl_xor_sync(0xffffffffu, best.second, o);
-      const float hi = fmaxf(best.best, ob);
-      if (ob < best.best || (ob == best.best && oi < best.idx)) {
-        best.best = ob;
-        best.idx = oi;
-      }
-      best.second = fminf(hi, fminf(best.second, os));
+      nearest_merge(best, ob, oi, os);
     }
     if (lane == 0) {
-      if (kTrack) ties += near_tie(best, n_codes) ? 1u : 0u;
-      store_code(codes, (n * R + r) * G + j, best.idx, code_bytes);
+      m_best[ul][part] = best.best;
+      m_second[ul][part] = best.second;
+      m_idx[ul][part] = best.idx;
     }
+    __syncthreads();
+    Nearest u;
+    u.best = m_best[ul][0];
+    u.second = m_second[ul][0];
+    u.idx = m_idx[ul][0];
 #pragma unroll
-    for (int q = 0; q < GG / kG; ++q) {
-      float w[kG];
-      load_row8(sub + static_cast<int64_t>(best.idx) * GG + q * kG, w);
+    for (int p = 1; p < kWarpsPerUnit; ++p) nearest_merge(u, m_best[ul][p], m_idx[ul][p], m_second[ul][p]);
+    __syncthreads();   // the slots are written again in the next round
+    if (leader) {
+      if (kTrack) ties += near_tie(u, n_codes) ? 1u : 0u;
+      store_code(codes, (n * R + r) * G + j, u.idx, code_bytes);
+    }
+    if (valid) {
 #pragma unroll
-      for (int k = 0; k < kG; ++k) res[q * kG + k] = __fsub_rn(res[q * kG + k], w[k]);
+      for (int q = 0; q < GG / kG; ++q) {
+        float w[kG];
+        load_row8(sub + static_cast<int64_t>(u.idx) * GG + q * kG, w);
+#pragma unroll
+        for (int k = 0; k < kG; ++k) res[q * kG + k] = __fsub_rn(res[q * kG + k], w[k]);
+      }
     }
   }
-  if (residual_out && lane == 0) {
+  if (residual_out && leader) {
     float4* dst = reinterpret_cast<float4*>(residual_out + n * d + j * GG);
 #pragma unroll
     for (int q = 0; q < GG / 4; ++q) dst[q] = make_float4(res[4 * q], res[4 * q + 1], res[4 * q + 2], res[4 * q + 3]);
   }
-  if (kTrack && lane == 0 && ties) atomicAdd(near_ties, static_cast<unsigned long long>(ties));
+  if (kTrack && leader && ties) atomicAdd(near_ties, static_cast<unsigned long long>(ties));
 }
 
 // Row counts up to this many (row, group) units take the warp-per-unit kernel.
@@ -248,12 +282,13 @@ void launch_encode_g(const EncodeJobs<XT>& jobs, int n_jobs, int64_t n_rows, int
   if (units <= kWarpEncodeMaxUnits) {
     const unsigned blocks = static_cast<unsigned>((units + kWarpUnitsPerBlock - 1) / kWarpUnitsPerBlock);
     const dim3 grid(blocks, 1, n_jobs);
+    const dim3 block(32 * kWarpsPerUnit * kWarpUnitsPerBlock);
     if (near_ties)
-      (void)launch_dependent(encode_warp_kernel<XT, true, GG>, grid, dim3(32 * kWarpUnitsPerBlock), 0, s, jobs,
-                             n_rows, d, R, n_codes, code_bytes, near_ties);
+      (void)launch_dependent(encode_warp_kernel<XT, true, GG>, grid, block, 0, s, jobs, n_rows, d, R, n_codes,
+                             code_bytes, near_ties);
     else
-      (void)launch_dependent(encode_warp_kernel<XT, false, GG>, grid, dim3(32 * kWarpUnitsPerBlock), 0, s, jobs,
-                             n_rows, d, R, n_codes, code_bytes, static_cast<unsigned long long*>(nullptr));
+      (void)launch_dependent(encode_warp_kernel<XT, false, GG>, grid, block, 0, s, jobs, n_rows, d, R, n_codes,
+                             code_bytes, static_cast<unsigned long long*>(nullptr));
     return;
   }
   const int64_t per_block = kThreads * kEncodeRows<GG>;
