@@ -118,7 +118,8 @@ typedef struct {
  *          after the last round (what a further round, or the next round of a codebook
  *          fit, would encode).
  * Supports g in {8, 16, 32, 64}, d % g == 0, 1 <= Nc' <= 65536, 1 <= R <= 32. n_tokens = 0 is
- * a no-op. */
+ * a no-op. A small encode (up to 4096 rows x groups) runs as described under commvq_encode_kv:
+ * a programmatic dependent launch that waits for the kernel before it first (stream order). */
 commvq_status commvq_encode(const commvq_config* cfg, const void* x, commvq_dtype x_dtype,
                             int64_t n_tokens, const float* codebook, void* codes,
                             unsigned long long* near_ties, float* residual_out, void* stream);
